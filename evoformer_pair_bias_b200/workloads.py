@@ -1,0 +1,190 @@
+"""Seeded synthetic workloads for Evoformer pair-bias attention.
+
+This module only draws random inputs and arranges them in memory; it holds
+none of the attention arithmetic.  Tests, the oracle checks and ``bench.py``
+all take their inputs from here, so the CUDA path and the fp64 oracle see the
+same rounded values.
+
+The shapes are the AF2/AF3 training shapes of the pages (MSA-row attention
+with pair bias at initial-training and fine-tuning size, triangle attention
+around the starting and the ending node, and a long AF3-style triangle case);
+no public dataset is involved, every tensor is drawn from N(0, 1) by a seeded
+CPU generator.
+
+Recipe (per workload, generator seeded with ``seed``): draw q, k, v, g,
+pair_bias and dout in fp32 in that order, scale pair_bias by ``bias_scale``,
+then draw the mask permutation; round everything to ``dtype``.  Masks are
+additive ``-1e9`` on a residue subset shared by every row s:
+``"tail:n"`` masks the last n residues, ``"frac:p"`` masks ``round(p*N)``
+residues chosen by a random permutation, ``"none"`` passes no mask.
+
+Layouts.  The op's logical tensors are ``[B, S, N, H, C]`` (row s, residue
+n).  ``msa_row`` and ``tri_start`` store them contiguously.  ``tri_end``
+(triangle attention around the ending node) stores the pair-derived tensors
+in the natural pair layout ``[B, N_i, N_j, H, C]`` and the op reads them
+through a transposed view (row s = j, residue n = i), with no copy.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+MASK_VALUE = -1e9
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    S: int
+    N: int
+    H: int
+    C: int
+    dtype: str            # "bf16" or "f32"
+    layout: str           # "msa_row" | "tri_start" | "tri_end"
+    bias_scale: float
+    mask: str             # "none" | "tail:n" | "frac:p"
+    seed: int
+    note: str = ""
+
+    @property
+    def torch_dtype(self):
+        return {"bf16": torch.bfloat16, "f32": torch.float32}[self.dtype]
+
+    @property
+    def logits(self) -> int:
+        """Number of attention logits B*S*H*N*N."""
+        return self.B * self.S * self.H * self.N * self.N
+
+    @property
+    def fwd_flops(self) -> int:
+        """FlashAttention convention: QK^T and PV, 2 flops per MAC."""
+        return 4 * self.logits * self.C
+
+    @property
+    def bwd_flops(self) -> int:
+        """FlashAttention convention: 2.5x forward (QK^T recompute, dP, dV, dK, dQ)."""
+        return 10 * self.logits * self.C
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five configurations (the fourth has two parts: MSA-row and triangle-end).
+WORKLOADS = {
+    "tiny_f32": Workload("tiny_f32", 1, 4, 32, 4, 8, "f32", "msa_row", 1.0, "tail:4", 20261,
+                         "tiny oracle case, fp32"),
+    "msa_row_256": Workload("msa_row_256", 1, 128, 256, 8, 32, "bf16", "msa_row", 0.5, "frac:0.1",
+                            20262, "MSA-row attention with pair bias, AF2 initial training"),
+    "tri_start_256": Workload("tri_start_256", 1, 256, 256, 4, 32, "bf16", "tri_start", 1.0, "none",
+                              20263, "triangle attention around the starting node"),
+    "msa_row_384": Workload("msa_row_384", 1, 512, 384, 8, 32, "bf16", "msa_row", 1.0, "frac:0.05",
+                            20264, "MSA-row attention, fine-tuning size"),
+    "tri_end_384": Workload("tri_end_384", 1, 384, 384, 4, 32, "bf16", "tri_end", 1.0, "frac:0.05",
+                            20265, "triangle attention around the ending node (transposed pair)"),
+    "tri_long_1536": Workload("tri_long_1536", 1, 1536, 1536, 4, 32, "bf16", "tri_start", 1.0,
+                              "tail:64", 20266, "long AF3-style triangle attention"),
+}
+
+#: Bench default: MSA-row attention at AF2 initial-training size.
+DEFAULT_BENCH = "msa_row_256"
+
+
+def mask_columns(w: Workload, gen: torch.Generator) -> torch.Tensor | None:
+    """Indices of the masked residues (shared by every row), or None."""
+    if w.mask == "none":
+        return None
+    kind, arg = w.mask.split(":")
+    if kind == "tail":
+        n = int(arg)
+        return torch.arange(w.N - n, w.N)
+    if kind == "frac":
+        n = int(round(float(arg) * w.N))
+        return torch.randperm(w.N, generator=gen)[:n].sort().values
+    raise ValueError(f"unknown mask recipe {w.mask!r}")
+
+
+def _storage_shape(w: Workload):
+    if w.layout == "tri_end":
+        # natural pair layout [B, N_i, N_j, H, C]; logical row s = j, residue n = i
+        return (w.B, w.N, w.S, w.H, w.C)
+    return (w.B, w.S, w.N, w.H, w.C)
+
+
+def logical_view(w: Workload, t: torch.Tensor) -> torch.Tensor:
+    """Logical [B, S, N, H, C] view of a tensor stored in the workload's layout."""
+    if w.layout == "tri_end":
+        return t.permute(0, 2, 1, 3, 4)
+    return t
+
+
+def storage_empty(w: Workload, dtype=None, device="cpu") -> torch.Tensor:
+    """An uninitialised per-row tensor in the workload's storage layout (logical view)."""
+    t = torch.empty(_storage_shape(w), dtype=dtype or w.torch_dtype, device=device)
+    return logical_view(w, t)
+
+
+def make_inputs(w: Workload, device="cpu", with_dout: bool = True) -> dict:
+    """Seeded inputs for workload ``w``.
+
+    Returns q, k, v, g, dout as logical ``[B,S,N,H,C]`` views (strided for
+    ``tri_end``), ``mask_bias`` ``[B,S,1,1,N]`` or None, ``pair_bias``
+    ``[B,1,H,N,N]``, all rounded to ``w.dtype`` and placed on ``device``.
+    """
+    if w.layout == "tri_end" and w.S != w.N:
+        raise ValueError("triangle attention needs S == N")
+    gen = torch.Generator("cpu").manual_seed(w.seed)
+    shp = _storage_shape(w)
+    out = {}
+    for name in ("q", "k", "v", "g"):
+        out[name] = torch.randn(shp, generator=gen, dtype=torch.float32)
+    pb = torch.randn((w.B, 1, w.H, w.N, w.N), generator=gen, dtype=torch.float32)
+    if w.bias_scale != 1.0:
+        pb = pb * w.bias_scale
+    out["pair_bias"] = pb
+    if with_dout:
+        out["dout"] = torch.randn(shp, generator=gen, dtype=torch.float32)
+    cols = mask_columns(w, gen)
+    if cols is not None:
+        m = torch.zeros((w.B, w.S, 1, 1, w.N), dtype=torch.float32)
+        m[..., cols] = MASK_VALUE
+        out["mask_bias"] = m
+    else:
+        out["mask_bias"] = None
+    res = {}
+    for name, t in out.items():
+        if t is None:
+            res[name] = None
+            continue
+        t = t.to(w.torch_dtype).to(device)
+        res[name] = logical_view(w, t) if name in ("q", "k", "v", "g", "dout") else t
+    return res
+
+
+def sample_rows(n: int, count: int, seed: int) -> list[int]:
+    """A seeded sorted sample of ``count`` distinct indices in [0, n), always with 0 and n-1."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    count = min(count, n)
+    pick = set(torch.randperm(n, generator=gen)[:count].tolist())
+    pick.update({0, n - 1})
+    return sorted(pick)
+
+
+def logits_bytes(n_res: int, heads: int, elem_bytes: int = 2) -> int:
+    """Bytes of one layer's triangle-attention logits, N^3 * H * elem (never materialised here)."""
+    return n_res ** 3 * heads * elem_bytes
+
+
+def pair_rep_bytes(n_res: int, c_z: int = 128, elem_bytes: int = 2) -> int:
+    """Bytes of the pair representation, N^2 * c_z * elem."""
+    return n_res ** 2 * c_z * elem_bytes
+
+
+def ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+__all__ = ["Workload", "WORKLOADS", "DEFAULT_BENCH", "MASK_VALUE", "make_inputs",
+           "logical_view", "storage_empty", "sample_rows", "logits_bytes", "pair_rep_bytes",
+           "mask_columns", "ceil_div"]

@@ -1,0 +1,270 @@
+/*
+ * evo_ref.c -- plain fp64 CPU oracle for Evoformer attention with pair bias.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only tests/, __graft_entry__.smoke() and bench.py's
+ * cpu_baseline / reference arm use it.  It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * What it computes (per batch b, row s, head h, query i, key j):
+ *
+ *   x[i,j]  = (sum_c q[b,s,i,h,c] * k[b,s,j,h,c]) / sqrt(C)
+ *             + mask_bias[b,s,j] + pair_bias[b,h,i,j]
+ *   lse[i]  = log(sum_j exp(x[i,j]))          (computed as m + log(sum exp(x - m)))
+ *   P[i,j]  = exp(x[i,j] - lse[i])
+ *   A[i,:]  = sum_j P[i,j] * v[b,s,j,h,:]
+ *   out     = sigmoid(g) * A
+ *
+ * This is the attention with an additive, broadcast pair-bias term that the
+ * MegaFold summary describes for EvoFlash-3D ("EvoFlash-3D : Attention 3D
+ * Econome en Memoire"), and the triangle attention of "Evoformer: the memory
+ * wall ZeRO cannot move" (section "The three operations"), whose logits are
+ * O(N_res^3 * n_heads) (section "Where the memory goes", first equation).
+ * The oracle materialises one logit row at a time in fp64: it is the plain
+ * definition, not a tiled or online-softmax rewrite.
+ *
+ * Backward, given dout (chain rule of the definition above):
+ *   sig   = sigmoid(g);   dA = dout * sig;   dg = dout * A * sig * (1 - sig)
+ *   dP[i,j] = sum_c dA[i,c] * v[j,c];        D[i] = sum_j P[i,j] * dP[i,j]
+ *   dS[i,j] = P[i,j] * (dP[i,j] - D[i])
+ *   dv[j] = sum_i P[i,j] dA[i];   dq[i] = sum_j dS[i,j] k[j] / sqrt(C);
+ *   dk[j] = sum_i dS[i,j] q[i] / sqrt(C)
+ *   d_pair_bias[b,h,i,j] = sum_s dS^{(b,s,h)}[i,j]     (mask_bias is a constant)
+ *
+ * Layouts (all contiguous, fp64):
+ *   q, g, out, dout, dq, dg : [B, S, Nq, H, C]
+ *   k, v, dk, dv            : [B, S, Nk, H, C]
+ *   mask_bias               : [B, S, Nk]        (NULL = zeros)
+ *   pair_bias, d_pair_bias  : [B, H, Nq, Nk]    (NULL = zeros)
+ *   lse                     : [B, S, H, Nq]
+ * Nq may differ from Nk so that a caller can evaluate the definition at a
+ * subset of query rows (a smaller, equally valid problem).
+ *
+ * Planted mistakes (mutation testing of the pins): building with
+ * -DEVO_REF_MUTANT=n swaps in one deliberate error, see mutant_* below.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef EVO_REF_MUTANT
+#define EVO_REF_MUTANT 0
+#endif
+
+typedef struct {
+    int64_t B, S, Nq, Nk, H, C;
+} evo_ref_dims;
+
+/* Index helpers for the layouts above. */
+static inline int64_t ix_q(const evo_ref_dims* d, int64_t b, int64_t s, int64_t i, int64_t h) {
+    return (((b * d->S + s) * d->Nq + i) * d->H + h) * d->C;
+}
+static inline int64_t ix_k(const evo_ref_dims* d, int64_t b, int64_t s, int64_t j, int64_t h) {
+    return (((b * d->S + s) * d->Nk + j) * d->H + h) * d->C;
+}
+static inline int64_t ix_mask(const evo_ref_dims* d, int64_t b, int64_t s, int64_t j) {
+    return (b * d->S + s) * d->Nk + j;
+}
+static inline int64_t ix_bias(const evo_ref_dims* d, int64_t b, int64_t h, int64_t i, int64_t j) {
+    return ((b * d->H + h) * d->Nq + i) * d->Nk + j;
+}
+static inline int64_t ix_lse(const evo_ref_dims* d, int64_t b, int64_t s, int64_t h, int64_t i) {
+    return ((b * d->S + s) * d->H + h) * d->Nq + i;
+}
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/* Logit row x[0..Nk) for (b, s, h, query i), straight from the definition. */
+static void logit_row(const evo_ref_dims* d, const double* q, const double* k,
+                      const double* mask, const double* bias,
+                      int64_t b, int64_t s, int64_t h, int64_t i, double* x) {
+    const double* qi = q + ix_q(d, b, s, i, h);
+#if EVO_REF_MUTANT == 3
+    const double scale = 1.0 / (double)d->C;           /* mutant: 1/C instead of 1/sqrt(C) */
+#else
+    const double scale = 1.0 / sqrt((double)d->C);
+#endif
+    for (int64_t j = 0; j < d->Nk; ++j) {
+        const double* kj = k + ix_k(d, b, s, j, h);
+        double dot = 0.0;
+        for (int64_t c = 0; c < d->C; ++c) dot += qi[c] * kj[c];
+        double xij = dot * scale;
+#if EVO_REF_MUTANT != 2                                /* mutant 2: mask dropped */
+        if (mask) xij += mask[ix_mask(d, b, s, j)];
+#endif
+#if EVO_REF_MUTANT == 5                                /* mutant 5: bias read transposed */
+        if (bias) xij += bias[ix_bias(d, b, h, j, i)];
+#elif EVO_REF_MUTANT != 1                              /* mutant 1: pair bias dropped */
+        if (bias) xij += bias[ix_bias(d, b, h, i, j)];
+#endif
+        x[j] = xij;
+    }
+}
+
+/* In place: x <- softmax(x); returns lse = m + log(sum exp(x - m)). */
+static double softmax_row(int64_t n, double* x) {
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) m = x[j] > m ? x[j] : m;
+    double l = 0.0;
+    for (int64_t j = 0; j < n; ++j) l += exp(x[j] - m);
+    const double lse = m + log(l);
+    for (int64_t j = 0; j < n; ++j) x[j] = exp(x[j] - lse);
+    return lse;
+}
+
+static double gate(double g) {
+#if EVO_REF_MUTANT == 4
+    (void)g;
+    return 1.0;                                        /* mutant 4: gate omitted */
+#else
+    return sigmoid(g);
+#endif
+}
+
+/* Everything one query row contributes to the backward pass.
+ * In:  the row's P (from logit_row + softmax_row).
+ * Out: A[C], dA[C], dP/dS row (dS written over dp), D.                  */
+static void backward_row(const evo_ref_dims* d, const double* v, const double* g,
+                         const double* dout, int64_t b, int64_t s, int64_t h, int64_t i,
+                         const double* p, double* A, double* dA, double* ds, double* dg_row) {
+    const int64_t C = d->C;
+    const double* gi = g + ix_q(d, b, s, i, h);
+    const double* doi = dout + ix_q(d, b, s, i, h);
+    for (int64_t c = 0; c < C; ++c) A[c] = 0.0;
+    for (int64_t j = 0; j < d->Nk; ++j) {
+        const double* vj = v + ix_k(d, b, s, j, h);
+        for (int64_t c = 0; c < C; ++c) A[c] += p[j] * vj[c];
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        const double sg = gate(gi[c]);
+        dA[c] = doi[c] * sg;
+        if (dg_row) dg_row[c] = doi[c] * A[c] * sg * (1.0 - sg);
+    }
+    double D = 0.0;
+    for (int64_t j = 0; j < d->Nk; ++j) {
+        const double* vj = v + ix_k(d, b, s, j, h);
+        double dp = 0.0;
+        for (int64_t c = 0; c < C; ++c) dp += dA[c] * vj[c];
+        ds[j] = dp;                                    /* dP for now */
+        D += p[j] * dp;
+    }
+#if EVO_REF_MUTANT == 6
+    D = -D;                                            /* mutant 6: sign of D flipped */
+#endif
+    for (int64_t j = 0; j < d->Nk; ++j) ds[j] = p[j] * (ds[j] - D);
+}
+
+int evo_ref_forward(const evo_ref_dims* d, const double* q, const double* k, const double* v,
+                    const double* g, const double* mask, const double* bias,
+                    double* out, double* lse) {
+    if (!d || d->B < 0 || d->S < 0 || d->Nq < 0 || d->Nk < 1 || d->H < 0 || d->C < 1) return 1;
+    const int64_t nslice = d->B * d->S * d->H;
+#pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)d->Nk);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < nslice; ++t) {
+            const int64_t h = t % d->H, s = (t / d->H) % d->S, b = t / (d->H * d->S);
+            for (int64_t i = 0; i < d->Nq; ++i) {
+                logit_row(d, q, k, mask, bias, b, s, h, i, x);
+                const double l = softmax_row(d->Nk, x);
+                if (lse) lse[ix_lse(d, b, s, h, i)] = l;
+                const double* gi = g + ix_q(d, b, s, i, h);
+                double* oi = out + ix_q(d, b, s, i, h);
+                for (int64_t c = 0; c < d->C; ++c) {
+                    double a = 0.0;
+                    for (int64_t j = 0; j < d->Nk; ++j) a += x[j] * v[ix_k(d, b, s, j, h) + c];
+                    oi[c] = gate(gi[c]) * a;
+                }
+            }
+        }
+        free(x);
+    }
+    return 0;
+}
+
+/* Gradients of the definition above.  Any output pointer may be NULL.
+ * dk and dv are sums over all Nq query rows, so they are only the true
+ * gradients when the caller passes every query row (Nq == Nk problem). */
+int evo_ref_backward(const evo_ref_dims* d, const double* q, const double* k, const double* v,
+                     const double* g, const double* mask, const double* bias,
+                     const double* dout, double* dq, double* dk, double* dv, double* dg,
+                     double* d_pair_bias) {
+    if (!d || d->B < 0 || d->S < 0 || d->Nq < 0 || d->Nk < 1 || d->H < 0 || d->C < 1) return 1;
+    const int64_t C = d->C;
+    const double rs = 1.0 / sqrt((double)C);
+    const int64_t nslice = d->B * d->S * d->H;
+
+    /* Pass 1: per (b, s, h) slice -- dq, dg (row-local) and dk, dv (sums over i). */
+#pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)d->Nk);
+        double* ds = (double*)malloc(sizeof(double) * (size_t)d->Nk);
+        double* A = (double*)malloc(sizeof(double) * (size_t)C);
+        double* dA = (double*)malloc(sizeof(double) * (size_t)C);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < nslice; ++t) {
+            const int64_t h = t % d->H, s = (t / d->H) % d->S, b = t / (d->H * d->S);
+            for (int64_t j = 0; j < d->Nk; ++j) {
+                if (dk) memset(dk + ix_k(d, b, s, j, h), 0, sizeof(double) * (size_t)C);
+                if (dv) memset(dv + ix_k(d, b, s, j, h), 0, sizeof(double) * (size_t)C);
+            }
+            for (int64_t i = 0; i < d->Nq; ++i) {
+                logit_row(d, q, k, mask, bias, b, s, h, i, p);
+                softmax_row(d->Nk, p);
+                backward_row(d, v, g, dout, b, s, h, i, p, A, dA,
+                             ds, dg ? dg + ix_q(d, b, s, i, h) : NULL);
+                const double* qi = q + ix_q(d, b, s, i, h);
+                double* dqi = dq ? dq + ix_q(d, b, s, i, h) : NULL;
+                if (dqi) for (int64_t c = 0; c < C; ++c) dqi[c] = 0.0;
+                for (int64_t j = 0; j < d->Nk; ++j) {
+                    const double* kj = k + ix_k(d, b, s, j, h);
+                    if (dqi) for (int64_t c = 0; c < C; ++c) dqi[c] += ds[j] * kj[c] * rs;
+                    if (dk) {
+                        double* dkj = dk + ix_k(d, b, s, j, h);
+#if EVO_REF_MUTANT == 7
+                        for (int64_t c = 0; c < C; ++c) dkj[c] += ds[j] * qi[c];     /* mutant 7: no 1/sqrt(C) */
+#else
+                        for (int64_t c = 0; c < C; ++c) dkj[c] += ds[j] * qi[c] * rs;
+#endif
+                    }
+                    if (dv) {
+                        double* dvj = dv + ix_k(d, b, s, j, h);
+                        for (int64_t c = 0; c < C; ++c) dvj[c] += p[j] * dA[c];
+                    }
+                }
+            }
+        }
+        free(p); free(ds); free(A); free(dA);
+    }
+
+    /* Pass 2: d_pair_bias rows, summed over s in order, one (b, h, i) per task. */
+    if (d_pair_bias) {
+        const int64_t nrow = d->B * d->H * d->Nq;
+#pragma omp parallel
+        {
+            double* p = (double*)malloc(sizeof(double) * (size_t)d->Nk);
+            double* ds = (double*)malloc(sizeof(double) * (size_t)d->Nk);
+            double* A = (double*)malloc(sizeof(double) * (size_t)C);
+            double* dA = (double*)malloc(sizeof(double) * (size_t)C);
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t t = 0; t < nrow; ++t) {
+                const int64_t i = t % d->Nq, h = (t / d->Nq) % d->H, b = t / (d->Nq * d->H);
+                double* row = d_pair_bias + ix_bias(d, b, h, i, 0);
+                for (int64_t j = 0; j < d->Nk; ++j) row[j] = 0.0;
+                for (int64_t s = 0; s < d->S; ++s) {
+                    logit_row(d, q, k, mask, bias, b, s, h, i, p);
+                    softmax_row(d->Nk, p);
+                    backward_row(d, v, g, dout, b, s, h, i, p, A, dA, ds, NULL);
+                    for (int64_t j = 0; j < d->Nk; ++j) row[j] += ds[j];
+                }
+            }
+            free(p); free(ds); free(A); free(dA);
+        }
+    }
+    return 0;
+}
+
+/* Which planted mistake this build carries (0 = none). */
+int evo_ref_mutant(void) { return EVO_REF_MUTANT; }
