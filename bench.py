@@ -1,0 +1,358 @@
+"""Benchmark: Evoformer pair-bias attention forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward and one backward pass (every kernel of the path) over
+one batch of the workload's synthetic inputs, which are resident in HBM when
+the timed region starts.  The L2 cache (126 MB) is flushed before every step
+by writing a 256 MB buffer outside the per-step CUDA-event brackets.  The
+metric is achieved TFLOP/s (FlashAttention flop convention: 4*L*C forward,
+10*L*C backward, L = B*S*H*N^2 logits) and its fraction of the measured bf16
+dense tensor peak.
+
+Multi-GPU: rows are independent problems, so every rank runs its own batch of
+the same workload with no collective on the data path (weak scaling); the
+reported time is the max over ranks and ``value`` counts the work of all
+ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the correctness reference)
+on a bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from evoformer_pair_bias_b200 import attention as A  # noqa: E402
+from evoformer_pair_bias_b200.workloads import WORKLOADS, DEFAULT_BENCH, logical_view, make_inputs  # noqa: E402
+
+METRIC = "Evoformer pair-bias attention fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(bf16=float(p["bf16_tflops"]), bf16_sustained=float(p["bf16_tflops_sustained"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9 or (self.uuid and self.uuid not in parts[0]):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(dev) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return ""
+
+
+def flops(w):
+    return w.fwd_flops, w.bwd_flops
+
+
+def cpu_oracle_sample(w, target_s: float = 12.0, max_rows=None):
+    """Time the fp64 oracle (fwd + bwd) on the first r rows s of the workload, r sized for ~target_s."""
+    import oracle
+    oracle.build()
+    inp = make_inputs(w.with_(S=min(w.S, 64)), device="cpu")
+
+    def run(r):
+        x = {k: (None if v is None else (v[:, :r] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v)
+                 ).double().numpy() if v is not None else None for k, v in inp.items()}
+        t0 = time.perf_counter()
+        oracle.forward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"])
+        oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"], x["dout"])
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    r = max(1, min(inp["q"].shape[1], int(target_s / max(t1, 1e-3))))
+    if max_rows:
+        r = min(r, max_rows)
+    t = run(r) if r > 1 else t1
+    L = w.B * r * w.H * w.N * w.N
+    fl = 14 * L * w.C
+    return dict(value=fl / t / 1e12, unit="TFLOP/s", cores=os.cpu_count(), kind="oracle",
+                sample=f"{r} of {w.S} rows s (all {w.H} heads, N={w.N}), fwd+bwd, fp64, {t:.2f} s",
+                seconds=t)
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    steps, warm = args.steps, args.warmup
+    info = cpu_oracle_sample(w, target_s=max(1.0, 60.0 / max(1, steps + warm)), max_rows=None)
+    rows = int(info["sample"].split()[0])
+    import oracle
+    inp = make_inputs(w.with_(S=min(w.S, 64)), device="cpu")
+    x = {k: (None if v is None else (v[:, :rows] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v)
+             ).double().numpy() if v is not None else None for k, v in inp.items()}
+    times = []
+    for i in range(warm + steps):
+        t0 = time.perf_counter()
+        oracle.forward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"])
+        oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"], x["dout"])
+        if i >= warm:
+            times.append(time.perf_counter() - t0)
+    t = sum(times)
+    fl = 14 * w.B * rows * w.H * w.N * w.N * w.C * steps
+    val = fl / t / 1e12
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps,
+            "warmup": warm, "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "N_seq": w.S, "N_res": w.N, "H": w.H, "c": w.C,
+                       "sample_rows": rows, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": f"{rows} of {w.S} rows s per step, fwd+bwd, fp64"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    import datetime
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    A.load_library()
+    inp = make_inputs(w, device="cpu")
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    out = A.empty_like_rows(d["q"])
+    lse = torch.empty((w.B, w.S, w.H, w.N), dtype=torch.float32, device=dev)
+    dout = d["dout"] if d["dout"].stride() == out.stride() else A.empty_like_rows(out).copy_(d["dout"])
+    grads = {n: A.empty_like_rows(d["q"]) for n in ("dq", "dk", "dv", "dg")}
+    grads["d_pair_bias"] = torch.empty((w.B, 1, w.H, w.N, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(A.workspace_bytes(d["q"]), 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out=out, lse=lse)
+        A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out, lse, dout,
+                       grads=grads, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported a timed-out wait during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    with ClockSampler(gpu_uuid(dev)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        n0 = A.launch_count()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record()
+            A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out=out, lse=lse)
+            ev[i][1].record()
+            A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out, lse, dout,
+                           grads=grads, workspace=ws)
+            ev[i][2].record()
+        torch.cuda.synchronize()
+        barrier()
+        launches = A.launch_count() - n0
+    fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    tot_ms = sum(fwd_ms) + sum(bwd_ms)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([tot_ms, sum(fwd_ms), sum(bwd_ms)], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, fsum, bsum = t.tolist()
+    else:
+        fsum, bsum = sum(fwd_ms), sum(bwd_ms)
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported a timed-out wait during the timed region")
+
+    ff, bf = flops(w)
+    pk = peaks()
+    value = (ff + bf) * K * world / (tot_ms * 1e-3) / 1e12
+    fwd_tf = ff * K / (fsum * 1e-3) / 1e12
+    bwd_tf = bf * K / (bsum * 1e-3) / 1e12
+
+    # end to end: pinned host inputs -> device, fwd + bwd through the public API, results -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        def storage(name, v):  # the underlying (contiguous) buffer of a logical view
+            if w.layout == "tri_end" and name in ("q", "k", "v", "g", "dout"):
+                return v.permute(0, 2, 1, 3, 4)
+            return v
+        hin = {k: (None if v is None else storage(k, v).contiguous().pin_memory()) for k, v in inp.items()}
+        hout = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
+        for n, g in grads.items():
+            hout[n] = torch.empty(g.shape, dtype=g.dtype).pin_memory()
+        dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in hin.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+
+        def e2e_step():
+            for k, v in hin.items():
+                if v is not None:
+                    dev_in[k].copy_(v, non_blocking=True)
+            q, k_, v_, g_, do = (logical_view(w, dev_in[n]) for n in ("q", "k", "v", "g", "dout"))
+            o, l_ = A.evo_attn_fwd(q, k_, v_, g_, dev_in["mask_bias"], dev_in["pair_bias"], out=out, lse=lse)
+            do = do if do.stride() == o.stride() else dout.copy_(do)
+            gr = A.evo_attn_bwd(q, k_, v_, g_, dev_in["mask_bias"], dev_in["pair_bias"], o, l_, do,
+                                grads=grads, workspace=ws)
+            hout["out"].copy_(o, non_blocking=True)
+            hout["lse"].copy_(l_, non_blocking=True)
+            for n in grads:
+                hout[n].copy_(gr[n], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        et = e0.elapsed_time(e1)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([et], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            et = t.item()
+        e2e = {"value": (ff + bf) * K * world / (et * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": et / K}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            cpu = cpu_oracle_sample(w)
+            cpu.pop("seconds", None)
+        except Exception as exc:  # the baseline is reported, never required
+            cpu = {"error": repr(exc)}
+
+    if rank == 0:
+        fwd_us = 1e3 * fsum / K
+        roof = {"bound": "tensor", "kernel": "fwd_bf16_kernel" if w.dtype == "bf16" else "simt fwd_kernel",
+                "achieved": fwd_tf, "peak": pk["bf16"], "unit": "TFLOP/s", "frac": fwd_tf / pk["bf16"],
+                "traffic": None, "peak_source": pk["source"] + " burst bf16",
+                "note": "forward kernel, one launch per evo_attn_fwd call, CUDA events on its stream"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": tot_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N_seq": w.S, "N_res": w.N, "H": w.H, "c": w.C,
+                       "layout": w.layout, "mask": w.mask, "l2": "flushed (256 MB write) before every step",
+                       "parallelism": f"replicas x{world}, rows independent, no collective"},
+            "fwd": {"tflops": fwd_tf, "us_per_call": fwd_us, "frac_measured_peak": fwd_tf / pk["bf16"],
+                    "frac_nominal_peak": fwd_tf / NOMINAL_BF16_TFLOPS},
+            "bwd": {"tflops": bwd_tf, "us_per_call": 1e3 * bsum / K, "frac_measured_peak": bwd_tf / pk["bf16"],
+                    "frac_nominal_peak": bwd_tf / NOMINAL_BF16_TFLOPS},
+            "frac_measured_peak": value / world / pk["bf16"],
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,206 @@
+"""Python binding of libevo_attn.so (include/evo_attn.h).
+
+Argument marshalling only: these functions turn torch tensors into the
+pointers, sizes and strides of the C-ABI and call it on the current CUDA
+stream.  Every step of the computation runs in the library's CUDA kernels;
+there is no fallback of any kind -- if the library is missing or rejects a
+call, an exception says why.
+
+    out, lse = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias)
+    grads = evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout)
+
+Per-row tensors (q, k, v, g, out, dout and the gradients) are logical
+``[B, S, N, H, C]`` views with a contiguous C axis; any other strides are
+passed through, so the triangle attention around the ending node is the same
+call on a transposed view.  ``mask_bias`` is ``[B, S, 1, 1, N]`` and
+``pair_bias`` ``[B, 1, H, N, N]`` (both contiguous, or None).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libevo_attn.so")
+
+EVO_OK = 0
+STATUS = {0: "EVO_OK", 1: "EVO_ERR_INVALID_ARG", 2: "EVO_ERR_UNSUPPORTED", 3: "EVO_ERR_WORKSPACE_TOO_SMALL",
+          4: "EVO_ERR_CUDA", 5: "EVO_ERR_DEVICE_TIMEOUT"}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+
+#: Every symbol include/evo_attn.h declares.
+EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
+           "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count")
+
+
+class EvoError(RuntimeError):
+    def __init__(self, where: str, code: int):
+        super().__init__(f"{where} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("B", "S", "N", "H", "C")]
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("b", "s", "n", "h")]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libevo_attn.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m evoformer_pair_bias_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sp, stp = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.POINTER(Strides)
+    lib.evo_attn_fwd.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, stp, vp, vp]
+    lib.evo_attn_fwd.restype = ctypes.c_int
+    lib.evo_attn_bwd.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, stp, vp,
+                                 vp, vp, vp, vp, stp, vp, vp, ctypes.c_size_t, vp]
+    lib.evo_attn_bwd.restype = ctypes.c_int
+    lib.evo_attn_bwd_workspace_bytes.argtypes = [sp, ctypes.c_int]
+    lib.evo_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.evo_status_string.argtypes = [ctypes.c_int]
+    lib.evo_status_string.restype = ctypes.c_char_p
+    lib.evo_attn_device_status.argtypes = [ctypes.c_int]
+    lib.evo_attn_device_status.restype = ctypes.c_int
+    lib.evo_attn_version.restype = ctypes.c_int
+    lib.evo_attn_launch_count.restype = ctypes.c_uint64
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _shape(q) -> Shape:
+    if q.dim() != 5:
+        raise ValueError(f"expected a [B,S,N,H,C] tensor, got shape {tuple(q.shape)}")
+    return Shape(*q.shape)
+
+
+def _strides(t) -> Strides:
+    st = t.stride()
+    if t.shape[4] > 1 and st[4] != 1:
+        raise ValueError("the C axis must be contiguous")
+    return Strides(st[0], st[1], st[2], st[3])
+
+
+def _same_strides(*ts):
+    ref = ts[0].stride()
+    for t in ts[1:]:
+        if t.stride() != ref:
+            raise ValueError("q, k, v and g (and out/dout, and the gradients) must share strides")
+
+
+def _check(where: str, rc: int):
+    if rc != EVO_OK:
+        raise EvoError(where, rc)
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def empty_like_rows(t: torch.Tensor, dtype=None) -> torch.Tensor:
+    """Uninitialised tensor with t's shape and strides (keeps the transposed-pair layout)."""
+    return torch.empty_strided(t.shape, t.stride(), dtype=dtype or t.dtype, device=t.device)
+
+
+def workspace_bytes(q: torch.Tensor) -> int:
+    lib = load_library()
+    return int(lib.evo_attn_bwd_workspace_bytes(ctypes.byref(_shape(q)), DTYPES[q.dtype]))
+
+
+def evo_attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None):
+    """Forward pass; returns (out, lse).  out/lse may be passed in preallocated."""
+    lib = load_library()
+    _same_strides(q, k, v, g)
+    sh = _shape(q)
+    B, S, N, H, C = q.shape
+    if out is None:
+        out = empty_like_rows(q)
+    if lse is None:
+        lse = torch.empty((B, S, H, N), dtype=torch.float32, device=q.device)
+    for t in (mask_bias, pair_bias):
+        if t is not None and (not t.is_contiguous() or t.dtype != q.dtype):
+            raise ValueError("mask_bias / pair_bias must be contiguous and of q's dtype")
+    rc = lib.evo_attn_fwd(ctypes.byref(sh), DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                          ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out),
+                          ctypes.byref(_strides(out)), _ptr(lse), _stream(q.device))
+    _check("evo_attn_fwd", rc)
+    return out, lse
+
+
+def evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, workspace=None):
+    """Backward pass; returns dict(dq, dk, dv, dg, d_pair_bias).
+
+    d_pair_bias is fp32 ``[B, 1, H, N, N]``.  ``grads`` may hold preallocated
+    outputs, ``workspace`` a preallocated uint8 buffer of ``workspace_bytes(q)``.
+    """
+    lib = load_library()
+    _same_strides(q, k, v, g)
+    _same_strides(out, dout)
+    sh = _shape(q)
+    B, S, N, H, C = q.shape
+    grads = dict(grads or {})
+    for n in ("dq", "dk", "dv", "dg"):
+        if grads.get(n) is None:
+            grads[n] = empty_like_rows(q)
+    if grads.get("d_pair_bias") is None:
+        grads["d_pair_bias"] = torch.empty((B, 1, H, N, N), dtype=torch.float32, device=q.device)
+    _same_strides(grads["dq"], grads["dk"], grads["dv"], grads["dg"])
+    need = int(lib.evo_attn_bwd_workspace_bytes(ctypes.byref(sh), DTYPES[q.dtype]))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    rc = lib.evo_attn_bwd(ctypes.byref(sh), DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                          ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out), _ptr(dout),
+                          ctypes.byref(_strides(out)), _ptr(lse), _ptr(grads["dq"]), _ptr(grads["dk"]),
+                          _ptr(grads["dv"]), _ptr(grads["dg"]), ctypes.byref(_strides(grads["dq"])),
+                          _ptr(grads["d_pair_bias"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                          _stream(q.device))
+    _check("evo_attn_bwd", rc)
+    return grads
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(load_library().evo_attn_launch_count())
+
+
+def device_status(clear: bool = True) -> int:
+    """Synchronises and returns the library's device status (0 = EVO_OK, 5 = a wait timed out)."""
+    return int(load_library().evo_attn_device_status(1 if clear else 0))
+
+
+class EvoformerAttention(torch.autograd.Function):
+    """autograd wrapper: out = sigmoid(g) * softmax(q k^T/sqrt(C) + mask_bias + pair_bias) v."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, mask_bias, pair_bias):
+        out, lse = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias)
+        ctx.save_for_backward(q, k, v, g, mask_bias, pair_bias, out, lse)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, g, mask_bias, pair_bias, out, lse = ctx.saved_tensors
+        dout = dout if dout.stride() == out.stride() else empty_like_rows(out).copy_(dout)
+        gr = evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout)
+        dpb = None
+        if pair_bias is not None and ctx.needs_input_grad[5]:
+            dpb = gr["d_pair_bias"].to(pair_bias.dtype)
+        return gr["dq"], gr["dk"], gr["dv"], gr["dg"], None, dpb
+
+
+def evoformer_attention(q, k, v, g, mask_bias=None, pair_bias=None):
+    return EvoformerAttention.apply(q, k, v, g, mask_bias, pair_bias)

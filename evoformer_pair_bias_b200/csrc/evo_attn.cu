@@ -1,0 +1,368 @@
+// evo_attn.cu -- C-ABI entry points, argument validation and launch layer.
+//
+// The whole library is one translation unit (it includes every kernel
+// header), so the device status word and all kernels share one module.
+//
+// Call shapes handled here (all through strides, no copies):
+//   MSA-row attention          rows s = MSA sequences
+//   triangle, starting node    rows s = pair rows
+//   triangle, ending node      transposed pair: s and n strides swapped
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "evo_attn.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "sm100.cuh"
+#include "fwd_sm100.cuh"
+#include "bwd_sm100.cuh"
+
+#define EVO_VERSION 10000
+
+namespace {
+
+using evo::Strides;
+
+std::atomic<uint64_t> g_launches{0};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+Strides to_strides(const evo_strides_t& s) { return Strides{s.b, s.s, s.n, s.h}; }
+
+bool strides_ok(const evo_strides_t* s) {
+    return s && s->b >= 0 && s->s >= 0 && s->n >= 0 && s->h >= 0;
+}
+
+bool strides_mult(const evo_strides_t* s, int64_t m) {
+    return s->b % m == 0 && s->s % m == 0 && s->n % m == 0 && s->h % m == 0;
+}
+
+// Every element of a [B,S,N,H,C] view must be addressed at most once: the
+// strides must not make two logical rows of the output overlap.  (Inputs may
+// alias freely.)  Checked by sorting the four (extent, stride) pairs.
+bool non_overlapping(const evo_shape_t& sh, const evo_strides_t& st) {
+    struct D { int64_t n, s; };
+    D d[5] = {{sh.B, st.b}, {sh.S, st.s}, {sh.N, st.n}, {sh.H, st.h}, {sh.C, 1}};
+    std::sort(d, d + 5, [](const D& a, const D& b) { return a.s < b.s; });
+    int64_t span = 1;  // elements covered by the inner dims so far
+    for (auto& e : d) {
+        if (e.n == 1) continue;
+        if (e.s < span) return false;
+        span = e.s * e.n;
+    }
+    return true;
+}
+
+evo_status_t check_shape(const evo_shape_t* sh) {
+    if (!sh) return EVO_ERR_INVALID_ARG;
+    if (sh->B < 0 || sh->S < 0 || sh->N < 0 || sh->H < 0 || sh->C < 1) return EVO_ERR_INVALID_ARG;
+    if (sh->B > 65535 || sh->S > (1 << 30) || sh->N > (1 << 30) || sh->H > 65535) return EVO_ERR_UNSUPPORTED;
+    if (sh->B * sh->H > 65535) return EVO_ERR_UNSUPPORTED;
+    return EVO_OK;
+}
+
+bool empty_call(const evo_shape_t* sh) { return sh->B == 0 || sh->S == 0 || sh->N == 0 || sh->H == 0; }
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// rank-r tiled bf16 map; dims[0] is contiguous; strides_b are byte strides of dims 1..r-1.
+bool encode_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_b,
+                 const uint32_t* box, CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[5];
+    cuuint64_t s[4];
+    cuuint32_t bx[5], es[5];
+    uint64_t span = dims[0] * 2;
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+    }
+    for (int i = 1; i < rank; ++i) span = std::max<uint64_t>(span, strides_b[i - 1] * dims[i]);
+    for (int i = 1; i < rank; ++i) {
+        // a size-1 dimension is never stepped along; give it any legal stride
+        uint64_t st = strides_b[i - 1];
+        if (dims[i] == 1) st = (span + 15) / 16 * 16;
+        if (st % 16 != 0 || st >= (1ull << 40)) return false;
+        s[i - 1] = st;
+    }
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, s, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// [B,S,N,H,C] per-row tensor, box = (C, rows, 1, 1, 1)
+bool map_rows(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, const evo_strides_t& st, uint32_t rows,
+              CUtensorMapSwizzle sw) {
+    const uint64_t dims[5] = {(uint64_t)sh.C, (uint64_t)sh.N, (uint64_t)sh.H, (uint64_t)sh.S, (uint64_t)sh.B};
+    const uint64_t str[4] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.s * 2, (uint64_t)st.b * 2};
+    const uint32_t box[5] = {(uint32_t)sh.C, rows, 1, 1, 1};
+    return encode_bf16(m, ptr, 5, dims, str, box, sw);
+}
+
+// pair_bias [B,1,H,N,N] viewed as (j, i, h, b), box = (64, rows, 1, 1), 128B swizzle
+bool map_bias(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, uint32_t rows) {
+    const uint64_t N = (uint64_t)sh.N, H = (uint64_t)sh.H;
+    const uint64_t dims[4] = {N, N, H, (uint64_t)sh.B};
+    const uint64_t str[3] = {N * 2, N * N * 2, H * N * N * 2};
+    const uint32_t box[4] = {64, rows, 1, 1};
+    return encode_bf16(m, ptr, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// mask_bias [B,S,1,1,N] viewed as (j, s, b), box = (128, 1, 1)
+bool map_mask(CUtensorMap* m, const void* ptr, const evo_shape_t& sh) {
+    const uint64_t N = (uint64_t)sh.N, S = (uint64_t)sh.S;
+    const uint64_t dims[3] = {N, S, (uint64_t)sh.B};
+    const uint64_t str[2] = {N * 2, S * N * 2};
+    const uint32_t box[3] = {128, 1, 1};
+    return encode_bf16(m, ptr, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// ---------------------------------------------------------------- forward
+evo_status_t fwd_f32(const evo_shape_t& sh, const void* q, const void* k, const void* v, const void* g,
+                     const evo_strides_t& in, const void* mask, const void* bias, void* out,
+                     const evo_strides_t& os, float* lse, cudaStream_t stream) {
+    evo::simt::Args a{};
+    a.B = (int)sh.B; a.S = (int)sh.S; a.N = (int)sh.N; a.H = (int)sh.H; a.C = (int)sh.C;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.in = to_strides(in);
+    a.mask = mask; a.bias = bias; a.out_w = out; a.os = to_strides(os); a.lse = lse;
+    dim3 grid((unsigned)((sh.N + evo::simt::kRowsPerCta - 1) / evo::simt::kRowsPerCta), (unsigned)sh.S,
+              (unsigned)(sh.B * sh.H));
+    evo::simt::fwd_kernel<float><<<grid, evo::simt::kWarps * 32, 0, stream>>>(a);
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+template <int NSUB, bool HM, bool HB>
+evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p, const evo_shape_t& sh,
+                             cudaStream_t stream) {
+    using L = evo::fwd::Layout<NSUB>;
+    auto kern = evo::fwd::fwd_bf16_kernel<NSUB, HM, HB>;
+    static cudaError_t attr = set_smem(kern, L::bytes);
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    dim3 grid((unsigned)((sh.N + evo::fwd::BM - 1) / evo::fwd::BM), (unsigned)((sh.S + NSUB - 1) / NSUB),
+              (unsigned)(sh.B * sh.H));
+    kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+constexpr int kFwdNsub = 2;
+
+evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const void* v, const void* g,
+                      const evo_strides_t& in, const void* mask, const void* bias, void* out,
+                      const evo_strides_t& os, float* lse, cudaStream_t stream) {
+    if (sh.C != evo::fwd::HD || sh.N % 8 != 0) return EVO_ERR_UNSUPPORTED;
+    if (!strides_mult(&in, 8) || !strides_mult(&os, 8)) return EVO_ERR_UNSUPPORTED;
+    for (const void* ptr : {q, k, v, g, (const void*)out}) if (!aligned(ptr, 16)) return EVO_ERR_UNSUPPORTED;
+    if ((mask && !aligned(mask, 16)) || (bias && !aligned(bias, 16))) return EVO_ERR_UNSUPPORTED;
+    if ((sh.S + kFwdNsub - 1) / kFwdNsub > 65535) return EVO_ERR_UNSUPPORTED;
+    CUtensorMap maps[5];
+    std::memset(maps, 0, sizeof(maps));
+    if (!map_rows(&maps[0], q, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !map_rows(&maps[1], k, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !map_rows(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B))
+        return EVO_ERR_CUDA;
+    if (bias && !map_bias(&maps[3], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
+    if (mask && !map_mask(&maps[4], mask, sh)) return EVO_ERR_CUDA;
+    evo::fwd::Params p{};
+    p.B = (int)sh.B; p.S = (int)sh.S; p.N = (int)sh.N; p.H = (int)sh.H;
+    p.n_kv = (int)((sh.N + evo::fwd::BN - 1) / evo::fwd::BN);
+    p.scale = 1.0f / sqrtf((float)sh.C);
+    p.g = static_cast<const __nv_bfloat16*>(g);
+    p.in = to_strides(in);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.os = to_strides(os);
+    p.lse = lse;
+    if (mask && bias) return launch_fwd_bf16<kFwdNsub, true, true>(maps, p, sh, stream);
+    if (mask) return launch_fwd_bf16<kFwdNsub, true, false>(maps, p, sh, stream);
+    if (bias) return launch_fwd_bf16<kFwdNsub, false, true>(maps, p, sh, stream);
+    return launch_fwd_bf16<kFwdNsub, false, false>(maps, p, sh, stream);
+}
+
+// ---------------------------------------------------------------- backward
+struct BwdWorkspace {
+    size_t d_off, doa_off, dqacc_off, biast_off, part_off, total;
+    int groups;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+BwdWorkspace bwd_workspace(const evo_shape_t& sh, evo_dtype_t dt) {
+    BwdWorkspace w{};
+    const size_t rows = (size_t)sh.B * sh.S * sh.H * sh.N;       // logit rows
+    const size_t T = rows * (size_t)sh.C;                         // elements of a per-row tensor
+    const size_t pair = (size_t)sh.B * sh.H * sh.N * sh.N;
+    size_t off = 0;
+    w.d_off = off;
+    off = align256(off + rows * 4);
+    if (dt == EVO_DTYPE_BF16) {
+        w.groups = evo::bwd::num_groups(sh.B, sh.S, sh.N, sh.H);
+        w.doa_off = off;
+        off = align256(off + T * 2);
+        w.dqacc_off = off;
+        off = align256(off + T * 4);
+        w.biast_off = off;
+        off = align256(off + pair * 2);
+        w.part_off = off;
+        off = align256(off + pair * 4 * (size_t)(w.groups > 1 ? w.groups : 0));
+    }
+    w.total = off;
+    return w;
+}
+
+evo_status_t bwd_f32(const evo_shape_t& sh, evo::simt::Args a, cudaStream_t stream) {
+    (void)sh;
+    const int64_t rows = (int64_t)a.B * a.S * a.N * a.H;
+    evo::simt::bwd_pre_kernel<float><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(a);
+    const dim3 grid((unsigned)((a.N + evo::simt::kRowsPerCta - 1) / evo::simt::kRowsPerCta), (unsigned)a.S,
+                    (unsigned)(a.B * a.H));
+    evo::simt::bwd_dq_kernel<float><<<grid, evo::simt::kWarps * 32, 0, stream>>>(a);
+    evo::simt::bwd_dkdv_kernel<float><<<grid, evo::simt::kWarps * 32, 0, stream>>>(a);
+    const dim3 gb((unsigned)((a.N + 127) / 128), (unsigned)a.N, (unsigned)(a.B * a.H));
+    evo::simt::bwd_dbias_kernel<float><<<gb, 128, 0, stream>>>(a);
+    g_launches += 4;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* evo_status_string(evo_status_t s) {
+    switch (s) {
+        case EVO_OK: return "EVO_OK";
+        case EVO_ERR_INVALID_ARG: return "EVO_ERR_INVALID_ARG";
+        case EVO_ERR_UNSUPPORTED: return "EVO_ERR_UNSUPPORTED";
+        case EVO_ERR_WORKSPACE_TOO_SMALL: return "EVO_ERR_WORKSPACE_TOO_SMALL";
+        case EVO_ERR_CUDA: return "EVO_ERR_CUDA";
+        case EVO_ERR_DEVICE_TIMEOUT: return "EVO_ERR_DEVICE_TIMEOUT";
+    }
+    return "EVO_ERR_UNKNOWN";
+}
+
+int evo_attn_version(void) { return EVO_VERSION; }
+
+uint64_t evo_attn_launch_count(void) { return g_launches.load(); }
+
+evo_status_t evo_attn_device_status(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return EVO_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_evo_status, sizeof(v)) != cudaSuccess) return EVO_ERR_CUDA;
+    if (clear) {
+        const unsigned int z = 0;
+        if (cudaMemcpyToSymbol(g_evo_status, &z, sizeof(z)) != cudaSuccess) return EVO_ERR_CUDA;
+    }
+    return v == 0 ? EVO_OK : EVO_ERR_DEVICE_TIMEOUT;
+}
+
+size_t evo_attn_bwd_workspace_bytes(const evo_shape_t* shape, evo_dtype_t dtype) {
+    if (check_shape(shape) != EVO_OK) return 0;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_F32) return 0;
+    return bwd_workspace(*shape, dtype).total;
+}
+
+evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
+                          const void* v, const void* g, const evo_strides_t* in_str, const void* mask_bias,
+                          const void* pair_bias, void* out, const evo_strides_t* out_str, float* lse,
+                          void* stream) {
+    evo_status_t st = check_shape(shape);
+    if (st != EVO_OK) return st;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_F32) return EVO_ERR_INVALID_ARG;
+    if (!strides_ok(in_str) || !strides_ok(out_str)) return EVO_ERR_INVALID_ARG;
+    if (empty_call(shape)) return EVO_OK;
+    if (!q || !k || !v || !g || !out || !lse) return EVO_ERR_INVALID_ARG;
+    if (!non_overlapping(*shape, *out_str)) return EVO_ERR_INVALID_ARG;
+    if (!aligned(lse, 4)) return EVO_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == EVO_DTYPE_F32) {
+        if (shape->C > evo::simt::kMaxC) return EVO_ERR_UNSUPPORTED;
+        for (const void* p : {q, k, v, g, (const void*)out})
+            if (!aligned(p, 4)) return EVO_ERR_INVALID_ARG;
+        if (shape->S > 65535) return EVO_ERR_UNSUPPORTED;
+        return fwd_f32(*shape, q, k, v, g, *in_str, mask_bias, pair_bias, out, *out_str, lse, s);
+    }
+    return fwd_bf16(*shape, q, k, v, g, *in_str, mask_bias, pair_bias, out, *out_str, lse, s);
+}
+
+evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
+                          const void* v, const void* g, const evo_strides_t* in_str, const void* mask_bias,
+                          const void* pair_bias, const void* out, const void* dout,
+                          const evo_strides_t* out_str, const float* lse, void* dq, void* dk, void* dv,
+                          void* dg, const evo_strides_t* grad_str, float* d_pair_bias, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    evo_status_t st = check_shape(shape);
+    if (st != EVO_OK) return st;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_F32) return EVO_ERR_INVALID_ARG;
+    if (!strides_ok(in_str) || !strides_ok(out_str) || !strides_ok(grad_str)) return EVO_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (shape->B == 0 || shape->H == 0 || shape->N == 0) return EVO_OK;
+    if (!d_pair_bias || !aligned(d_pair_bias, 4)) return EVO_ERR_INVALID_ARG;
+    const size_t pair_bytes = (size_t)shape->B * shape->H * shape->N * shape->N * sizeof(float);
+    if (shape->S == 0) {
+        return cudaMemsetAsync(d_pair_bias, 0, pair_bytes, s) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+    }
+    if (!q || !k || !v || !g || !out || !dout || !lse || !dq || !dk || !dv || !dg) return EVO_ERR_INVALID_ARG;
+    if (!non_overlapping(*shape, *grad_str)) return EVO_ERR_INVALID_ARG;
+    const BwdWorkspace ws = bwd_workspace(*shape, dtype);
+    if (ws.total > 0 && (!workspace || workspace_bytes < ws.total)) return EVO_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace && !aligned(workspace, 256)) return EVO_ERR_INVALID_ARG;
+    if (!aligned(lse, 4)) return EVO_ERR_INVALID_ARG;
+
+    evo::simt::Args a{};
+    a.B = (int)shape->B; a.S = (int)shape->S; a.N = (int)shape->N; a.H = (int)shape->H; a.C = (int)shape->C;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.in = to_strides(*in_str);
+    a.mask = mask_bias; a.bias = pair_bias; a.out = out; a.dout = dout; a.os = to_strides(*out_str);
+    a.lse = const_cast<float*>(lse);
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.gs = to_strides(*grad_str);
+    a.dbias = d_pair_bias;
+    a.D = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.d_off);
+    if (dtype == EVO_DTYPE_F32) {
+        if (shape->C > evo::simt::kMaxC) return EVO_ERR_UNSUPPORTED;
+        for (const void* p : {q, k, v, g, out, dout, (const void*)dq, (const void*)dk, (const void*)dv,
+                              (const void*)dg})
+            if (!aligned(p, 4)) return EVO_ERR_INVALID_ARG;
+        if (shape->S > 65535 || shape->N > 65535) return EVO_ERR_UNSUPPORTED;
+        return bwd_f32(*shape, a, s);
+    }
+    evo::bwd::Call c{};
+    c.shape = *shape;
+    c.q = q; c.k = k; c.v = v; c.g = g; c.in = *in_str;
+    c.mask = mask_bias; c.bias = pair_bias; c.out = out; c.dout = dout; c.os = *out_str; c.lse = lse;
+    c.dq = dq; c.dk = dk; c.dv = dv; c.dg = dg; c.gs = *grad_str; c.dbias = d_pair_bias;
+    c.ws = static_cast<char*>(workspace);
+    c.d_off = ws.d_off; c.doa_off = ws.doa_off; c.dqacc_off = ws.dqacc_off;
+    c.biast_off = ws.biast_off; c.part_off = ws.part_off; c.groups = ws.groups;
+    int launched = 0;
+    const evo_status_t rs = evo::bwd::run(c, s, &launched);
+    g_launches += (uint64_t)launched;
+    return rs;
+}
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+/*
+ * evo_attn.h -- C-ABI of the B200 (sm_100a) Evoformer attention with pair bias.
+ *
+ * The operation.  For batch b, row s (an MSA sequence for MSA-row attention,
+ * a pair row for triangle attention), head h, query residue i and key j:
+ *
+ *   x[i,j] = (q[b,s,i,h,:] . k[b,s,j,h,:]) / sqrt(C)
+ *            + mask_bias[b,s,0,0,j] + pair_bias[b,0,h,i,j]
+ *   out[b,s,i,h,:] = sigmoid(g[b,s,i,h,:]) * sum_j softmax_j(x[i,:])[j] * v[b,s,j,h,:]
+ *   lse[b,s,h,i]   = log sum_j exp(x[i,j])            (natural log, fp32)
+ *
+ * This is the attention whose additive, broadcast pair-bias term MegaFold's
+ * EvoFlash-3D handles with an online, numerically stable softmax computed
+ * tile by tile in on-chip memory (MegaFold summary, section "EvoFlash-3D :
+ * Attention 3D Econome en Memoire"), and the triangle attention around a node
+ * whose logits are O(N_res^3 * n_heads) ("Evoformer: the memory wall ZeRO
+ * cannot move", sections "Where the memory goes" and "The three operations").
+ * The library never materialises those logits: peak extra memory is linear in
+ * B*H*N^2 and in the per-row tensors.
+ *
+ * Call shapes.  All per-row tensors are logical [B, S, N, H, C] with the C
+ * axis contiguous and the other four axes given by element strides:
+ *   - MSA-row attention:       rows s = MSA sequences, contiguous strides;
+ *   - triangle, starting node: rows s = pair rows i, contiguous strides;
+ *   - triangle, ending node:   the same op on the transposed pair, expressed by
+ *     swapping the s and n strides of a tensor stored as [B, N, N, H, C]
+ *     (no copy).
+ *
+ * Ownership and execution.  The caller allocates every buffer (device
+ * memory), including the backward workspace.  The library never allocates,
+ * frees or synchronises in evo_attn_fwd / evo_attn_bwd: they validate the
+ * arguments on the host, enqueue kernels on `stream` and return.  Outputs are
+ * overwritten, never accumulated into.
+ *
+ * Errors.  Argument problems are found on the host before any launch and
+ * returned as a status (nothing is enqueued then).  A launch failure returns
+ * EVO_ERR_CUDA.  There is no fallback: a shape the kernels do not cover is
+ * EVO_ERR_UNSUPPORTED, never a silent slower path and never a CPU path.
+ * Every wait inside a kernel is bounded; a wait that runs out sets a device
+ * status word, the kernel returns early, and evo_attn_device_status() reports
+ * EVO_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef EVO_ATTN_H_
+#define EVO_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EVO_OK = 0,
+    EVO_ERR_INVALID_ARG = 1,         /* null pointer, negative size, shape mismatch      */
+    EVO_ERR_UNSUPPORTED = 2,         /* valid, but outside what the kernels implement    */
+    EVO_ERR_WORKSPACE_TOO_SMALL = 3, /* backward workspace smaller than the query says   */
+    EVO_ERR_CUDA = 4,                /* a CUDA runtime/driver call or launch failed      */
+    EVO_ERR_DEVICE_TIMEOUT = 5       /* a bounded in-kernel wait ran out (see below)     */
+} evo_status_t;
+
+typedef enum {
+    EVO_DTYPE_BF16 = 0,  /* bf16 storage, fp32 accumulation, tcgen05 tensor cores    */
+    EVO_DTYPE_F32 = 1    /* fp32 storage and arithmetic on the FMA pipe (no TF32)    */
+} evo_dtype_t;
+
+/* Logical sizes: batch B, rows S (N_seq), residues N (N_res), heads H, head dim C. */
+typedef struct {
+    int64_t B, S, N, H, C;
+} evo_shape_t;
+
+/* Element strides of a logical [B, S, N, H, C] tensor; the C stride is 1. */
+typedef struct {
+    int64_t b, s, n, h;
+} evo_strides_t;
+
+/* Limits of the kernels (EVO_ERR_UNSUPPORTED outside them).
+ *   bf16: C == 32; N % 8 == 0; every stride a multiple of 8 elements; every
+ *         pointer 16-byte aligned.
+ *   f32:  1 <= C <= 64; any N >= 1; pointers 4-byte aligned.
+ * Sizes B, S, N or H equal to 0 are an empty call: EVO_OK, nothing launched
+ * except that evo_attn_bwd zero-fills d_pair_bias when S == 0.               */
+
+/*
+ * Bytes of device workspace evo_attn_bwd needs for this shape and dtype
+ * (a pure function of its arguments).  Returns 0 for a null or invalid shape.
+ * The workspace holds the gated output gradient, the row sums D_i, the fp32
+ * dq accumulator, a transposed copy of pair_bias and the per-row-group
+ * partial sums of d_pair_bias; all of it is linear in the per-row tensors and
+ * in B*H*N^2.
+ */
+size_t evo_attn_bwd_workspace_bytes(const evo_shape_t* shape, evo_dtype_t dtype);
+
+/*
+ * Forward pass.
+ *   shape        logical sizes (see above).
+ *   dtype        element type of q, k, v, g, mask_bias, pair_bias and out.
+ *   q, k, v, g   device pointers, logical [B,S,N,H,C] with strides `in_str`.
+ *   in_str       element strides shared by q, k, v and g.
+ *   mask_bias    device pointer, contiguous [B,S,1,1,N] additive mask over the
+ *                keys (e.g. -1e9 for padding), or NULL for none.
+ *   pair_bias    device pointer, contiguous [B,1,H,N,N] indexed [b,h,i,j]
+ *                (query i, key j), or NULL for none.
+ *   out          device pointer, logical [B,S,N,H,C] with strides `out_str`.
+ *   lse          device pointer, contiguous fp32 [B,S,H,N]: the natural-log
+ *                sum-exp of each logit row, saved for the backward pass.
+ *   stream       cudaStream_t to enqueue on (NULL = legacy default stream).
+ */
+evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype,
+                          const void* q, const void* k, const void* v, const void* g,
+                          const evo_strides_t* in_str,
+                          const void* mask_bias, const void* pair_bias,
+                          void* out, const evo_strides_t* out_str,
+                          float* lse, void* stream);
+
+/*
+ * Backward pass.  Recomputes the softmax from q, k, the biases and the saved
+ * lse (no logits are stored), and returns every input gradient:
+ *   dq, dk, dv, dg    device pointers, logical [B,S,N,H,C] with strides
+ *                     `grad_str`, same dtype as the inputs.
+ *   d_pair_bias       device pointer, contiguous fp32 [B,1,H,N,N]: the sum over
+ *                     all rows s of dL/dx.  It is bitwise reproducible: partial
+ *                     sums over fixed row groups are added in a fixed order,
+ *                     with no floating-point atomics.
+ *   out, dout         the forward output and its gradient (strides `out_str`).
+ *   lse               the forward's saved lse.
+ *   workspace         device buffer of at least evo_attn_bwd_workspace_bytes()
+ *                     bytes, 256-byte aligned; contents need not be initialised.
+ * mask_bias gets no gradient (it is a constant).  dq is accumulated in fp32
+ * across key tiles with atomic adds, so its last bits may vary run to run;
+ * every other output is deterministic.
+ */
+evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype,
+                          const void* q, const void* k, const void* v, const void* g,
+                          const evo_strides_t* in_str,
+                          const void* mask_bias, const void* pair_bias,
+                          const void* out, const void* dout, const evo_strides_t* out_str,
+                          const float* lse,
+                          void* dq, void* dk, void* dv, void* dg, const evo_strides_t* grad_str,
+                          float* d_pair_bias,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* evo_status_string(evo_status_t status);
+
+/*
+ * Reports whether any kernel on the current device gave up on a bounded wait
+ * since the last clear.  Synchronises the current device first.  Returns
+ * EVO_OK or EVO_ERR_DEVICE_TIMEOUT (EVO_ERR_CUDA if the device cannot be
+ * queried).  If `clear` is non-zero the status word is reset to zero.
+ */
+evo_status_t evo_attn_device_status(int clear);
+
+/* ABI version, major * 10000 + minor * 100 + patch. */
+int evo_attn_version(void);
+
+/* Number of CUDA kernels this library has enqueued in this process so far
+ * (all devices, all streams).  Host-side counter; never synchronises. */
+uint64_t evo_attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EVO_ATTN_H_ */

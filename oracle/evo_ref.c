@@ -197,8 +197,9 @@ int evo_ref_backward(const evo_ref_dims* d, const double* q, const double* k, co
     const int64_t nslice = d->B * d->S * d->H;
 
     /* Pass 1: per (b, s, h) slice -- dq, dg (row-local) and dk, dv (sums over i). */
-#pragma omp parallel
-    {
+    const int pass1 = dq || dk || dv || dg;
+#pragma omp parallel if (pass1)
+    if (pass1) {
         double* p = (double*)malloc(sizeof(double) * (size_t)d->Nk);
         double* ds = (double*)malloc(sizeof(double) * (size_t)d->Nk);
         double* A = (double*)malloc(sizeof(double) * (size_t)C);

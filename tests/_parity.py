@@ -1,0 +1,96 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the C-ABI
+binding, run the fp64 oracle on the same rounded inputs, compare.
+
+Tolerances (per output tensor, over the compared elements):
+  bf16 inputs, fp32 accumulation: max|gpu - oracle| <= 2e-2 and
+                                  ||gpu - oracle||_2 / ||oracle||_2 <= 5e-3
+  fp32 path:                      ||gpu - oracle||_2 / ||oracle||_2 <= 1e-4
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from evoformer_pair_bias_b200 import attention as A
+from evoformer_pair_bias_b200.workloads import make_inputs
+
+TOL = {"bf16": dict(max_abs=2e-2, rel_l2=5e-3), "f32": dict(max_abs=None, rel_l2=1e-4)}
+ROW_TENSORS = ("q", "k", "v", "g", "dout")
+
+
+def to_gpu(inp):
+    return {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+
+
+def f64(t):
+    return None if t is None else t.detach().to("cpu", torch.float64).numpy()
+
+
+def gpu_fwd_bwd(d, want_bwd=True):
+    out, lse = A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"])
+    res = {"out": out, "lse": lse}
+    if want_bwd:
+        dout = d["dout"]
+        if dout.stride() != out.stride():
+            dout = A.empty_like_rows(out).copy_(dout)
+        res.update(A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"],
+                                  out, lse, dout))
+    torch.cuda.synchronize()
+    return res
+
+
+def oracle_fwd_bwd(inp, want=("dq", "dk", "dv", "dg", "d_pair_bias")):
+    x = {k: f64(v) for k, v in inp.items()}
+    out, lse = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"])
+    res = {"out": out, "lse": lse}
+    if want:
+        res.update(oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"],
+                                   x["dout"], want=want))
+    return res
+
+
+def metrics(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = got - ref
+    den = np.linalg.norm(ref.ravel())
+    return dict(max_abs=float(np.max(np.abs(diff))) if diff.size else 0.0,
+                rel_l2=float(np.linalg.norm(diff.ravel()) / (den if den > 0 else 1.0)),
+                finite=bool(np.all(np.isfinite(got))))
+
+
+def report(case, name, m):
+    path = os.environ.get("EVO_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(case=case, tensor=name, **m)) + "\n")
+
+
+def assert_close(case, name, got, ref, dtype):
+    m = metrics(got, ref)
+    report(case, name, m)
+    tol = TOL[dtype]
+    assert m["finite"], (case, name, "non-finite values")
+    assert m["rel_l2"] <= tol["rel_l2"], (case, name, m)
+    if tol["max_abs"] is not None:
+        assert m["max_abs"] <= tol["max_abs"], (case, name, m)
+    return m
+
+
+def compare_all(case, gpu, ref, dtype, names=("out", "lse", "dq", "dk", "dv", "dg", "d_pair_bias")):
+    for n in names:
+        if n in ref:
+            assert_close(case, n, f64(gpu[n]), ref[n], dtype)
+
+
+def workload_inputs(w, drop_bias=False, drop_mask=False):
+    inp = make_inputs(w, device="cpu")
+    if drop_bias:
+        inp["pair_bias"] = None
+    if drop_mask:
+        inp["mask_bias"] = None
+    return inp

@@ -1,0 +1,88 @@
+"""The C-ABI library builds, loads and exports every symbol include/evo_attn.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from evoformer_pair_bias_b200 import attention as A
+from evoformer_pair_bias_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "evo_attn.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(evo_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return A.load_library()
+
+
+def test_header_declares_the_binding_exports():
+    assert header_functions() == sorted(A.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {A.LIB_PATH}").read()
+    for name in header_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_status_strings_and_version(lib):
+    for code, name in A.STATUS.items():
+        assert lib.evo_status_string(code).decode() == name
+    assert lib.evo_attn_version() >= 10000
+
+
+def test_workspace_query_is_pure_and_linear(lib):
+    def ws(Bb, S, N, H, C, dt):
+        return lib.evo_attn_bwd_workspace_bytes(ctypes.byref(A.Shape(Bb, S, N, H, C)), dt)
+    assert ws(1, 128, 256, 8, 32, 0) == ws(1, 128, 256, 8, 32, 0)
+    assert ws(1, 4, 32, 4, 8, 1) > 0
+    assert lib.evo_attn_bwd_workspace_bytes(None, 0) == 0
+    assert ws(1, 4, 32, 4, 0, 0) == 0            # C = 0 is invalid
+    # no cubic term: for S = N rows the workspace grows like N^2 * (per-row + pair) terms
+    big, small = ws(1, 1536, 1536, 4, 32, 0), ws(1, 768, 768, 4, 32, 0)
+    assert big < 4.5 * small
+
+
+def test_host_argument_errors_need_no_gpu(lib):
+    st = A.Strides(0, 0, 0, 0)
+    sh = A.Shape(1, 2, 8, 1, 32)
+    nul = None
+    rc = lib.evo_attn_fwd(None, 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, ctypes.byref(st), nul, nul)
+    assert rc == 1
+    rc = lib.evo_attn_fwd(ctypes.byref(sh), 7, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+                          ctypes.byref(st), nul, nul)
+    assert rc == 1                                # unknown dtype
+    rc = lib.evo_attn_fwd(ctypes.byref(sh), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+                          ctypes.byref(st), nul, nul)
+    assert rc == 1                                # null tensors
+    empty = A.Shape(1, 0, 8, 1, 32)
+    rc = lib.evo_attn_fwd(ctypes.byref(empty), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+                          ctypes.byref(st), nul, nul)
+    assert rc == 0                                # empty call: nothing to do
+    neg = A.Shape(1, -1, 8, 1, 32)
+    rc = lib.evo_attn_fwd(ctypes.byref(neg), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+                          ctypes.byref(st), nul, nul)
+    assert rc == 1
+
+
+def test_product_path_never_touches_the_oracle():
+    """The package must not import, load or mention the CPU oracle."""
+    pkg = os.path.join(ROOT, "evoformer_pair_bias_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "evo_ref" not in text and "libevo_ref" not in text, f

@@ -1,0 +1,211 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle.
+
+Small cases span several 128-row/128-key tiles and ragged tails and are
+compared element by element on every output.  The two AF2-size configurations
+(MSA-row N=256, triangle-start N=256) are compared in full; the fine-tuning
+and long-sequence configurations are compared on sampled rows s (every head,
+query and key of those rows) and on sampled d_pair_bias rows (summed over all
+rows s), which the oracle evaluates one by one at the full sizes.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import (TOL, assert_close, compare_all, f64, gpu_fwd_bwd, oracle_fwd_bwd, to_gpu,
+                     workload_inputs)
+from evoformer_pair_bias_b200 import attention as A
+from evoformer_pair_bias_b200.workloads import WORKLOADS, Workload, make_inputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # name, B, S, N, H, C, dtype, layout, mask
+    ("ragged_200", 1, 3, 200, 2, 32, "bf16", "msa_row", "frac:0.1"),
+    ("n64_b2", 2, 2, 64, 3, 32, "bf16", "msa_row", "tail:5"),
+    ("n8_tiny", 1, 5, 8, 1, 32, "bf16", "msa_row", "none"),
+    ("three_tiles_392", 1, 1, 392, 1, 32, "bf16", "msa_row", "frac:0.05"),
+    ("tri_end_136", 1, 136, 136, 2, 32, "bf16", "tri_end", "frac:0.05"),
+    ("tri_start_264", 1, 264, 264, 1, 32, "bf16", "tri_start", "tail:3"),
+    ("f32_ragged", 1, 2, 45, 3, 16, "f32", "msa_row", "frac:0.1"),
+    ("f32_c64", 1, 2, 33, 1, 64, "f32", "msa_row", "tail:2"),
+    ("f32_tri_end", 1, 20, 20, 2, 8, "f32", "tri_end", "none"),
+]
+
+
+def small_workload(name, B, S, N, H, C, dt, layout, mask):
+    return Workload(name, B, S, N, H, C, dt, layout, 1.0, mask, seed=zlib.crc32(name.encode()) % 100000 + 7)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from evoformer_pair_bias_b200 import build
+    build.build()
+    A.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    assert A.device_status(clear=True) == 0, "a kernel reported a timed-out wait"
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=[s[0] for s in SMALL])
+def test_small_cases_all_outputs(spec):
+    w = small_workload(*spec)
+    inp = workload_inputs(w)
+    gpu = gpu_fwd_bwd(to_gpu(inp))
+    ref = oracle_fwd_bwd(inp)
+    compare_all(w.name, gpu, ref, w.dtype)
+
+
+@pytest.mark.parametrize("drop", ["bias", "mask", "both"])
+def test_optional_biases(drop):
+    w = Workload("opt_" + drop, 1, 3, 136, 2, 32, "bf16", "msa_row", 1.0, "frac:0.1", 911)
+    inp = workload_inputs(w, drop_bias=drop in ("bias", "both"), drop_mask=drop in ("mask", "both"))
+    gpu = gpu_fwd_bwd(to_gpu(inp))
+    ref = oracle_fwd_bwd(inp)
+    compare_all(w.name, gpu, ref, "bf16")
+
+
+def test_tiny_fp32_config():
+    w = WORKLOADS["tiny_f32"]
+    inp = workload_inputs(w)
+    gpu = gpu_fwd_bwd(to_gpu(inp))
+    ref = oracle_fwd_bwd(inp)
+    compare_all(w.name, gpu, ref, "f32")
+
+
+@pytest.mark.parametrize("name", ["msa_row_256", "tri_start_256"])
+def test_full_af2_configs(name):
+    w = WORKLOADS[name]
+    inp = workload_inputs(w)
+    gpu = gpu_fwd_bwd(to_gpu(inp))
+    ref = oracle_fwd_bwd(inp)
+    compare_all(w.name, gpu, ref, "bf16")
+
+
+def _sampled(w, n_rows=3, n_bias_rows=4):
+    inp = workload_inputs(w)
+    d = to_gpu(inp)
+    gpu = gpu_fwd_bwd(d)
+    srows = sample_rows(w.S, n_rows, w.seed)
+    # every head / query / key of the sampled rows s
+    sub = {k: (None if v is None else (v[:, srows] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v))
+           for k, v in inp.items()}
+    ref = oracle_fwd_bwd(sub, want=("dq", "dk", "dv", "dg"))
+    for n in ("out", "dq", "dk", "dv", "dg"):
+        assert_close(w.name + "[s-sample]", n, f64(gpu[n])[:, srows], ref[n], "bf16")
+    assert_close(w.name + "[s-sample]", "lse", f64(gpu["lse"])[:, srows], ref["lse"], "bf16")
+    # d_pair_bias rows i, summed over every row s, one head at a time
+    irows = sample_rows(w.N, n_bias_rows, w.seed + 1)
+    got, want = [], []
+    for h in range(w.H):
+        hs = slice(h, h + 1)
+        x = {
+            "q": f64(inp["q"][:, :, irows, hs]), "k": f64(inp["k"][:, :, :, hs]), "v": f64(inp["v"][:, :, :, hs]),
+            "g": f64(inp["g"][:, :, irows, hs]), "dout": f64(inp["dout"][:, :, irows, hs]),
+            "mask_bias": f64(inp["mask_bias"]), "pair_bias": f64(inp["pair_bias"][:, :, hs][..., irows, :]),
+        }
+        r = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"], x["dout"],
+                            want=("d_pair_bias",))
+        want.append(r["d_pair_bias"])
+        got.append(f64(gpu["d_pair_bias"][:, :, hs][..., irows, :]))
+    assert_close(w.name + "[i-sample]", "d_pair_bias", np.concatenate(got, 2), np.concatenate(want, 2), "bf16")
+    return gpu
+
+
+@pytest.mark.parametrize("name", ["msa_row_384", "tri_end_384", "tri_long_1536"])
+def test_large_configs_sampled(name):
+    _sampled(WORKLOADS[name])
+
+
+def test_d_pair_bias_is_bitwise_deterministic():
+    w = WORKLOADS["msa_row_256"]
+    d = to_gpu(workload_inputs(w))
+    runs = [gpu_fwd_bwd(d)["d_pair_bias"].clone() for _ in range(4)]
+    for r in runs[1:]:
+        assert torch.equal(r, runs[0])
+
+
+def test_residue_permutation_equivariance_on_gpu():
+    """Relabelling the residues permutes every output (within the bf16 tolerance)."""
+    w = Workload("perm", 1, 4, 160, 2, 32, "bf16", "msa_row", 1.0, "frac:0.1", 4242)
+    inp = workload_inputs(w)
+    perm = torch.randperm(w.N, generator=torch.Generator().manual_seed(5))
+    pinp = {}
+    for k, v in inp.items():
+        if k in ("q", "k", "v", "g", "dout"):
+            pinp[k] = v[:, :, perm].contiguous()
+        elif k == "mask_bias":
+            pinp[k] = v[..., perm].contiguous()
+        else:
+            pinp[k] = v[..., perm, :][..., perm].contiguous()
+    a = gpu_fwd_bwd(to_gpu(inp))
+    b = gpu_fwd_bwd(to_gpu(pinp))
+    for n in ("out", "dq", "dk", "dv", "dg"):
+        assert_close("perm", n, f64(b[n]), f64(a[n])[:, :, perm.numpy()], "bf16")
+    assert_close("perm", "lse", f64(b["lse"]), f64(a["lse"])[..., perm.numpy()], "bf16")
+    pn = perm.numpy()
+    assert_close("perm", "d_pair_bias", f64(b["d_pair_bias"]), f64(a["d_pair_bias"])[..., pn, :][..., pn], "bf16")
+
+
+def test_fully_masked_row_stays_finite():
+    w = Workload("allmask", 1, 2, 64, 1, 32, "bf16", "msa_row", 1.0, "none", 77)
+    inp = workload_inputs(w)
+    m = torch.zeros((1, 2, 1, 1, 64), dtype=torch.bfloat16)
+    m[0, 1] = -1e9                                  # every key of row s = 1 masked
+    inp["mask_bias"] = m
+    gpu = gpu_fwd_bwd(to_gpu(inp))
+    for n in ("out", "lse", "dq", "dk", "dv", "dg", "d_pair_bias"):
+        assert torch.isfinite(gpu[n].float()).all(), n
+    ref = oracle_fwd_bwd({k: (v[:, :1] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v)
+                          for k, v in inp.items()}, want=("dq",))
+    assert_close("allmask", "out", f64(gpu["out"])[:, :1], ref["out"], "bf16")
+
+
+def test_unsupported_and_invalid_calls_fail_cleanly():
+    w = Workload("err", 1, 2, 64, 1, 32, "bf16", "msa_row", 1.0, "none", 3)
+    d = to_gpu(workload_inputs(w))
+    # head dim outside the bf16 kernels
+    q64 = torch.randn(1, 2, 64, 1, 64, device="cuda").bfloat16()
+    with pytest.raises(A.EvoError) as e:
+        A.evo_attn_fwd(q64, q64, q64, q64)
+    assert e.value.code == 2
+    # misaligned base pointer (2 bytes off)
+    buf = torch.empty(d["q"].numel() + 8, dtype=torch.bfloat16, device="cuda")
+    qm = buf[1:1 + d["q"].numel()].view(d["q"].shape)
+    with pytest.raises(A.EvoError) as e:
+        A.evo_attn_fwd(qm, d["k"], d["v"], d["g"])
+    assert e.value.code == 2
+    # workspace too small
+    out, lse = A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], None, d["pair_bias"])
+    with pytest.raises(A.EvoError) as e:
+        A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], None, d["pair_bias"], out, lse, d["dout"],
+                       workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 3
+    # empty batch of rows: d_pair_bias is the empty sum
+    e0 = {k: (v[:, :0] if (v is not None and k in ("q", "k", "v", "g", "dout")) else v) for k, v in d.items()}
+    g0 = A.evo_attn_bwd(e0["q"], e0["k"], e0["v"], e0["g"], None, e0["pair_bias"], e0["q"],
+                        torch.empty(1, 0, 1, 64, device="cuda"), e0["dout"])
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(g0["d_pair_bias"]) == 0
+    assert A.device_status(clear=False) == 0
+
+
+def test_peak_memory_is_linear_not_cubic():
+    """Config 5: the library allocates nothing; everything beyond inputs is outputs + workspace."""
+    w = WORKLOADS["tri_long_1536"]
+    d = to_gpu(make_inputs(w, device="cpu"))
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    gpu = gpu_fwd_bwd(d)
+    peak = torch.cuda.max_memory_allocated() - base
+    T = w.B * w.S * w.N * w.H * w.C
+    pair = w.B * w.H * w.N * w.N
+    outputs = T * 2 * 5 + w.B * w.S * w.H * w.N * 4 + pair * 4
+    ws = A.workspace_bytes(d["q"])
+    assert peak <= outputs + ws + (64 << 20)
+    logits_fp32 = w.logits * 4
+    assert peak < logits_fp32 / 8, (peak, logits_fp32)
+    del gpu
