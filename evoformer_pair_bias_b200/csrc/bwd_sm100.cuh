@@ -1,24 +1,554 @@
-// bwd_sm100.cuh -- bf16 backward of Evoformer pair-bias attention.
+// bwd_sm100.cuh -- bf16 backward of Evoformer pair-bias attention on sm_100a.
+//
+// Like the forward, the backward never stores a logit: P is recomputed tile
+// by tile from q, k, the biases and the saved log-sum-exp, which is how
+// EvoFlash-3D treats the backward pass (MegaFold summary, section
+// "EvoFlash-3D": logits computed incrementally in on-chip memory in the
+// forward and the backward passes).
+//
+// Kernels (one stream, in order):
+//   bwd_pre        per logit row: D_i = sum_c dout*out, dOa = dout*sigmoid(g)
+//                  (bf16), dg = dout*out*(1-sigmoid(g)), nl_i = -lse_i*log2(e);
+//                  zeroes the fp32 dq accumulator.
+//   transpose_bias pair_bias[b,h,i,j] -> biasT[b,h,j,i] (bf16), so that the
+//                  main kernel reads bias rows along its TMEM lanes (keys).
+//   bwd_main       CTA = (key tile j, row group g, b*H + h); loops over the
+//                  group's rows s (outer) and query tiles i (inner):
+//                    S^T  = K_j Q_i^T      dP^T = V_j dOa_i^T       (TMEM)
+//                    P^T  = exp2(S^T*scale*log2e + bias + mask + nl_i)
+//                    dS^T = P^T (dP^T - D_i)
+//                    dV_j += P^T dOa_i     dK_j += dS^T Q_i         (TMEM)
+//                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
+//                    d_pair_bias partial[g][i,j] += dS (plain load/store: the
+//                    CTA is the only writer of its strip, rows s in order)
+//   bwd_post       dq = bf16(accumulator); d_pair_bias = sum over g of the
+//                  partials in index order (skipped when there is one group).
+// The result of d_pair_bias is therefore bitwise reproducible; dq's last bits
+// depend on the order of the atomic adds.
 #pragma once
 
 #include "sm100.cuh"
-#include "simt.cuh"
+#include "tma_maps.cuh"
 
 namespace evo {
 namespace bwd {
 
+using namespace evo::sm100;
+
+constexpr int BQ = 128;   // query tile (columns of S^T)
+constexpr int BK = 128;   // key tile (TMEM lanes)
+constexpr int HD = 32;
+constexpr int TILE_BYTES = 128 * HD * 2;          // 8 KB, 64-byte rows, 64B swizzle
+constexpr int BT_BOX = 128 * 64 * 2;              // 16 KB: 128 key rows x 64 queries, 128B swizzle
+constexpr int KVB = 2 * TILE_BYTES + 1024;        // K, V, mask row (256 B), padded to 1 KB
+constexpr int STB = 2 * TILE_BYTES + 2 * BT_BOX + 1024;  // Q, dOa, biasT, nl (512 B), D (512 B)
+constexpr int OFF_KV = 0;
+constexpr int OFF_ST = 2 * KVB;
+constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tile, 2 boxes of 128 rows x 128 B
+constexpr int OFF_BAR = OFF_DS + 2 * BT_BOX;
+// kv_full[2] kv_empty[2] q_full[2] q_empty[2] sdp_full sdp_free ds_full ds_free
+// dq_full dq_free dkv_full dkv_free mma_done
+constexpr int NBARS = 17;
+constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 320;                       // warp 0 TMA, warp 1 MMA, warps 2..9 dS
+constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 320, TM_DK = 352, TM_DQ = 384, TM_COLS = 512;
+
 // Row groups for the deterministic d_pair_bias reduction: enough CTAs
 // (key tiles x heads x batch x groups) for about two per SM of a 148-SM B200.
 inline int num_groups(int64_t B, int64_t S, int64_t N, int64_t H) {
-    const int64_t njt = (N + 127) / 128;
+    const int64_t njt = (N + BK - 1) / BK;
     const int64_t base = njt * B * H;
-    if (base <= 0) return 1;
+    if (base <= 0 || S <= 0) return 1;
     int64_t g = (2 * 148 + base - 1) / base;
     if (g > S) g = S;
     if (g < 1) g = 1;
-    return (int)g;
+    const int64_t gsz = (S + g - 1) / g;       // rows per group; drop groups left empty
+    return (int)((S + gsz - 1) / gsz);
 }
 
+struct MainParams {
+    int B, S, N, H;
+    int n_it;            // query tiles
+    int gsz;             // rows s per group
+    float sc2;           // log2(e) / sqrt(C)
+    float rs;            // 1 / sqrt(C)
+    float* part;         // [G,B,H,N,N] partials, or d_pair_bias when G == 1
+    float* dq_acc;       // [B,S,N,H,C] fp32, contiguous
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    Strides gs;
+};
+
+enum : unsigned int { kTimeoutBase = 0x2000u };
+
+template <bool HAS_MASK, bool HAS_BIAS>
+__global__ void __launch_bounds__(THREADS, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_doa,
+                    const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_mask,
+                    const __grid_constant__ CUtensorMap tm_nl, const __grid_constant__ CUtensorMap tm_d,
+                    const MainParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j0 = blockIdx.x * BK;
+    const int grp = blockIdx.y;
+    const int b = blockIdx.z / p.H, h = blockIdx.z % p.H;
+    const int s_begin = grp * p.gsz;
+    const int ns = min(p.gsz, p.S - s_begin);
+    const int ni = p.n_it;
+    const int T = ns * ni;
+
+    const uint32_t bar0 = base + OFF_BAR;
+    auto kv_full = [&](int x) { return bar0 + 8u * (0 + x); };
+    auto kv_empty = [&](int x) { return bar0 + 8u * (2 + x); };
+    auto q_full = [&](int x) { return bar0 + 8u * (4 + x); };
+    auto q_empty = [&](int x) { return bar0 + 8u * (6 + x); };
+    const uint32_t sdp_full = bar0 + 8u * 8, sdp_free = bar0 + 8u * 9;
+    const uint32_t ds_full = bar0 + 8u * 10, ds_free = bar0 + 8u * 11;
+    const uint32_t dq_full = bar0 + 8u * 12, dq_free = bar0 + 8u * 13;
+    const uint32_t dkv_full = bar0 + 8u * 14, dkv_free = bar0 + 8u * 15;
+    const uint32_t mma_done = bar0 + 8u * 16;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(kv_full(x), 1);
+            mbar_init(kv_empty(x), 1 + 8);
+            mbar_init(q_full(x), 1);
+            mbar_init(q_empty(x), 1 + 8);
+        }
+        mbar_init(sdp_full, 1);
+        mbar_init(sdp_free, 8);
+        mbar_init(ds_full, 8);
+        mbar_init(ds_free, 1);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_free, 8);
+        mbar_init(dkv_full, 1);
+        mbar_init(dkv_free, 8);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_doa);
+        prefetch_tmap(&tm_nl); prefetch_tmap(&tm_d);
+        if (HAS_BIAS) prefetch_tmap(&tm_bt);
+        if (HAS_MASK) prefetch_tmap(&tm_mask);
+    }
+    if (warp == 1) {
+        tmem_alloc(base + OFF_MISC, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0 && T > 0) {
+            int kv_issued[2] = {0, 0}, q_issued[2] = {0, 0};
+            bool ok = true;
+            for (int si = 0; si < ns && ok; ++si) {
+                const int s = s_begin + si, x = si & 1;
+                const uint32_t kb = base + OFF_KV + x * KVB;
+                if (si >= 2) ok = mbar_wait(kv_empty(x), ((si >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01);
+                if (!ok) break;
+                mbar_arrive_expect_tx(kv_full(x), 2 * TILE_BYTES + (HAS_MASK ? 256 : 0));
+                tma_load_5d(kb, &tm_k, kv_full(x), 0, j0, h, s, b);
+                tma_load_5d(kb + TILE_BYTES, &tm_v, kv_full(x), 0, j0, h, s, b);
+                if (HAS_MASK) tma_load_3d(kb + 2 * TILE_BYTES, &tm_mask, kv_full(x), j0, s, b);
+                ++kv_issued[x];
+                for (int it = 0; it < ni; ++it) {
+                    const int t = si * ni + it, st = t & 1, i0 = it * BQ;
+                    const uint32_t sb = base + OFF_ST + st * STB;
+                    if (t >= 2) ok = mbar_wait(q_empty(st), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(q_full(st), 2 * TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 1024);
+                    tma_load_5d(sb, &tm_q, q_full(st), 0, i0, h, s, b);
+                    tma_load_5d(sb + TILE_BYTES, &tm_doa, q_full(st), 0, i0, h, s, b);
+                    if (HAS_BIAS) {
+                        tma_load_4d(sb + 2 * TILE_BYTES, &tm_bt, q_full(st), i0, j0, h, b);
+                        tma_load_4d(sb + 2 * TILE_BYTES + BT_BOX, &tm_bt, q_full(st), i0 + 64, j0, h, b);
+                    }
+                    tma_load_4d(sb + 2 * TILE_BYTES + 2 * BT_BOX, &tm_nl, q_full(st), i0, h, s, b);
+                    tma_load_4d(sb + 2 * TILE_BYTES + 2 * BT_BOX + 512, &tm_d, q_full(st), i0, h, s, b);
+                    ++q_issued[st];
+                }
+            }
+            volatile int no_abort = 0;
+            for (int x = 0; x < 2; ++x) {
+                if (kv_issued[x]) mbar_wait(kv_full(x), (kv_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x03);
+                if (q_issued[x]) mbar_wait(q_full(x), (q_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0 && T > 0) {
+            constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // S^T, dP^T
+            constexpr uint32_t ID_KV = idesc_bf16(BK, HD, false, true);    // dV, dK (B MN-major)
+            constexpr uint32_t ID_Q = idesc_bf16(BQ, HD, true, true);      // dQ (A and B MN-major)
+            bool ok = true;
+            auto issue_sdp = [&](int t) -> bool {
+                const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
+                if (it == 0 && !mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x11)) return false;
+                if (!mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x12)) return false;
+                if (t > 0 && !mbar_wait(sdp_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x13)) return false;
+                tc_fence_after();
+                const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    mma_ss(tmem + TM_ST, smem_desc(kb + kk * 32, 16, 512, kSw64), smem_desc(sb + kk * 32, 16, 512, kSw64),
+                           ID_SS, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    mma_ss(tmem + TM_DPT, smem_desc(kb + TILE_BYTES + kk * 32, 16, 512, kSw64),
+                           smem_desc(sb + TILE_BYTES + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                }
+                mma_commit(sdp_full);
+                return true;
+            };
+            ok = issue_sdp(0);
+            for (int t = 0; ok && t < T; ++t) {
+                const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
+                if (t + 1 < T) ok = issue_sdp(t + 1);
+                if (!ok) break;
+                ok = mbar_wait(ds_full, t & 1, abort_flag, kTimeoutBase | 0x14);
+                if (ok && it == 0 && si > 0) ok = mbar_wait(dkv_free, (si - 1) & 1, abort_flag, kTimeoutBase | 0x15);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
+                const uint32_t ds = base + OFF_DS;
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk) {   // dV_j += P^T dOa_i
+                    mma_ts(tmem + TM_DV, tmem + TM_PT + kk * 8, smem_desc(sb + TILE_BYTES + kk * 1024, TILE_BYTES, 512, kSw64),
+                           ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk) {   // dK_j += dS^T Q_i
+                    const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
+                    mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128), smem_desc(sb + kk * 1024, TILE_BYTES, 512, kSw64),
+                           ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x16);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {   // dQ_i = dS K_j
+                    mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
+                           smem_desc(kb + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(ds_free);
+                mma_commit(dq_full);
+                mma_commit(q_empty(st));
+                if (it == ni - 1) {
+                    mma_commit(dkv_full);
+                    mma_commit(kv_empty(x));
+                }
+            }
+            mma_commit(mma_done);
+            volatile int no_abort = 0;
+            mbar_wait(mma_done, 0, &no_abort, kTimeoutBase | 0x17);
+        }
+    } else if (T > 0) {
+        // ---------------------------------------------------------------- dS warpgroups
+        const int wg = (warp - 2) >> 2;          // 0: queries 0..63 of the tile, 1: 64..127
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;          // key row within the tile = TMEM lane
+        const int j = j0 + r;
+        const bool jvalid = j < p.N;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+        const float sc2 = p.sc2;
+        float* part = p.part + ((int64_t)(b * p.H + h) * p.N) * p.N;
+        bool ok = true;
+        float m2 = 0.f;
+
+        // drain helpers -------------------------------------------------
+        auto drain_dq = [&](int t) -> bool {   // dQ rows of step t: lanes = queries
+            if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) return false;
+            tc_fence_after();
+            uint32_t v[16];
+            tmem_ld16_sync(lane_addr + TM_DQ + wg * 16, v);
+            const int si = t / ni, it = t - si * ni;
+            const int i = it * BQ + r, s = s_begin + si;
+            if (i < p.N) {
+                float* dst = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + i) * p.H + h) * HD + wg * 16;
+#pragma unroll
+                for (int c = 0; c < 16; c += 4) {
+                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c),
+                                 "f"(__uint_as_float(v[c]) * p.rs), "f"(__uint_as_float(v[c + 1]) * p.rs),
+                                 "f"(__uint_as_float(v[c + 2]) * p.rs), "f"(__uint_as_float(v[c + 3]) * p.rs)
+                                 : "memory");
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dq_free);
+            return true;
+        };
+        auto drain_dkv = [&](int si) -> bool {   // dK (wg 0) / dV (wg 1) of row s: lanes = keys
+            if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
+            tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32_sync(lane_addr + (wg == 0 ? TM_DK : TM_DV), v);
+            if (jvalid) {
+                const float f = wg == 0 ? p.rs : 1.0f;
+                __nv_bfloat16* dst = (wg == 0 ? p.dk : p.dv) + p.gs.off(b, s_begin + si, j, h);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * f, __uint_as_float(v[8 * q + 1]) * f);
+                    w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * f, __uint_as_float(v[8 * q + 3]) * f);
+                    w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * f, __uint_as_float(v[8 * q + 5]) * f);
+                    w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * f, __uint_as_float(v[8 * q + 7]) * f);
+                    *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dkv_free);
+            return true;
+        };
+
+        for (int t = 0; t < T; ++t) {
+            const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
+            const int i0 = it * BQ;
+            if (it == 0) {
+                ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x23);
+                if (!ok) break;
+                if (HAS_MASK) {
+                    const uint16_t mb = *reinterpret_cast<const uint16_t*>(gbase + OFF_KV + x * KVB + 2 * TILE_BYTES + r * 2);
+                    m2 = __uint_as_float((uint32_t)mb << 16) * EVO_LOG2E;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(kv_empty(x));
+            }
+            ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sv[64], dp[64];
+            tmem_ld32_sync(lane_addr + TM_ST + wg * 64, sv);
+            tmem_ld32_sync(lane_addr + TM_ST + wg * 64 + 32, sv + 32);
+            tmem_ld32_sync(lane_addr + TM_DPT + wg * 64, dp);
+            tmem_ld32_sync(lane_addr + TM_DPT + wg * 64 + 32, dp + 32);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sdp_free);
+
+            if (t > 0) {
+                ok = drain_dq(t - 1);
+                if (ok && it == 0) ok = drain_dkv(si - 1);
+                if (!ok) break;
+            }
+
+            ok = mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x25);
+            if (!ok) break;
+            const uint32_t sb = base + OFF_ST + st * STB;
+            const uint32_t nl_addr = sb + 2 * TILE_BYTES + 2 * BT_BOX + wg * 256;
+            const uint32_t d_addr = nl_addr + 512;
+            const uint32_t bt_addr = sb + 2 * TILE_BYTES + wg * BT_BOX + r * 128;
+            const int ivalid = min(64, p.N - i0 - wg * 64);   // queries of this half inside N
+            float dsf[64];
+            uint32_t pk[32], dk2[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {                      // 8 columns at a time
+                float bt[8];
+                if (HAS_BIAS) {
+                    const uint4 w = lds128(bt_addr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
+                    bt[0] = bf16lo(w.x); bt[1] = bf16hi(w.x); bt[2] = bf16lo(w.y); bt[3] = bf16hi(w.y);
+                    bt[4] = bf16lo(w.z); bt[5] = bf16hi(w.z); bt[6] = bf16lo(w.w); bt[7] = bf16hi(w.w);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) bt[e] = 0.f;
+                }
+                const uint4 n0 = lds128(nl_addr + q * 32), n1 = lds128(nl_addr + q * 32 + 16);
+                const uint4 d0 = lds128(d_addr + q * 32), d1 = lds128(d_addr + q * 32 + 16);
+                const float nl[8] = {__uint_as_float(n0.x), __uint_as_float(n0.y), __uint_as_float(n0.z), __uint_as_float(n0.w),
+                                     __uint_as_float(n1.x), __uint_as_float(n1.y), __uint_as_float(n1.z), __uint_as_float(n1.w)};
+                const float dd[8] = {__uint_as_float(d0.x), __uint_as_float(d0.y), __uint_as_float(d0.z), __uint_as_float(d0.w),
+                                     __uint_as_float(d1.x), __uint_as_float(d1.y), __uint_as_float(d1.z), __uint_as_float(d1.w)};
+                float pv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = q * 8 + e;
+                    const float xx = fmaf(__uint_as_float(sv[c]), sc2, fmaf(bt[e], EVO_LOG2E, m2 + nl[e]));
+                    float pe = ex2(xx);
+                    if (!jvalid || c >= ivalid) pe = 0.f;
+                    pv[e] = pe;
+                    dsf[c] = pe * (__uint_as_float(dp[c]) - dd[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    pk[q * 4 + e] = pack_bf16(pv[2 * e], pv[2 * e + 1]);
+                    dk2[q * 4 + e] = pack_bf16(dsf[q * 8 + 2 * e], dsf[q * 8 + 2 * e + 1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_empty(st));           // bias / nl / D of this stage consumed
+
+            if (t > 0) ok = mbar_wait(ds_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x26);
+            if (!ok) break;
+            tc_fence_after();
+            tmem_st32(lane_addr + TM_PT + wg * 32, pk);
+            const uint32_t ds_row = base + OFF_DS + wg * BT_BOX + r * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t addr = ds_row + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk2[4 * q]),
+                             "r"(dk2[4 * q + 1]), "r"(dk2[4 * q + 2]), "r"(dk2[4 * q + 3])
+                             : "memory");
+            }
+            tc_wait_st();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_full);
+
+            // d_pair_bias partial: this CTA alone owns column strip j of group g
+            if (jvalid) {
+                float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
+                if (si == 0) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < ivalid) col[(int64_t)c * p.N] = dsf[c];
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < ivalid) col[(int64_t)c * p.N] += dsf[c];
+                }
+            }
+        }
+        if (ok) ok = drain_dq(T - 1);
+        if (ok) ok = drain_dkv(ns - 1);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ elementwise kernels
+struct PreParams {
+    int B, S, N, H;
+    const __nv_bfloat16* out; const __nv_bfloat16* dout; Strides os;
+    const __nv_bfloat16* g; Strides in;
+    const float* lse;
+    __nv_bfloat16* dg; Strides gs;
+    __nv_bfloat16* doa;   // contiguous [B,S,N,H,C]
+    float* D;             // [B,S,H,N]
+    float* nl;            // [B,S,H,N]
+    float* dq_acc;        // contiguous [B,S,N,H,C] fp32
+};
+
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
+    const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows; t += (int64_t)gridDim.x * blockDim.x) {
+        const int h = (int)(t % p.H);
+        const int i = (int)((t / p.H) % p.N);
+        const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
+        const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
+        const uint4* o4 = reinterpret_cast<const uint4*>(p.out + p.os.off(b, s, i, h));
+        const uint4* d4 = reinterpret_cast<const uint4*>(p.dout + p.os.off(b, s, i, h));
+        const uint4* g4 = reinterpret_cast<const uint4*>(p.g + p.in.off(b, s, i, h));
+        uint4* dg4 = reinterpret_cast<uint4*>(p.dg + p.gs.off(b, s, i, h));
+        uint4* da4 = reinterpret_cast<uint4*>(p.doa + t * HD);
+        float D = 0.f;
+#pragma unroll
+        for (int q = 0; q < HD / 8; ++q) {
+            const uint4 ow = o4[q], dw = d4[q], gw = g4[q];
+            const uint32_t ov[4] = {ow.x, ow.y, ow.z, ow.w}, dv[4] = {dw.x, dw.y, dw.z, dw.w},
+                           gv[4] = {gw.x, gw.y, gw.z, gw.w};
+            uint32_t dgv[4], dav[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float o0 = bf16lo(ov[e]), o1 = bf16hi(ov[e]);
+                const float d0 = bf16lo(dv[e]), d1 = bf16hi(dv[e]);
+                const float s0 = 1.0f / (1.0f + __expf(-bf16lo(gv[e]))), s1 = 1.0f / (1.0f + __expf(-bf16hi(gv[e])));
+                D = fmaf(d0, o0, D);
+                D = fmaf(d1, o1, D);
+                dgv[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
+                dav[e] = pack_bf16(d0 * s0, d1 * s1);
+            }
+            dg4[q] = make_uint4(dgv[0], dgv[1], dgv[2], dgv[3]);
+            da4[q] = make_uint4(dav[0], dav[1], dav[2], dav[3]);
+        }
+        const int64_t ri = (((int64_t)b * p.S + s) * p.H + h) * p.N + i;
+        p.D[ri] = D;
+        p.nl[ri] = -p.lse[ri] * EVO_LOG2E;
+        float4* acc = reinterpret_cast<float4*>(p.dq_acc + t * HD);
+#pragma unroll
+        for (int q = 0; q < HD / 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// biasT[b,h,j,i] = pair_bias[b,h,i,j]  (32x32 tiles through shared memory)
+__global__ void __launch_bounds__(256) transpose_bias_kernel(const __nv_bfloat16* __restrict__ src,
+                                                             __nv_bfloat16* __restrict__ dst, int N) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int64_t plane = (int64_t)blockIdx.z * N * N;
+    const int bx = blockIdx.x * 32, by = blockIdx.y * 32;
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        const int i = by + y, jj = bx + threadIdx.x;
+        if (i < N && jj < N) tile[y][threadIdx.x] = src[plane + (int64_t)i * N + jj];
+    }
+    __syncthreads();
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        const int jj = bx + y, i = by + threadIdx.x;
+        if (i < N && jj < N) dst[plane + (int64_t)jj * N + i] = tile[threadIdx.x][y];
+    }
+}
+
+struct PostParams {
+    int B, S, N, H;
+    const float* dq_acc;  // contiguous fp32
+    __nv_bfloat16* dq; Strides gs;
+    const float* part; int groups;
+    float* dbias;
+};
+
+// dq (bf16, caller strides) from the fp32 accumulator: one thread per row.
+__global__ void __launch_bounds__(256) dq_convert_kernel(const PostParams p) {
+    const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows; t += (int64_t)gridDim.x * blockDim.x) {
+        const int h = (int)(t % p.H);
+        const int i = (int)((t / p.H) % p.N);
+        const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
+        const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
+        const float4* a = reinterpret_cast<const float4*>(p.dq_acc + t * HD);
+        uint4* o = reinterpret_cast<uint4*>(p.dq + p.gs.off(b, s, i, h));
+#pragma unroll
+        for (int q = 0; q < HD / 8; ++q) {
+            const float4 x = a[2 * q], y = a[2 * q + 1];
+            o[q] = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+        }
+    }
+}
+
+// d_pair_bias = sum over groups g = 0, 1, ... of the partials, in that order.
+__global__ void __launch_bounds__(256) dbias_reduce_kernel(const PostParams p) {
+    const int64_t n4 = (int64_t)p.B * p.H * p.N * p.N / 4;
+    const int64_t stride = (int64_t)p.B * p.H * p.N * p.N;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n4; t += (int64_t)gridDim.x * blockDim.x) {
+        float4 acc = reinterpret_cast<const float4*>(p.part)[t];
+        for (int g = 1; g < p.groups; ++g) {
+            const float4 v = reinterpret_cast<const float4*>(p.part + g * stride)[t];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        reinterpret_cast<float4*>(p.dbias)[t] = acc;
+    }
+}
+
+// ------------------------------------------------------------------ host side
 struct Call {
     evo_shape_t shape;
     const void *q, *k, *v, *g;
@@ -30,32 +560,108 @@ struct Call {
     evo_strides_t gs;
     float* dbias;
     char* ws;
-    size_t d_off, doa_off, dqacc_off, biast_off, part_off;
+    size_t d_off, nl_off, doa_off, dqacc_off, biast_off, part_off;
     int groups;
 };
 
+inline bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+inline int grid_for(int64_t items, int per_block) {
+    const int64_t blocks = (items + per_block - 1) / per_block;
+    return (int)std::min<int64_t>(std::max<int64_t>(blocks, 1), 148 * 16);
+}
+
+template <bool HM, bool HB>
+inline cudaError_t launch_main(const CUtensorMap* m, const MainParams& mp, dim3 grid, cudaStream_t stream) {
+    auto kern = bwd_main_kernel<HM, HB>;
+    static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (attr != cudaSuccess) return attr;
+    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], mp);
+    return cudaGetLastError();
+}
+
 inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     const evo_shape_t& sh = c.shape;
-    simt::Args a{};
-    a.B = (int)sh.B; a.S = (int)sh.S; a.N = (int)sh.N; a.H = (int)sh.H; a.C = (int)sh.C;
-    if (sh.C > simt::kMaxC || sh.S > 65535 || sh.N > 65535) return EVO_ERR_UNSUPPORTED;
-    a.q = c.q; a.k = c.k; a.v = c.v; a.g = c.g; a.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
-    a.mask = c.mask; a.bias = c.bias; a.out = c.out; a.dout = c.dout;
-    a.os = Strides{c.os.b, c.os.s, c.os.n, c.os.h};
-    a.lse = const_cast<float*>(c.lse);
-    a.dq = c.dq; a.dk = c.dk; a.dv = c.dv; a.dg = c.dg; a.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
-    a.dbias = c.dbias;
-    a.D = reinterpret_cast<float*>(c.ws + c.d_off);
-    using T = __nv_bfloat16;
-    const int64_t rows = (int64_t)a.B * a.S * a.N * a.H;
-    simt::bwd_pre_kernel<T><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(a);
-    const dim3 grid((unsigned)((a.N + simt::kRowsPerCta - 1) / simt::kRowsPerCta), (unsigned)a.S,
-                    (unsigned)(a.B * a.H));
-    simt::bwd_dq_kernel<T><<<grid, simt::kWarps * 32, 0, stream>>>(a);
-    simt::bwd_dkdv_kernel<T><<<grid, simt::kWarps * 32, 0, stream>>>(a);
-    const dim3 gb((unsigned)((a.N + 127) / 128), (unsigned)a.N, (unsigned)(a.B * a.H));
-    simt::bwd_dbias_kernel<T><<<gb, 128, 0, stream>>>(a);
-    *launched = 4;
+    *launched = 0;
+    if (sh.C != HD || sh.N % 8 != 0) return EVO_ERR_UNSUPPORTED;
+    const evo_strides_t* strs[3] = {&c.in, &c.os, &c.gs};
+    for (auto s : strs)
+        if (s->b % 8 || s->s % 8 || s->n % 8 || s->h % 8) return EVO_ERR_UNSUPPORTED;
+    for (const void* ptr : {c.q, c.k, c.v, c.g, c.out, c.dout, (const void*)c.dq, (const void*)c.dk,
+                            (const void*)c.dv, (const void*)c.dg})
+        if (!aligned16(ptr)) return EVO_ERR_UNSUPPORTED;
+    if ((c.mask && !aligned16(c.mask)) || (c.bias && !aligned16(c.bias)) || !aligned16(c.dbias))
+        return EVO_ERR_UNSUPPORTED;
+
+    const int B = (int)sh.B, S = (int)sh.S, N = (int)sh.N, H = (int)sh.H;
+    float* D = reinterpret_cast<float*>(c.ws + c.d_off);
+    float* nl = reinterpret_cast<float*>(c.ws + c.nl_off);
+    __nv_bfloat16* doa = reinterpret_cast<__nv_bfloat16*>(c.ws + c.doa_off);
+    float* dq_acc = reinterpret_cast<float*>(c.ws + c.dqacc_off);
+    __nv_bfloat16* biasT = reinterpret_cast<__nv_bfloat16*>(c.ws + c.biast_off);
+    float* part = c.groups > 1 ? reinterpret_cast<float*>(c.ws + c.part_off) : c.dbias;
+
+    const int64_t rows = (int64_t)B * S * N * H;
+    PreParams pp{};
+    pp.B = B; pp.S = S; pp.N = N; pp.H = H;
+    pp.out = static_cast<const __nv_bfloat16*>(c.out); pp.dout = static_cast<const __nv_bfloat16*>(c.dout);
+    pp.os = Strides{c.os.b, c.os.s, c.os.n, c.os.h};
+    pp.g = static_cast<const __nv_bfloat16*>(c.g); pp.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
+    pp.lse = c.lse; pp.dg = static_cast<__nv_bfloat16*>(c.dg); pp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
+    pp.doa = doa; pp.D = D; pp.nl = nl; pp.dq_acc = dq_acc;
+    bwd_pre_kernel<<<grid_for(rows, 256), 256, 0, stream>>>(pp);
+    ++*launched;
+    if (c.bias) {
+        transpose_bias_kernel<<<dim3((N + 31) / 32, (N + 31) / 32, B * H), dim3(32, 8), 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(c.bias), biasT, N);
+        ++*launched;
+    }
+
+    // tensor maps
+    const evo_strides_t contig{(int64_t)S * N * H * HD, (int64_t)N * H * HD, (int64_t)H * HD, (int64_t)HD};
+    CUtensorMap m[8];
+    std::memset(m, 0, sizeof(m));
+    const evo_shape_t& s5 = sh;
+    if (!tma::rows_bf16(&m[0], c.q, s5, c.in, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !tma::rows_bf16(&m[1], c.k, s5, c.in, BK, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !tma::rows_bf16(&m[2], c.v, s5, c.in, BK, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !tma::rows_bf16(&m[3], doa, s5, contig, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !tma::rowscalar_f32(&m[6], nl, s5) || !tma::rowscalar_f32(&m[7], D, s5))
+        return EVO_ERR_CUDA;
+    if (c.bias && !tma::square_bf16(&m[4], biasT, s5, BK)) return EVO_ERR_CUDA;
+    if (c.mask && !tma::mask_bf16(&m[5], c.mask, s5)) return EVO_ERR_CUDA;
+
+    MainParams mp{};
+    mp.B = B; mp.S = S; mp.N = N; mp.H = H;
+    mp.n_it = (N + BQ - 1) / BQ;
+    const int G = c.groups;
+    mp.gsz = (S + G - 1) / G;
+    mp.sc2 = EVO_LOG2E / sqrtf((float)HD);
+    mp.rs = 1.0f / sqrtf((float)HD);
+    mp.part = part;
+    mp.dq_acc = dq_acc;
+    mp.dk = static_cast<__nv_bfloat16*>(c.dk);
+    mp.dv = static_cast<__nv_bfloat16*>(c.dv);
+    mp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
+    const dim3 grid((unsigned)((N + BK - 1) / BK), (unsigned)G, (unsigned)(B * H));
+    cudaError_t e;
+    if (c.mask && c.bias) e = launch_main<true, true>(m, mp, grid, stream);
+    else if (c.mask) e = launch_main<true, false>(m, mp, grid, stream);
+    else if (c.bias) e = launch_main<false, true>(m, mp, grid, stream);
+    else e = launch_main<false, false>(m, mp, grid, stream);
+    if (e != cudaSuccess) return EVO_ERR_CUDA;
+    ++*launched;
+
+    PostParams qp{};
+    qp.B = B; qp.S = S; qp.N = N; qp.H = H;
+    qp.dq_acc = dq_acc; qp.dq = static_cast<__nv_bfloat16*>(c.dq); qp.gs = mp.gs;
+    qp.part = part; qp.groups = G; qp.dbias = c.dbias;
+    dq_convert_kernel<<<grid_for(rows, 256), 256, 0, stream>>>(qp);
+    ++*launched;
+    if (G > 1) {
+        dbias_reduce_kernel<<<grid_for((int64_t)B * H * N * N / 4, 256), 256, 0, stream>>>(qp);
+        ++*launched;
+    }
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 

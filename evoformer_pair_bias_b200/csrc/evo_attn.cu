@@ -8,19 +8,18 @@
 //   triangle, starting node    rows s = pair rows
 //   triangle, ending node      transposed pair: s and n strides swapped
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 
 #include "evo_attn.h"
 #include "common.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
+#include "tma_maps.cuh"
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
 
@@ -70,75 +69,6 @@ evo_status_t check_shape(const evo_shape_t* sh) {
 
 bool empty_call(const evo_shape_t* sh) { return sh->B == 0 || sh->S == 0 || sh->N == 0 || sh->H == 0; }
 
-// ---------------------------------------------------------------- TMA maps
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static std::once_flag once;
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// rank-r tiled bf16 map; dims[0] is contiguous; strides_b are byte strides of dims 1..r-1.
-bool encode_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_b,
-                 const uint32_t* box, CUtensorMapSwizzle sw) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t d[5];
-    cuuint64_t s[4];
-    cuuint32_t bx[5], es[5];
-    uint64_t span = dims[0] * 2;
-    for (int i = 0; i < rank; ++i) {
-        d[i] = dims[i];
-        bx[i] = box[i];
-        es[i] = 1;
-    }
-    for (int i = 1; i < rank; ++i) span = std::max<uint64_t>(span, strides_b[i - 1] * dims[i]);
-    for (int i = 1; i < rank; ++i) {
-        // a size-1 dimension is never stepped along; give it any legal stride
-        uint64_t st = strides_b[i - 1];
-        if (dims[i] == 1) st = (span + 15) / 16 * 16;
-        if (st % 16 != 0 || st >= (1ull << 40)) return false;
-        s[i - 1] = st;
-    }
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, s, bx, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// [B,S,N,H,C] per-row tensor, box = (C, rows, 1, 1, 1)
-bool map_rows(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, const evo_strides_t& st, uint32_t rows,
-              CUtensorMapSwizzle sw) {
-    const uint64_t dims[5] = {(uint64_t)sh.C, (uint64_t)sh.N, (uint64_t)sh.H, (uint64_t)sh.S, (uint64_t)sh.B};
-    const uint64_t str[4] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.s * 2, (uint64_t)st.b * 2};
-    const uint32_t box[5] = {(uint32_t)sh.C, rows, 1, 1, 1};
-    return encode_bf16(m, ptr, 5, dims, str, box, sw);
-}
-
-// pair_bias [B,1,H,N,N] viewed as (j, i, h, b), box = (64, rows, 1, 1), 128B swizzle
-bool map_bias(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, uint32_t rows) {
-    const uint64_t N = (uint64_t)sh.N, H = (uint64_t)sh.H;
-    const uint64_t dims[4] = {N, N, H, (uint64_t)sh.B};
-    const uint64_t str[3] = {N * 2, N * N * 2, H * N * N * 2};
-    const uint32_t box[4] = {64, rows, 1, 1};
-    return encode_bf16(m, ptr, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-// mask_bias [B,S,1,1,N] viewed as (j, s, b), box = (128, 1, 1)
-bool map_mask(CUtensorMap* m, const void* ptr, const evo_shape_t& sh) {
-    const uint64_t N = (uint64_t)sh.N, S = (uint64_t)sh.S;
-    const uint64_t dims[3] = {N, S, (uint64_t)sh.B};
-    const uint64_t str[2] = {N * 2, S * N * 2};
-    const uint32_t box[3] = {128, 1, 1};
-    return encode_bf16(m, ptr, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -185,12 +115,12 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
     if ((sh.S + kFwdNsub - 1) / kFwdNsub > 65535) return EVO_ERR_UNSUPPORTED;
     CUtensorMap maps[5];
     std::memset(maps, 0, sizeof(maps));
-    if (!map_rows(&maps[0], q, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !map_rows(&maps[1], k, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !map_rows(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!evo::tma::rows_bf16(&maps[0], q, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !evo::tma::rows_bf16(&maps[1], k, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B))
         return EVO_ERR_CUDA;
-    if (bias && !map_bias(&maps[3], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
-    if (mask && !map_mask(&maps[4], mask, sh)) return EVO_ERR_CUDA;
+    if (bias && !evo::tma::square_bf16(&maps[3], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
+    if (mask && !evo::tma::mask_bf16(&maps[4], mask, sh)) return EVO_ERR_CUDA;
     evo::fwd::Params p{};
     p.B = (int)sh.B; p.S = (int)sh.S; p.N = (int)sh.N; p.H = (int)sh.H;
     p.n_kv = (int)((sh.N + evo::fwd::BN - 1) / evo::fwd::BN);
@@ -208,7 +138,7 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
 
 // ---------------------------------------------------------------- backward
 struct BwdWorkspace {
-    size_t d_off, doa_off, dqacc_off, biast_off, part_off, total;
+    size_t d_off, nl_off, doa_off, dqacc_off, biast_off, part_off, total;
     int groups;
 };
 
@@ -224,6 +154,8 @@ BwdWorkspace bwd_workspace(const evo_shape_t& sh, evo_dtype_t dt) {
     off = align256(off + rows * 4);
     if (dt == EVO_DTYPE_BF16) {
         w.groups = evo::bwd::num_groups(sh.B, sh.S, sh.N, sh.H);
+        w.nl_off = off;
+        off = align256(off + rows * 4);
         w.doa_off = off;
         off = align256(off + T * 2);
         w.dqacc_off = off;
@@ -357,7 +289,7 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
     c.mask = mask_bias; c.bias = pair_bias; c.out = out; c.dout = dout; c.os = *out_str; c.lse = lse;
     c.dq = dq; c.dk = dk; c.dv = dv; c.dg = dg; c.gs = *grad_str; c.dbias = d_pair_bias;
     c.ws = static_cast<char*>(workspace);
-    c.d_off = ws.d_off; c.doa_off = ws.doa_off; c.dqacc_off = ws.dqacc_off;
+    c.d_off = ws.d_off; c.nl_off = ws.nl_off; c.doa_off = ws.doa_off; c.dqacc_off = ws.dqacc_off;
     c.biast_off = ws.biast_off; c.part_off = ws.part_off; c.groups = ws.groups;
     int launched = 0;
     const evo_status_t rs = evo::bwd::run(c, s, &launched);
