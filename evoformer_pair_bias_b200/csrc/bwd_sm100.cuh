@@ -19,8 +19,8 @@
 //                    dS^T = P^T (dP^T - D_i)
 //                    dV_j += P^T dOa_i     dK_j += dS^T Q_i         (TMEM)
 //                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
-//                    d_pair_bias partial[g][i,j] += dS (plain load/store: the
-//                    CTA is the only writer of its strip, rows s in order)
+//                    d_pair_bias partial[g][i,j] += dS (atomic add; one thread
+//                    is the only writer of each address, rows s in order)
 //   bwd_post       dq = bf16(accumulator); d_pair_bias = sum over g of the
 //                  partials in index order (skipped when there is one group).
 // The result of d_pair_bias is therefore bitwise reproducible; dq's last bits
@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool jvalid = j < p.N;
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
         const float sc2 = p.sc2;
-        float* part = p.part + ((int64_t)(b * p.H + h) * p.N) * p.N;
+        // this group's slab of the partial sums (the output itself when there is one group)
+        float* part = p.part + ((int64_t)grp * p.B * p.H + (int64_t)b * p.H + h) * p.N * p.N;
         bool ok = true;
         float m2 = 0.f;
 
@@ -411,18 +412,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(ds_full);
 
-            // d_pair_bias partial: this CTA alone owns column strip j of group g
+            // d_pair_bias partial (zeroed before the launch).  Each address of this
+            // group's slab is updated by exactly one thread, in row order s, with
+            // fire-and-forget atomic adds; same-thread atomics to one address are
+            // performed in program order, so the sum is bitwise reproducible.
             if (jvalid) {
                 float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
-                if (si == 0) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (c < ivalid) col[(int64_t)c * p.N] = dsf[c];
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (c < ivalid) col[(int64_t)c * p.N] += dsf[c];
-                }
+                for (int c = 0; c < 64; ++c)
+                    if (c < ivalid)
+                        asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (int64_t)c * p.N),
+                                     "f"(dsf[c])
+                                     : "memory");
             }
         }
         if (ok) ok = drain_dq(T - 1);
@@ -616,6 +617,10 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
             static_cast<const __nv_bfloat16*>(c.bias), biasT, N);
         ++*launched;
     }
+
+    // the partial slabs (or the output itself) accumulate by atomic adds from zero
+    const size_t part_bytes = (size_t)c.groups * B * H * N * N * sizeof(float);
+    if (cudaMemsetAsync(part, 0, part_bytes, stream) != cudaSuccess) return EVO_ERR_CUDA;
 
     // tensor maps
     const evo_strides_t contig{(int64_t)S * N * H * HD, (int64_t)N * H * HD, (int64_t)H * HD, (int64_t)HD};

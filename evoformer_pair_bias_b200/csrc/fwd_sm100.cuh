@@ -251,7 +251,8 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, Layout<NSUB>::min_block
             if (!ok) break;
 
             // x = S/sqrt(C) + pair_bias[i, j] + mask_bias[s, j]   (natural-log units)
-            float mloc = -INFINITY;
+            // Row max over 4 independent partial maxima (short dependency chains).
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int q = 0; q < BN / 8; ++q) {
                 float add[8];
@@ -273,9 +274,10 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, Layout<NSUB>::min_block
                 for (int e = 0; e < 8; ++e) {
                     const float xv = fmaf(__uint_as_float(xr[q * 8 + e]), scale, add[e]);
                     xr[q * 8 + e] = __float_as_uint(xv);
-                    mloc = fmaxf(mloc, xv);
+                    mq[e & 3] = fmaxf(mq[e & 3], xv);
                 }
             }
+            float mloc = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             const int valid = p.N - j * BN;      // keys beyond N are padding: exclude them
             if (valid < BN) {
                 mloc = -INFINITY;
@@ -290,15 +292,16 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, Layout<NSUB>::min_block
 
             const float ms_new = fmaxf(ms, mloc * EVO_LOG2E);
             const float alpha = ex2(ms - ms_new);       // 0 on the first tile, exactly 1 if the max stays
-            float rs = 0.f;
+            float rq[4] = {0.f, 0.f, 0.f, 0.f};     // 4 independent partial sums
             uint32_t pk[BN / 2];
 #pragma unroll
             for (int c = 0; c < BN / 2; ++c) {
                 const float p0 = ex2(fmaf(__uint_as_float(xr[2 * c]), EVO_LOG2E, -ms_new));
                 const float p1 = ex2(fmaf(__uint_as_float(xr[2 * c + 1]), EVO_LOG2E, -ms_new));
-                rs += p0 + p1;
+                rq[c & 3] += p0 + p1;
                 pk[c] = pack_bf16(p0, p1);
             }
+            const float rs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
             l = l * alpha + rs;
             ms = ms_new;
             if (j > 0) {
