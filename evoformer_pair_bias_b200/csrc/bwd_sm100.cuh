@@ -8,16 +8,19 @@
 //
 // Kernels (one stream, in order):
 //   bwd_pre        per logit row: D_i = sum_c dout*out, dOa = dout*sigmoid(g)
-//                  (bf16), dg = dout*out*(1-sigmoid(g)), nl_i = -lse_i*log2(e);
-//                  zeroes the fp32 dq accumulator.
+//                  split into a bf16 high part and a bf16 low part (their sum
+//                  carries ~16 mantissa bits into dP), dg = dout*out*(1-sigmoid(g)),
+//                  nl_i = -lse_i*log2(e); zeroes the fp32 dq accumulator.  The
+//                  row terms nl and -D are stored with the query axis padded to
+//                  whole tiles, padding nl = -inf, so padded queries get P = 0.
 //   transpose_bias pair_bias[b,h,i,j] -> biasT[b,h,j,i] (bf16), so that the
 //                  main kernel reads bias rows along its TMEM lanes (keys).
 //   bwd_main       CTA = (key tile j, row group g, b*H + h); loops over the
 //                  group's rows s (outer) and query tiles i (inner):
-//                    S^T  = K_j Q_i^T      dP^T = V_j dOa_i^T       (TMEM)
+//                    S^T  = K_j Q_i^T      dP^T = V_j (dOa_hi + dOa_lo)_i^T  (TMEM)
 //                    P^T  = exp2(S^T*scale*log2e + bias + mask + nl_i)
 //                    dS^T = P^T (dP^T - D_i)
-//                    dV_j += P^T dOa_i     dK_j += dS^T Q_i         (TMEM)
+//                    dV_j += P^T dOa_hi_i  dK_j += dS^T Q_i         (TMEM)
 //                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
 //                    d_pair_bias partial[g][i,j] += dS (atomic add; one thread
 //                    is the only writer of each address, rows s in order)
@@ -41,7 +44,10 @@ constexpr int HD = 32;
 constexpr int TILE_BYTES = 128 * HD * 2;          // 8 KB, 64-byte rows, 64B swizzle
 constexpr int BT_BOX = 128 * 64 * 2;              // 16 KB: 128 key rows x 64 queries, 128B swizzle
 constexpr int KVB = 2 * TILE_BYTES + 1024;        // K, V, mask row (256 B), padded to 1 KB
-constexpr int STB = 2 * TILE_BYTES + 2 * BT_BOX + 1024;  // Q, dOa, biasT, nl (512 B), D (512 B)
+// Q, dOa (bf16 hi part), dOa (lo part), biasT, nl (512 B), -D (512 B)
+constexpr int STB = 3 * TILE_BYTES + 2 * BT_BOX + 1024;
+constexpr int ST_Q = 0, ST_DOH = TILE_BYTES, ST_DOL = 2 * TILE_BYTES, ST_BT = 3 * TILE_BYTES;
+constexpr int ST_NL = 3 * TILE_BYTES + 2 * BT_BOX, ST_ND = ST_NL + 512;
 constexpr int OFF_KV = 0;
 constexpr int OFF_ST = 2 * KVB;
 constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tile, 2 boxes of 128 rows x 128 B
@@ -54,13 +60,13 @@ constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr int THREADS = 320;                       // warp 0 TMA, warp 1 MMA, warps 2..9 dS
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 320, TM_DK = 352, TM_DQ = 384, TM_COLS = 512;
 
-// Row groups for the deterministic d_pair_bias reduction: enough CTAs
-// (key tiles x heads x batch x groups) for about two per SM of a 148-SM B200.
+// Row groups for the deterministic d_pair_bias reduction: about one CTA
+// (key tile x head x batch x group) per SM of a 148-SM B200, in one wave.
 inline int num_groups(int64_t B, int64_t S, int64_t N, int64_t H) {
     const int64_t njt = (N + BK - 1) / BK;
     const int64_t base = njt * B * H;
     if (base <= 0 || S <= 0) return 1;
-    int64_t g = (2 * 148 + base - 1) / base;
+    int64_t g = 148 / base;
     if (g > S) g = S;
     if (g < 1) g = 1;
     const int64_t gsz = (S + g - 1) / g;       // rows per group; drop groups left empty
@@ -70,6 +76,7 @@ inline int num_groups(int64_t B, int64_t S, int64_t N, int64_t H) {
 struct MainParams {
     int B, S, N, H;
     int n_it;            // query tiles
+    int n_pad;           // n_it * BQ: row length of the padded row-term arrays
     int gsz;             // rows s per group
     float sc2;           // log2(e) / sqrt(C)
     float rs;            // 1 / sqrt(C)
@@ -86,6 +93,7 @@ template <bool HAS_MASK, bool HAS_BIAS>
 __global__ void __launch_bounds__(THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_doa,
+                    const __grid_constant__ CUtensorMap tm_dol,
                     const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_mask,
                     const __grid_constant__ CUtensorMap tm_nl, const __grid_constant__ CUtensorMap tm_d,
                     const MainParams p) {
@@ -137,6 +145,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_doa);
+        prefetch_tmap(&tm_dol);
         prefetch_tmap(&tm_nl); prefetch_tmap(&tm_d);
         if (HAS_BIAS) prefetch_tmap(&tm_bt);
         if (HAS_MASK) prefetch_tmap(&tm_mask);
@@ -170,15 +179,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t sb = base + OFF_ST + st * STB;
                     if (t >= 2) ok = mbar_wait(q_empty(st), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(q_full(st), 2 * TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 1024);
-                    tma_load_5d(sb, &tm_q, q_full(st), 0, i0, h, s, b);
-                    tma_load_5d(sb + TILE_BYTES, &tm_doa, q_full(st), 0, i0, h, s, b);
+                    mbar_arrive_expect_tx(q_full(st), 3 * TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 1024);
+                    tma_load_5d(sb + ST_Q, &tm_q, q_full(st), 0, i0, h, s, b);
+                    tma_load_5d(sb + ST_DOH, &tm_doa, q_full(st), 0, i0, h, s, b);
+                    tma_load_5d(sb + ST_DOL, &tm_dol, q_full(st), 0, i0, h, s, b);
                     if (HAS_BIAS) {
-                        tma_load_4d(sb + 2 * TILE_BYTES, &tm_bt, q_full(st), i0, j0, h, b);
-                        tma_load_4d(sb + 2 * TILE_BYTES + BT_BOX, &tm_bt, q_full(st), i0 + 64, j0, h, b);
+                        tma_load_4d(sb + ST_BT, &tm_bt, q_full(st), i0, j0, h, b);
+                        tma_load_4d(sb + ST_BT + BT_BOX, &tm_bt, q_full(st), i0 + 64, j0, h, b);
                     }
-                    tma_load_4d(sb + 2 * TILE_BYTES + 2 * BT_BOX, &tm_nl, q_full(st), i0, h, s, b);
-                    tma_load_4d(sb + 2 * TILE_BYTES + 2 * BT_BOX + 512, &tm_d, q_full(st), i0, h, s, b);
+                    tma_load_4d(sb + ST_NL, &tm_nl, q_full(st), i0, h, s, b);
+                    tma_load_4d(sb + ST_ND, &tm_d, q_full(st), i0, h, s, b);
                     ++q_issued[st];
                 }
             }
@@ -210,7 +220,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     mma_ss(tmem + TM_DPT, smem_desc(kb + TILE_BYTES + kk * 32, 16, 512, kSw64),
-                           smem_desc(sb + TILE_BYTES + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                           smem_desc(sb + ST_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    mma_ss(tmem + TM_DPT, smem_desc(kb + TILE_BYTES + kk * 32, 16, 512, kSw64),
+                           smem_desc(sb + ST_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
                 }
                 mma_commit(sdp_full);
                 return true;
@@ -228,13 +243,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t ds = base + OFF_DS;
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {   // dV_j += P^T dOa_i
-                    mma_ts(tmem + TM_DV, tmem + TM_PT + kk * 8, smem_desc(sb + TILE_BYTES + kk * 1024, TILE_BYTES, 512, kSw64),
+                    mma_ts(tmem + TM_DV, tmem + TM_PT + kk * 8, smem_desc(sb + ST_DOH + kk * 1024, TILE_BYTES, 512, kSw64),
                            ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {   // dK_j += dS^T Q_i
                     const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
-                    mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128), smem_desc(sb + kk * 1024, TILE_BYTES, 512, kSw64),
+                    mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128), smem_desc(sb + ST_Q + kk * 1024, TILE_BYTES, 512, kSw64),
                            ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
                 }
                 if (t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x16);
@@ -265,18 +280,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int j = j0 + r;
         const bool jvalid = j < p.N;
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-        const float sc2 = p.sc2;
+        const uint64_t SC2 = f2(p.sc2, p.sc2);
+        const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
         // this group's slab of the partial sums (the output itself when there is one group)
         float* part = p.part + ((int64_t)grp * p.B * p.H + (int64_t)b * p.H + h) * p.N * p.N;
         bool ok = true;
-        float m2 = 0.f;
+        uint64_t RB2 = 0;                        // per-key term: mask*log2e, or -inf for padded keys
 
-        // drain helpers -------------------------------------------------
-        auto drain_dq = [&](int t) -> bool {   // dQ rows of step t: lanes = queries
+        auto drain_dq = [&](int t) -> bool {     // dQ rows of step t: lanes = queries
             if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) return false;
             tc_fence_after();
             uint32_t v[16];
             tmem_ld16_sync(lane_addr + TM_DQ + wg * 16, v);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dq_free);
             const int si = t / ni, it = t - si * ni;
             const int i = it * BQ + r, s = s_begin + si;
             if (i < p.N) {
@@ -289,9 +307,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                                  : "memory");
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dq_free);
             return true;
         };
         auto drain_dkv = [&](int si) -> bool {   // dK (wg 0) / dV (wg 1) of row s: lanes = keys
@@ -299,6 +314,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             uint32_t v[32];
             tmem_ld32_sync(lane_addr + (wg == 0 ? TM_DK : TM_DV), v);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dkv_free);
             if (jvalid) {
                 const float f = wg == 0 ? p.rs : 1.0f;
                 __nv_bfloat16* dst = (wg == 0 ? p.dk : p.dv) + p.gs.off(b, s_begin + si, j, h);
@@ -312,9 +330,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     *reinterpret_cast<uint4*>(dst + 8 * q) = w;
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dkv_free);
             return true;
         };
 
@@ -324,71 +339,65 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (it == 0) {
                 ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x23);
                 if (!ok) break;
+                float rb = 0.f;
                 if (HAS_MASK) {
                     const uint16_t mb = *reinterpret_cast<const uint16_t*>(gbase + OFF_KV + x * KVB + 2 * TILE_BYTES + r * 2);
-                    m2 = __uint_as_float((uint32_t)mb << 16) * EVO_LOG2E;
+                    rb = __uint_as_float((uint32_t)mb << 16) * EVO_LOG2E;
                 }
+                if (!jvalid) rb = -INFINITY;
+                RB2 = f2(rb, rb);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(kv_empty(x));
             }
             ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[64], dp[64];
-            tmem_ld32_sync(lane_addr + TM_ST + wg * 64, sv);
-            tmem_ld32_sync(lane_addr + TM_ST + wg * 64 + 32, sv + 32);
-            tmem_ld32_sync(lane_addr + TM_DPT + wg * 64, dp);
-            tmem_ld32_sync(lane_addr + TM_DPT + wg * 64 + 32, dp + 32);
+            uint32_t sv[128];                    // [0,64): S^T columns, [64,128): dP^T columns
+            tmem_ld32x4_sync(lane_addr + TM_ST + wg * 64, lane_addr + TM_ST + wg * 64 + 32,
+                             lane_addr + TM_DPT + wg * 64, lane_addr + TM_DPT + wg * 64 + 32, sv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sdp_free);
 
-            if (t > 0) {
-                ok = drain_dq(t - 1);
-                if (ok && it == 0) ok = drain_dkv(si - 1);
-                if (!ok) break;
-            }
-
             ok = mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x25);
             if (!ok) break;
             const uint32_t sb = base + OFF_ST + st * STB;
-            const uint32_t nl_addr = sb + 2 * TILE_BYTES + 2 * BT_BOX + wg * 256;
-            const uint32_t d_addr = nl_addr + 512;
-            const uint32_t bt_addr = sb + 2 * TILE_BYTES + wg * BT_BOX + r * 128;
-            const int ivalid = min(64, p.N - i0 - wg * 64);   // queries of this half inside N
+            const uint32_t nl_addr = sb + ST_NL + wg * 256;
+            const uint32_t nd_addr = sb + ST_ND + wg * 256;
+            const uint32_t bt_addr = sb + ST_BT + wg * BT_BOX + r * 128;
+            // P = exp2(S*scale*log2e + bias*log2e + nl_i + rb_j), dS = P * (dP - D_i), two columns per op
             float dsf[64];
             uint32_t pk[32], dk2[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {                      // 8 columns at a time
-                float bt[8];
+                uint32_t bw[4] = {0u, 0u, 0u, 0u};
                 if (HAS_BIAS) {
                     const uint4 w = lds128(bt_addr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
-                    bt[0] = bf16lo(w.x); bt[1] = bf16hi(w.x); bt[2] = bf16lo(w.y); bt[3] = bf16hi(w.y);
-                    bt[4] = bf16lo(w.z); bt[5] = bf16hi(w.z); bt[6] = bf16lo(w.w); bt[7] = bf16hi(w.w);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) bt[e] = 0.f;
+                    bw[0] = w.x; bw[1] = w.y; bw[2] = w.z; bw[3] = w.w;
                 }
                 const uint4 n0 = lds128(nl_addr + q * 32), n1 = lds128(nl_addr + q * 32 + 16);
-                const uint4 d0 = lds128(d_addr + q * 32), d1 = lds128(d_addr + q * 32 + 16);
-                const float nl[8] = {__uint_as_float(n0.x), __uint_as_float(n0.y), __uint_as_float(n0.z), __uint_as_float(n0.w),
-                                     __uint_as_float(n1.x), __uint_as_float(n1.y), __uint_as_float(n1.z), __uint_as_float(n1.w)};
-                const float dd[8] = {__uint_as_float(d0.x), __uint_as_float(d0.y), __uint_as_float(d0.z), __uint_as_float(d0.w),
-                                     __uint_as_float(d1.x), __uint_as_float(d1.y), __uint_as_float(d1.z), __uint_as_float(d1.w)};
-                float pv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int c = q * 8 + e;
-                    const float xx = fmaf(__uint_as_float(sv[c]), sc2, fmaf(bt[e], EVO_LOG2E, m2 + nl[e]));
-                    float pe = ex2(xx);
-                    if (!jvalid || c >= ivalid) pe = 0.f;
-                    pv[e] = pe;
-                    dsf[c] = pe * (__uint_as_float(dp[c]) - dd[e]);
-                }
+                const uint4 d0 = lds128(nd_addr + q * 32), d1 = lds128(nd_addr + q * 32 + 16);
+                const uint64_t nl2[4] = {f2(__uint_as_float(n0.x), __uint_as_float(n0.y)),
+                                         f2(__uint_as_float(n0.z), __uint_as_float(n0.w)),
+                                         f2(__uint_as_float(n1.x), __uint_as_float(n1.y)),
+                                         f2(__uint_as_float(n1.z), __uint_as_float(n1.w))};
+                const uint64_t nd2[4] = {f2(__uint_as_float(d0.x), __uint_as_float(d0.y)),
+                                         f2(__uint_as_float(d0.z), __uint_as_float(d0.w)),
+                                         f2(__uint_as_float(d1.x), __uint_as_float(d1.y)),
+                                         f2(__uint_as_float(d1.z), __uint_as_float(d1.w))};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    pk[q * 4 + e] = pack_bf16(pv[2 * e], pv[2 * e + 1]);
-                    dk2[q * 4 + e] = pack_bf16(dsf[q * 8 + 2 * e], dsf[q * 8 + 2 * e + 1]);
+                    const int c = q * 8 + 2 * e;
+                    uint64_t t2 = HAS_BIAS ? ffma2(bf16x2_to_f2(bw[e]), L2E2, nl2[e]) : nl2[e];
+                    t2 = fadd2(t2, RB2);
+                    const uint64_t x2 = ffma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), SC2, t2);
+                    const float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));
+                    const uint64_t dd = fadd2(f2(__uint_as_float(sv[64 + c]), __uint_as_float(sv[65 + c])), nd2[e]);
+                    const uint64_t ds2 = fmul2(f2(p0, p1), dd);
+                    dsf[c] = f2lo(ds2);
+                    dsf[c + 1] = f2hi(ds2);
+                    pk[q * 4 + e] = pack_bf16(p0, p1);
+                    dk2[q * 4 + e] = pack_bf16(dsf[c], dsf[c + 1]);
                 }
             }
             __syncwarp();
@@ -412,18 +421,36 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(ds_full);
 
+            // The previous step's dQ and (at a row change) the previous row's dK/dV
+            // are drained here, after this step's exponentials, so the MMAs that
+            // produce them overlap this step's work.
+            if (t > 0) {
+                ok = drain_dq(t - 1);
+                if (ok && it == 0) ok = drain_dkv(si - 1);
+                if (!ok) break;
+            }
+
             // d_pair_bias partial (zeroed before the launch).  Each address of this
             // group's slab is updated by exactly one thread, in row order s, with
             // fire-and-forget atomic adds; same-thread atomics to one address are
             // performed in program order, so the sum is bitwise reproducible.
             if (jvalid) {
                 float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
+                const int ivalid = p.N - i0 - wg * 64;          // queries of this half inside N
+                if (ivalid >= 64) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c < ivalid)
+                    for (int c = 0; c < 64; ++c)
                         asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (int64_t)c * p.N),
                                      "f"(dsf[c])
                                      : "memory");
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c < ivalid)
+                            asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (int64_t)c * p.N),
+                                         "f"(dsf[c])
+                                         : "memory");
+                }
             }
         }
         if (ok) ok = drain_dq(T - 1);
@@ -440,20 +467,32 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ------------------------------------------------------------------ elementwise kernels
 struct PreParams {
-    int B, S, N, H;
+    int B, S, N, H, n_pad;
     const __nv_bfloat16* out; const __nv_bfloat16* dout; Strides os;
     const __nv_bfloat16* g; Strides in;
     const float* lse;
     __nv_bfloat16* dg; Strides gs;
-    __nv_bfloat16* doa;   // contiguous [B,S,N,H,C]
-    float* D;             // [B,S,H,N]
-    float* nl;            // [B,S,H,N]
-    float* dq_acc;        // contiguous [B,S,N,H,C] fp32
+    __nv_bfloat16* doa_hi;  // contiguous [B,S,N,H,C]
+    __nv_bfloat16* doa_lo;  // contiguous [B,S,N,H,C]: dOa - float(doa_hi), rounded
+    float* nd;              // [B,S,H,n_pad]: -D_i, 0 on padding
+    float* nl;              // [B,S,H,n_pad]: -lse_i * log2(e), -inf on padding
+    float* dq_acc;          // contiguous [B,S,N,H,C] fp32
 };
 
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
     const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t pads = (int64_t)p.B * p.S * p.H * (p.n_pad - p.N);
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows + pads;
+         t += (int64_t)gridDim.x * blockDim.x) {
+        if (t >= rows) {   // padded query slots of the row-term arrays
+            const int64_t u = t - rows;
+            const int w = p.n_pad - p.N;
+            const int64_t bsh = u / w;
+            const int i = p.N + (int)(u % w);
+            p.nl[bsh * p.n_pad + i] = -INFINITY;
+            p.nd[bsh * p.n_pad + i] = 0.f;
+            continue;
+        }
         const int h = (int)(t % p.H);
         const int i = (int)((t / p.H) % p.N);
         const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
@@ -462,14 +501,15 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
         const uint4* d4 = reinterpret_cast<const uint4*>(p.dout + p.os.off(b, s, i, h));
         const uint4* g4 = reinterpret_cast<const uint4*>(p.g + p.in.off(b, s, i, h));
         uint4* dg4 = reinterpret_cast<uint4*>(p.dg + p.gs.off(b, s, i, h));
-        uint4* da4 = reinterpret_cast<uint4*>(p.doa + t * HD);
+        uint4* hi4 = reinterpret_cast<uint4*>(p.doa_hi + t * HD);
+        uint4* lo4 = reinterpret_cast<uint4*>(p.doa_lo + t * HD);
         float D = 0.f;
 #pragma unroll
         for (int q = 0; q < HD / 8; ++q) {
             const uint4 ow = o4[q], dw = d4[q], gw = g4[q];
             const uint32_t ov[4] = {ow.x, ow.y, ow.z, ow.w}, dv[4] = {dw.x, dw.y, dw.z, dw.w},
                            gv[4] = {gw.x, gw.y, gw.z, gw.w};
-            uint32_t dgv[4], dav[4];
+            uint32_t dgv[4], hv[4], lv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float o0 = bf16lo(ov[e]), o1 = bf16hi(ov[e]);
@@ -478,14 +518,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
                 D = fmaf(d0, o0, D);
                 D = fmaf(d1, o1, D);
                 dgv[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
-                dav[e] = pack_bf16(d0 * s0, d1 * s1);
+                const float a0 = d0 * s0, a1 = d1 * s1;
+                hv[e] = pack_bf16(a0, a1);
+                lv[e] = pack_bf16(a0 - bf16lo(hv[e]), a1 - bf16hi(hv[e]));
             }
             dg4[q] = make_uint4(dgv[0], dgv[1], dgv[2], dgv[3]);
-            da4[q] = make_uint4(dav[0], dav[1], dav[2], dav[3]);
+            hi4[q] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            lo4[q] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
-        const int64_t ri = (((int64_t)b * p.S + s) * p.H + h) * p.N + i;
-        p.D[ri] = D;
-        p.nl[ri] = -p.lse[ri] * EVO_LOG2E;
+        const int64_t bsh = ((int64_t)b * p.S + s) * p.H + h;
+        p.nd[bsh * p.n_pad + i] = -D;
+        p.nl[bsh * p.n_pad + i] = -p.lse[bsh * p.N + i] * EVO_LOG2E;
         float4* acc = reinterpret_cast<float4*>(p.dq_acc + t * HD);
 #pragma unroll
         for (int q = 0; q < HD / 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -561,7 +604,7 @@ struct Call {
     evo_strides_t gs;
     float* dbias;
     char* ws;
-    size_t d_off, nl_off, doa_off, dqacc_off, biast_off, part_off;
+    size_t d_off, nl_off, doa_off, dol_off, dqacc_off, biast_off, part_off;
     int groups;
 };
 
@@ -577,7 +620,7 @@ inline cudaError_t launch_main(const CUtensorMap* m, const MainParams& mp, dim3 
     auto kern = bwd_main_kernel<HM, HB>;
     static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (attr != cudaSuccess) return attr;
-    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], mp);
+    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[8], m[4], m[5], m[6], m[7], mp);
     return cudaGetLastError();
 }
 
@@ -595,22 +638,24 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
         return EVO_ERR_UNSUPPORTED;
 
     const int B = (int)sh.B, S = (int)sh.S, N = (int)sh.N, H = (int)sh.H;
-    float* D = reinterpret_cast<float*>(c.ws + c.d_off);
+    const int n_pad = (N + BQ - 1) / BQ * BQ;
+    float* nd = reinterpret_cast<float*>(c.ws + c.d_off);
     float* nl = reinterpret_cast<float*>(c.ws + c.nl_off);
     __nv_bfloat16* doa = reinterpret_cast<__nv_bfloat16*>(c.ws + c.doa_off);
+    __nv_bfloat16* dol = reinterpret_cast<__nv_bfloat16*>(c.ws + c.dol_off);
     float* dq_acc = reinterpret_cast<float*>(c.ws + c.dqacc_off);
     __nv_bfloat16* biasT = reinterpret_cast<__nv_bfloat16*>(c.ws + c.biast_off);
     float* part = c.groups > 1 ? reinterpret_cast<float*>(c.ws + c.part_off) : c.dbias;
 
     const int64_t rows = (int64_t)B * S * N * H;
     PreParams pp{};
-    pp.B = B; pp.S = S; pp.N = N; pp.H = H;
+    pp.B = B; pp.S = S; pp.N = N; pp.H = H; pp.n_pad = n_pad;
     pp.out = static_cast<const __nv_bfloat16*>(c.out); pp.dout = static_cast<const __nv_bfloat16*>(c.dout);
     pp.os = Strides{c.os.b, c.os.s, c.os.n, c.os.h};
     pp.g = static_cast<const __nv_bfloat16*>(c.g); pp.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
     pp.lse = c.lse; pp.dg = static_cast<__nv_bfloat16*>(c.dg); pp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
-    pp.doa = doa; pp.D = D; pp.nl = nl; pp.dq_acc = dq_acc;
-    bwd_pre_kernel<<<grid_for(rows, 256), 256, 0, stream>>>(pp);
+    pp.doa_hi = doa; pp.doa_lo = dol; pp.nd = nd; pp.nl = nl; pp.dq_acc = dq_acc;
+    bwd_pre_kernel<<<grid_for(rows + (int64_t)B * S * H * (n_pad - N), 256), 256, 0, stream>>>(pp);
     ++*launched;
     if (c.bias) {
         transpose_bias_kernel<<<dim3((N + 31) / 32, (N + 31) / 32, B * H), dim3(32, 8), 0, stream>>>(
@@ -624,14 +669,15 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
 
     // tensor maps
     const evo_strides_t contig{(int64_t)S * N * H * HD, (int64_t)N * H * HD, (int64_t)H * HD, (int64_t)HD};
-    CUtensorMap m[8];
+    CUtensorMap m[9];
     std::memset(m, 0, sizeof(m));
     const evo_shape_t& s5 = sh;
     if (!tma::rows_bf16(&m[0], c.q, s5, c.in, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !tma::rows_bf16(&m[1], c.k, s5, c.in, BK, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !tma::rows_bf16(&m[2], c.v, s5, c.in, BK, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !tma::rows_bf16(&m[3], doa, s5, contig, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !tma::rowscalar_f32(&m[6], nl, s5) || !tma::rowscalar_f32(&m[7], D, s5))
+        !tma::rows_bf16(&m[8], dol, s5, contig, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !tma::rowscalar_f32(&m[6], nl, s5, n_pad) || !tma::rowscalar_f32(&m[7], nd, s5, n_pad))
         return EVO_ERR_CUDA;
     if (c.bias && !tma::square_bf16(&m[4], biasT, s5, BK)) return EVO_ERR_CUDA;
     if (c.mask && !tma::mask_bf16(&m[5], c.mask, s5)) return EVO_ERR_CUDA;
@@ -639,6 +685,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     MainParams mp{};
     mp.B = B; mp.S = S; mp.N = N; mp.H = H;
     mp.n_it = (N + BQ - 1) / BQ;
+    mp.n_pad = n_pad;
     const int G = c.groups;
     mp.gsz = (S + G - 1) / G;
     mp.sc2 = EVO_LOG2E / sqrtf((float)HD);

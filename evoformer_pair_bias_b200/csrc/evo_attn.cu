@@ -138,7 +138,7 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
 
 // ---------------------------------------------------------------- backward
 struct BwdWorkspace {
-    size_t d_off, nl_off, doa_off, dqacc_off, biast_off, part_off, total;
+    size_t d_off, nl_off, doa_off, dol_off, dqacc_off, biast_off, part_off, total;
     int groups;
 };
 
@@ -153,10 +153,15 @@ BwdWorkspace bwd_workspace(const evo_shape_t& sh, evo_dtype_t dt) {
     w.d_off = off;
     off = align256(off + rows * 4);
     if (dt == EVO_DTYPE_BF16) {
+        // row terms -D and nl are stored with the query axis padded to whole tiles
+        const size_t padded_rows = (size_t)sh.B * sh.S * sh.H * (size_t)((sh.N + 127) / 128 * 128);
+        off = align256(w.d_off + padded_rows * 4);
         w.groups = evo::bwd::num_groups(sh.B, sh.S, sh.N, sh.H);
         w.nl_off = off;
-        off = align256(off + rows * 4);
+        off = align256(off + padded_rows * 4);
         w.doa_off = off;
+        off = align256(off + T * 2);
+        w.dol_off = off;
         off = align256(off + T * 2);
         w.dqacc_off = off;
         off = align256(off + T * 4);
@@ -289,7 +294,8 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
     c.mask = mask_bias; c.bias = pair_bias; c.out = out; c.dout = dout; c.os = *out_str; c.lse = lse;
     c.dq = dq; c.dk = dk; c.dv = dv; c.dg = dg; c.gs = *grad_str; c.dbias = d_pair_bias;
     c.ws = static_cast<char*>(workspace);
-    c.d_off = ws.d_off; c.nl_off = ws.nl_off; c.doa_off = ws.doa_off; c.dqacc_off = ws.dqacc_off;
+    c.d_off = ws.d_off; c.nl_off = ws.nl_off; c.doa_off = ws.doa_off; c.dol_off = ws.dol_off;
+    c.dqacc_off = ws.dqacc_off;
     c.biast_off = ws.biast_off; c.part_off = ws.part_off; c.groups = ws.groups;
     int launched = 0;
     const evo_status_t rs = evo::bwd::run(c, s, &launched);

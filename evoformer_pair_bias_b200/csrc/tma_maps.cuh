@@ -86,9 +86,9 @@ inline bool mask_bf16(CUtensorMap* m, const void* ptr, const evo_shape_t& sh) {
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// fp32 per-row scalar [B,S,H,N] viewed as (i, h, s, b); box (128, 1, 1, 1).
-inline bool rowscalar_f32(CUtensorMap* m, const void* ptr, const evo_shape_t& sh) {
-    const uint64_t N = (uint64_t)sh.N, H = (uint64_t)sh.H, S = (uint64_t)sh.S;
+// fp32 per-row scalar [B,S,H,n_row] viewed as (i, h, s, b); box (128, 1, 1, 1).
+inline bool rowscalar_f32(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, int64_t n_row) {
+    const uint64_t N = (uint64_t)n_row, H = (uint64_t)sh.H, S = (uint64_t)sh.S;
     const uint64_t dims[4] = {N, H, S, (uint64_t)sh.B};
     const uint64_t str[3] = {N * 4, H * N * 4, S * H * N * 4};
     const uint32_t box[4] = {128, 1, 1, 1};
