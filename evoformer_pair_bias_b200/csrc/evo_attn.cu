@@ -89,16 +89,21 @@ evo_status_t fwd_f32(const evo_shape_t& sh, const void* q, const void* k, const 
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
 template <int NSUB, bool HM, bool HB>
-evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p, const evo_shape_t& sh,
-                             cudaStream_t stream) {
+evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p, cudaStream_t stream) {
     using L = evo::fwd::Layout<NSUB>;
     auto kern = evo::fwd::fwd_bf16_kernel<NSUB, HM, HB>;
     static cudaError_t attr = set_smem(kern, L::bytes);
     if (attr != cudaSuccess) return EVO_ERR_CUDA;
-    dim3 grid((unsigned)((sh.N + evo::fwd::BM - 1) / evo::fwd::BM), (unsigned)((sh.S + NSUB - 1) / NSUB),
-              (unsigned)(sh.B * sh.H));
-    kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    const int grid = std::min(p.n_items, sm_count());
+    kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
@@ -112,28 +117,33 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
     if (!strides_mult(&in, 8) || !strides_mult(&os, 8)) return EVO_ERR_UNSUPPORTED;
     for (const void* ptr : {q, k, v, g, (const void*)out}) if (!aligned(ptr, 16)) return EVO_ERR_UNSUPPORTED;
     if ((mask && !aligned(mask, 16)) || (bias && !aligned(bias, 16))) return EVO_ERR_UNSUPPORTED;
-    if ((sh.S + kFwdNsub - 1) / kFwdNsub > 65535) return EVO_ERR_UNSUPPORTED;
-    CUtensorMap maps[5];
+    const int64_t n_it = (sh.N + evo::fwd::BM - 1) / evo::fwd::BM;
+    const int64_t n_sg = (sh.S + kFwdNsub - 1) / kFwdNsub;
+    const int64_t n_items = sh.B * sh.H * n_sg * n_it;
+    if (n_items > (int64_t)1 << 30) return EVO_ERR_UNSUPPORTED;
+    CUtensorMap maps[6];
     std::memset(maps, 0, sizeof(maps));
     if (!evo::tma::rows_bf16(&maps[0], q, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !evo::tma::rows_bf16(&maps[1], k, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B))
+        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !evo::tma::rows_bf16(&maps[3], g, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B))
         return EVO_ERR_CUDA;
-    if (bias && !evo::tma::square_bf16(&maps[3], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
-    if (mask && !evo::tma::mask_bf16(&maps[4], mask, sh)) return EVO_ERR_CUDA;
+    if (bias && !evo::tma::square_bf16(&maps[4], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
+    if (mask && !evo::tma::mask_bf16(&maps[5], mask, sh)) return EVO_ERR_CUDA;
     evo::fwd::Params p{};
     p.B = (int)sh.B; p.S = (int)sh.S; p.N = (int)sh.N; p.H = (int)sh.H;
     p.n_kv = (int)((sh.N + evo::fwd::BN - 1) / evo::fwd::BN);
+    p.n_it = (int)n_it;
+    p.n_sg = (int)n_sg;
+    p.n_items = (int)n_items;
     p.scale = 1.0f / sqrtf((float)sh.C);
-    p.g = static_cast<const __nv_bfloat16*>(g);
-    p.in = to_strides(in);
     p.out = static_cast<__nv_bfloat16*>(out);
     p.os = to_strides(os);
     p.lse = lse;
-    if (mask && bias) return launch_fwd_bf16<kFwdNsub, true, true>(maps, p, sh, stream);
-    if (mask) return launch_fwd_bf16<kFwdNsub, true, false>(maps, p, sh, stream);
-    if (bias) return launch_fwd_bf16<kFwdNsub, false, true>(maps, p, sh, stream);
-    return launch_fwd_bf16<kFwdNsub, false, false>(maps, p, sh, stream);
+    if (mask && bias) return launch_fwd_bf16<kFwdNsub, true, true>(maps, p, stream);
+    if (mask) return launch_fwd_bf16<kFwdNsub, true, false>(maps, p, stream);
+    if (bias) return launch_fwd_bf16<kFwdNsub, false, true>(maps, p, stream);
+    return launch_fwd_bf16<kFwdNsub, false, false>(maps, p, stream);
 }
 
 // ---------------------------------------------------------------- backward

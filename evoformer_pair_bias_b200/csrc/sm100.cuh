@@ -292,11 +292,13 @@ __device__ __forceinline__ uint64_t f2(float lo, float hi) {
 __device__ __forceinline__ float f2lo(uint64_t v) {
     float lo, hi;
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    (void)hi;
     return lo;
 }
 __device__ __forceinline__ float f2hi(uint64_t v) {
     float lo, hi;
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    (void)lo;
     return hi;
 }
 __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
