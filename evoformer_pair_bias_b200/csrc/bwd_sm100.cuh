@@ -24,6 +24,9 @@
 //                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
 //                    d_pair_bias partial[g][i,j] += dS (atomic add; one thread
 //                    is the only writer of each address, rows s in order)
+//                  The dS^T smem tile and the P^T TMEM tile are double-buffered
+//                  by step parity, so the dS warps write step t while the MMAs of
+//                  step t-1 still read the other buffer.
 //   bwd_post       dq = bf16(accumulator); d_pair_bias = sum over g of the
 //                  partials in index order (skipped when there is one group).
 // The result of d_pair_bias is therefore bitwise reproducible; dq's last bits
@@ -50,15 +53,17 @@ constexpr int ST_Q = 0, ST_DOH = TILE_BYTES, ST_DOL = 2 * TILE_BYTES, ST_BT = 3 
 constexpr int ST_NL = 3 * TILE_BYTES + 2 * BT_BOX, ST_ND = ST_NL + 512;
 constexpr int OFF_KV = 0;
 constexpr int OFF_ST = 2 * KVB;
-constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tile, 2 boxes of 128 rows x 128 B
-constexpr int OFF_BAR = OFF_DS + 2 * BT_BOX;
-// kv_full[2] kv_empty[2] q_full[2] q_empty[2] sdp_full sdp_free ds_full ds_free
+constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tiles (2 buffers), each 2 boxes of 128 rows x 128 B
+constexpr int DS_BYTES = 2 * BT_BOX;
+constexpr int OFF_BAR = OFF_DS + 2 * DS_BYTES;
+// kv_full[2] kv_empty[2] q_full[2] q_empty[2] sdp_full sdp_free ds_full ds_free[2]
 // dq_full dq_free dkv_full dkv_free mma_done
-constexpr int NBARS = 17;
+constexpr int NBARS = 18;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr int THREADS = 320;                       // warp 0 TMA, warp 1 MMA, warps 2..9 dS
-constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 320, TM_DK = 352, TM_DQ = 384, TM_COLS = 512;
+// TMEM columns: S^T, dP^T, two P^T buffers (bf16 pairs), dV, dK, dQ accumulators
+constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 384, TM_DK = 416, TM_DQ = 448, TM_COLS = 512;
 
 // Row groups for the deterministic d_pair_bias reduction: about one CTA
 // (key tile x head x batch x group) per SM of a 148-SM B200, in one wave.
@@ -117,10 +122,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto q_full = [&](int x) { return bar0 + 8u * (4 + x); };
     auto q_empty = [&](int x) { return bar0 + 8u * (6 + x); };
     const uint32_t sdp_full = bar0 + 8u * 8, sdp_free = bar0 + 8u * 9;
-    const uint32_t ds_full = bar0 + 8u * 10, ds_free = bar0 + 8u * 11;
-    const uint32_t dq_full = bar0 + 8u * 12, dq_free = bar0 + 8u * 13;
-    const uint32_t dkv_full = bar0 + 8u * 14, dkv_free = bar0 + 8u * 15;
-    const uint32_t mma_done = bar0 + 8u * 16;
+    const uint32_t ds_full = bar0 + 8u * 10;
+    auto ds_free = [&](int x) { return bar0 + 8u * (11 + x); };
+    const uint32_t dq_full = bar0 + 8u * 13, dq_free = bar0 + 8u * 14;
+    const uint32_t dkv_full = bar0 + 8u * 15, dkv_free = bar0 + 8u * 16;
+    const uint32_t mma_done = bar0 + 8u * 17;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
 
@@ -134,7 +140,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(sdp_full, 1);
         mbar_init(sdp_free, 8);
         mbar_init(ds_full, 8);
-        mbar_init(ds_free, 1);
+        mbar_init(ds_free(0), 1);
+        mbar_init(ds_free(1), 1);
         mbar_init(dq_full, 1);
         mbar_init(dq_free, 8);
         mbar_init(dkv_full, 1);
@@ -240,10 +247,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
-                const uint32_t ds = base + OFF_DS;
+                const int db = t & 1;                    // dS^T / P^T buffer of this step
+                const uint32_t ds = base + OFF_DS + db * DS_BYTES;
+                const uint32_t pt = TM_PT + db * 64;
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk) {   // dV_j += P^T dOa_i
-                    mma_ts(tmem + TM_DV, tmem + TM_PT + kk * 8, smem_desc(sb + ST_DOH + kk * 1024, TILE_BYTES, 512, kSw64),
+                    mma_ts(tmem + TM_DV, tmem + pt + kk * 8, smem_desc(sb + ST_DOH + kk * 1024, TILE_BYTES, 512, kSw64),
                            ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
@@ -260,7 +269,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
                            smem_desc(kb + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(ds_free);
+                mma_commit(ds_free(db));
                 mma_commit(dq_full);
                 mma_commit(q_empty(st));
                 if (it == ni - 1) {
@@ -360,14 +369,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(sdp_free);
 
             ok = mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x25);
+            const int db = t & 1;                // dS^T / P^T buffer of this step
+            if (ok && t >= 2) ok = mbar_wait(ds_free(db), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
             if (!ok) break;
             const uint32_t sb = base + OFF_ST + st * STB;
             const uint32_t nl_addr = sb + ST_NL + wg * 256;
             const uint32_t nd_addr = sb + ST_ND + wg * 256;
             const uint32_t bt_addr = sb + ST_BT + wg * BT_BOX + r * 128;
+            const uint32_t ds_row = base + OFF_DS + db * DS_BYTES + wg * BT_BOX + r * 128;
+            // d_pair_bias partial (zeroed before the launch).  Each address of this
+            // group's slab is updated by exactly one thread, in row order s, with
+            // fire-and-forget atomic adds; same-thread atomics to one address are
+            // performed in program order, so the sum is bitwise reproducible.
+            const int ivalid = jvalid ? p.N - i0 - wg * 64 : 0;   // queries of this half inside N
+            float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
+            const int64_t rstride = p.N;
             // P = exp2(S*scale*log2e + bias*log2e + nl_i + rb_j), dS = P * (dP - D_i), two columns per op
-            float dsf[64];
-            uint32_t pk[32], dk2[32];
+            uint32_t pk[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {                      // 8 columns at a time
                 uint32_t bw[4] = {0u, 0u, 0u, 0u};
@@ -385,6 +403,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                                          f2(__uint_as_float(d0.z), __uint_as_float(d0.w)),
                                          f2(__uint_as_float(d1.x), __uint_as_float(d1.y)),
                                          f2(__uint_as_float(d1.z), __uint_as_float(d1.w))};
+                float dsq[8];
+                uint32_t dkq[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = q * 8 + 2 * e;
@@ -394,27 +414,34 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));
                     const uint64_t dd = fadd2(f2(__uint_as_float(sv[64 + c]), __uint_as_float(sv[65 + c])), nd2[e]);
                     const uint64_t ds2 = fmul2(f2(p0, p1), dd);
-                    dsf[c] = f2lo(ds2);
-                    dsf[c + 1] = f2hi(ds2);
+                    dsq[2 * e] = f2lo(ds2);
+                    dsq[2 * e + 1] = f2hi(ds2);
                     pk[q * 4 + e] = pack_bf16(p0, p1);
-                    dk2[q * 4 + e] = pack_bf16(dsf[c], dsf[c + 1]);
+                    dkq[e] = pack_bf16(dsq[2 * e], dsq[2 * e + 1]);
+                }
+                const uint32_t addr = ds_row + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dkq[0]), "r"(dkq[1]),
+                             "r"(dkq[2]), "r"(dkq[3])
+                             : "memory");
+                if (ivalid >= 64) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (q * 8 + e) * rstride),
+                                     "f"(dsq[e])
+                                     : "memory");
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (q * 8 + e < ivalid)
+                            asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (q * 8 + e) * rstride),
+                                         "f"(dsq[e])
+                                         : "memory");
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(q_empty(st));           // bias / nl / D of this stage consumed
-
-            if (t > 0) ok = mbar_wait(ds_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x26);
-            if (!ok) break;
             tc_fence_after();
-            tmem_st32(lane_addr + TM_PT + wg * 32, pk);
-            const uint32_t ds_row = base + OFF_DS + wg * BT_BOX + r * 128;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint32_t addr = ds_row + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk2[4 * q]),
-                             "r"(dk2[4 * q + 1]), "r"(dk2[4 * q + 2]), "r"(dk2[4 * q + 3])
-                             : "memory");
-            }
+            tmem_st32(lane_addr + TM_PT + db * 64 + wg * 32, pk);
             tc_wait_st();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
@@ -428,29 +455,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ok = drain_dq(t - 1);
                 if (ok && it == 0) ok = drain_dkv(si - 1);
                 if (!ok) break;
-            }
-
-            // d_pair_bias partial (zeroed before the launch).  Each address of this
-            // group's slab is updated by exactly one thread, in row order s, with
-            // fire-and-forget atomic adds; same-thread atomics to one address are
-            // performed in program order, so the sum is bitwise reproducible.
-            if (jvalid) {
-                float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
-                const int ivalid = p.N - i0 - wg * 64;          // queries of this half inside N
-                if (ivalid >= 64) {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (int64_t)c * p.N),
-                                     "f"(dsf[c])
-                                     : "memory");
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (c < ivalid)
-                            asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (int64_t)c * p.N),
-                                         "f"(dsf[c])
-                                         : "memory");
-                }
             }
         }
         if (ok) ok = drain_dq(T - 1);

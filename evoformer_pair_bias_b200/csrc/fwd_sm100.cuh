@@ -399,7 +399,6 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             tmem_ld32_sync(lane_addr + COL_O, o);
             const int i = itm.i0 + r;
             if (s < p.S && i < p.N) {
-                const float inv_l = 1.0f / l;
                 // gate row r of the g tile (64-byte rows, 64B swizzle: chunk ^= (row >> 1) & 3)
                 const uint32_t grow = base + L::gbuf(qb, u) + r * 64;
                 __nv_bfloat16* op = p.out + p.os.off(itm.b, s, i, itm.h);
@@ -410,12 +409,11 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     uint32_t ov[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        // sigmoid(g) = 0.5 + 0.5 * tanh(g / 2)
-                        float t0, t1;
-                        asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(0.5f * bf16lo(gv[e])));
-                        asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(0.5f * bf16hi(gv[e])));
-                        const float o0 = __uint_as_float(o[q * 8 + 2 * e]) * inv_l * fmaf(0.5f, t0, 0.5f);
-                        const float o1 = __uint_as_float(o[q * 8 + 2 * e + 1]) * inv_l * fmaf(0.5f, t1, 0.5f);
+                        // out = O / (l * (1 + exp(-g))): the backward's D = sum(dout * out)
+                        // feeds a cancellation, so the gate is computed accurately.
+                        const float e0 = ex2(-EVO_LOG2E * bf16lo(gv[e])), e1 = ex2(-EVO_LOG2E * bf16hi(gv[e]));
+                        const float o0 = __fdividef(__uint_as_float(o[q * 8 + 2 * e]), l * (1.0f + e0));
+                        const float o1 = __fdividef(__uint_as_float(o[q * 8 + 2 * e + 1]), l * (1.0f + e1));
                         ov[e] = pack_bf16(o0, o1);
                     }
                     *reinterpret_cast<uint4*>(op + q * 8) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
