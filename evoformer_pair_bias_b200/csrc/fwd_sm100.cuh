@@ -5,24 +5,34 @@
 // NSUB consecutive rows s (MSA sequences or pair rows).  The key axis is
 // streamed in 128-key tiles; no logit ever leaves TMEM/registers (the
 // flash-style, online-softmax treatment EvoFlash-3D gives this op in the
-// MegaFold summary, section "EvoFlash-3D").  The pair-bias tile of
-// (h, i-tile, j-tile) is the same for every row s, so one TMA load of it
-// serves all NSUB softmax warpgroups.
+// MegaFold summary, section "EvoFlash-3D").
 //
-// Warp roles (64 + 128*NSUB threads):
-//   warp 0   TMA producer: per item Q and the gate g (double-buffered by item
-//            parity), then per key tile K, V (per row s), the pair-bias tile
-//            and the mask row into a 2-stage ring that runs across items.
-//   warp 1   TMEM owner and MMA issuer (one lane):
-//              S_u  = Q_u K_u^T     (M=128, N=128, K=32)          -> TMEM
-//              O_u += P_u V_u       (M=128, N=32,  K=128, P in TMEM)
-//            The S MMA of the next tile (and of the next item) is issued
-//            before the PV MMA of the current one, so it overlaps softmax.
-//   warps 2+ one 4-warp softmax group per row s (thread = query row): load S
-//            from TMEM, add scale/bias/mask, online max and sum in fp32 with a
-//            lazy rescale (the running max moves only when a tile's max
-//            exceeds it by more than 2^8), P (bf16) back to TMEM, and at the
-//            end of the item out = sigmoid(g) * O / l, lse = log(l) + max.
+// The biases are added by the tensor core, not by the softmax threads:
+//   S_u = Q_u K_u^T + (r I) B + (r e_0) m_u^T,        r = bf16(sqrt(C))
+// accumulates, in fp32 TMEM, the logits scaled by sqrt(C): I is a constant
+// identity tile, B the pair-bias tile (TMA-loaded once per key tile and shared
+// by all NSUB rows s -- it is the same for every s), and the last term is one
+// 16-deep K step whose B block carries the mask row of row s in its first
+// row.  Products with the exact bf16 inputs are exact in fp32, so the biases
+// enter with only the relative error of r/sqrt(C) (1.1e-4 for C = 32; exact
+// for C = 16 or 64).  The softmax threads then need one fused multiply-add
+// per logit before the exponential.
+//
+// Warp roles (128*NSUB + 128 threads; the last warpgroup gives up registers
+// to the softmax warpgroups with setmaxnreg):
+//   warps 0 .. 4*NSUB-1   one 4-warp softmax group per row s (see below)
+//   warp 4*NSUB           TMA producer: per item Q (double-buffered by item
+//            parity), then per key tile K, V and the mask row (per row s) and
+//            the pair-bias tile into a 2-stage ring that runs across items.
+//   warp 4*NSUB+1         TMEM owner and MMA issuer (one lane): S_u as above
+//            (M=128, N=128), then O_u += P_u V_u (M=128, N=32, K=128, P read
+//            from TMEM).  The S MMAs of the next tile are issued before the PV
+//            of the current one, so they overlap the softmax.
+//   softmax: thread = query row.  Load S
+//            from TMEM, online max and sum in fp32 with a lazy rescale (the
+//            running max moves only when a tile's max exceeds it by more than
+//            2^8), P (bf16) back to TMEM, and at the end of the item
+//            out = sigmoid(g) * O / l, lse = log(l) + max.
 // TMEM per row s: S 128 columns, P 64 columns (bf16 pairs), O 32 columns.
 #pragma once
 
@@ -41,7 +51,9 @@ constexpr int Q_BYTES = BM * HD * 2;    // 8 KB, 64-byte rows, 64B swizzle
 constexpr int KV_BYTES = BN * HD * 2;   // 8 KB each for K and V
 constexpr int BIAS_BOX = BM * 64 * 2;   // 16 KB: 128 rows x 64 keys, 128B swizzle
 constexpr int BIAS_BYTES = 2 * BIAS_BOX;
-constexpr int MASK_BYTES = BN * 2;
+constexpr int MASKB_BYTES = 4096;       // 16 x 128 bf16 B block (row 0 = mask row), 128B swizzle
+constexpr int IDENT_BYTES = 128 * 128 * 2;   // r * I, K-major, no swizzle
+constexpr int ONES_BYTES = 128 * 16 * 2;     // r * e_0 column, K-major, no swizzle
 constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192, SUBCOLS = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
 
@@ -49,22 +61,28 @@ __host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / 
 
 template <int NSUB>
 struct Layout {
-    // per item parity: Q tiles then gate tiles
-    static constexpr int qbuf(int k, int u) { return (k * 2 * NSUB + u) * Q_BYTES; }
-    static constexpr int gbuf(int k, int u) { return (k * 2 * NSUB + NSUB + u) * Q_BYTES; }
-    static constexpr int stage0 = 4 * NSUB * Q_BYTES;
+    static constexpr int qbuf(int k, int u) { return (k * NSUB + u) * Q_BYTES; }   // per item parity k
+    static constexpr int ident = 2 * NSUB * Q_BYTES;
+    static constexpr int ones = ident + IDENT_BYTES;
+    static constexpr int stage0 = round_up(ones + ONES_BYTES, 1024);
     static constexpr int k_off(int u) { return u * KV_BYTES; }
     static constexpr int v_off(int u) { return (NSUB + u) * KV_BYTES; }
     static constexpr int bias_off = 2 * NSUB * KV_BYTES;
-    static constexpr int mask_off(int u) { return bias_off + BIAS_BYTES + u * MASK_BYTES; }
-    static constexpr int stage_bytes = round_up(bias_off + BIAS_BYTES + NSUB * MASK_BYTES, 1024);
+    static constexpr int maskb_off(int u) { return bias_off + BIAS_BYTES + u * MASKB_BYTES; }
+    static constexpr int stage_bytes = round_up(bias_off + BIAS_BYTES + NSUB * MASKB_BYTES, 1024);
     static constexpr int bars = stage0 + STAGES * stage_bytes;
     // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[u], s_free[u], p_full[u], o_full[u], mma_done
     static constexpr int nbars = 4 + 2 * STAGES + 4 * NSUB + 1;
     static constexpr int misc = bars + nbars * 8;   // tmem base (u32), abort flag (u32)
     static constexpr int bytes = misc + 16 + 1024;  // + slack to align the base to 1024
     static constexpr uint32_t tmem_cols = NSUB == 1 ? 256 : 512;
-    static constexpr int threads = 64 + 128 * NSUB;
+    static constexpr int threads = 128 * NSUB + 128;
+    // register split: launch count (65536 / threads, rounded down to 8) and the
+    // per-warpgroup counts after setmaxnreg; softmax + control <= launch pool
+    static constexpr int launch_regs = (65536 / threads) / 8 * 8;
+    static constexpr uint32_t softmax_regs = NSUB == 2 ? 208 : 240;
+    static constexpr uint32_t control_regs = 88;
+    static_assert((int)(NSUB * softmax_regs + control_regs) * 128 <= launch_regs * threads, "register split");
 };
 
 struct Params {
@@ -74,6 +92,9 @@ struct Params {
     int n_sg;                 // row groups of NSUB rows
     int n_items;              // B * H * n_sg * n_it
     float scale;              // 1/sqrt(C)
+    float r_bf16;             // bf16(sqrt(C)), the diagonal of the identity tile
+    const __nv_bfloat16* g;   // gate, strides `in`
+    Strides in;
     __nv_bfloat16* out;       // strides `os`
     Strides os;
     float* lse;               // [B,S,H,N]
@@ -102,9 +123,8 @@ enum : unsigned int { kTimeoutBase = 0x1000u };
 template <int NSUB, bool HAS_MASK, bool HAS_BIAS>
 __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                    const __grid_constant__ CUtensorMap tm_bias, const __grid_constant__ CUtensorMap tm_mask,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
+                    const __grid_constant__ CUtensorMap tm_mask, const Params p) {
     using L = Layout<NSUB>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -112,6 +132,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kProducer = 4 * NSUB, kMma = 4 * NSUB + 1;
 
     const uint32_t bar0 = base + L::bars;
     auto q_full = [&](int x) { return bar0 + 8u * (0 + x); };
@@ -129,11 +150,11 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(q_full(x), 1);
-            mbar_init(q_empty(x), 1 + 4 * NSUB);
+            mbar_init(q_empty(x), 1);
         }
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(kv_full(st), 1);
-            mbar_init(kv_empty(st), 1 + 4 * NSUB);
+            mbar_init(kv_empty(st), 1);
         }
         for (int u = 0; u < NSUB; ++u) {
             mbar_init(s_full(u), 1);
@@ -145,27 +166,54 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == kProducer && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        prefetch_tmap(&tm_g);
         if (HAS_BIAS) prefetch_tmap(&tm_bias);
         if (HAS_MASK) prefetch_tmap(&tm_mask);
     }
-    if (warp == 1) {
+    if (warp == kMma) {
         tmem_alloc(base + L::misc, L::tmem_cols);
         tmem_relinquish();
+    }
+    if (warp < 4 * NSUB) {
+        // Constant MMA operands (element (row, k) of a no-swizzle K-major tile is
+        // at (row % 8) * 16 + (row / 8) * SBO + (k / 8) * 128 + (k % 8) * 2):
+        //   identity r*I (SBO 2048), column r*e_0 (SBO 256), and rows 1..15 of
+        //   every mask block zero (the TMA writes row 0 each stage).
+        const int t = threadIdx.x;
+        const int nt = 128 * NSUB;
+        const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
+        for (int o = t * 16; o < IDENT_BYTES; o += nt * 16)
+            *reinterpret_cast<uint4*>(gbase + L::ident + o) = make_uint4(0u, 0u, 0u, 0u);
+        for (int o = t * 16; o < ONES_BYTES; o += nt * 16)
+            *reinterpret_cast<uint4*>(gbase + L::ones + o) = make_uint4(0u, 0u, 0u, 0u);
+        for (int st = 0; st < STAGES; ++st)
+            for (int u = 0; u < NSUB; ++u)
+                for (int o = t * 16; o < MASKB_BYTES; o += nt * 16)
+                    *reinterpret_cast<uint4*>(gbase + L::stage0 + st * L::stage_bytes + L::maskb_off(u) + o) =
+                        make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+        asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");
+        if (t < 128) {
+            const int rr = t;
+            *reinterpret_cast<uint16_t*>(gbase + L::ident + (rr % 8) * 16 + (rr / 8) * 2048 + (rr / 8) * 128 +
+                                         (rr % 8) * 2) = rb;
+            *reinterpret_cast<uint16_t*>(gbase + L::ones + (rr % 8) * 16 + (rr / 8) * 256) = rb;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == kProducer) {
+        regs_decrease<L::control_regs>();
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            constexpr uint32_t tx = 2 * NSUB * KV_BYTES + (HAS_BIAS ? BIAS_BYTES : 0) + (HAS_MASK ? NSUB * MASK_BYTES : 0);
+            constexpr uint32_t tx = 2 * NSUB * KV_BYTES + (HAS_BIAS ? BIAS_BYTES : 0) + (HAS_MASK ? NSUB * 256 : 0);
             int q_issued[2] = {0, 0}, kv_issued[STAGES] = {};
             int tg = 0;
             bool ok = true;
@@ -178,12 +226,10 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 const int qb = k & 1;
                 if (k >= 2) ok = mbar_wait(q_empty(qb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x001);
                 if (!ok) break;
-                mbar_arrive_expect_tx(q_full(qb), 2 * NSUB * Q_BYTES);
+                mbar_arrive_expect_tx(q_full(qb), NSUB * Q_BYTES);
 #pragma unroll
-                for (int u = 0; u < NSUB; ++u) {
+                for (int u = 0; u < NSUB; ++u)
                     tma_load_5d(base + L::qbuf(qb, u), &tm_q, q_full(qb), 0, itm.i0, itm.h, s_ld[u], itm.b);
-                    tma_load_5d(base + L::gbuf(qb, u), &tm_g, q_full(qb), 0, itm.i0, itm.h, s_ld[u], itm.b);
-                }
                 ++q_issued[qb];
                 for (int j = 0; j < p.n_kv; ++j, ++tg) {
                     const int st = tg % STAGES;
@@ -203,8 +249,10 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     }
                     if (HAS_MASK) {
 #pragma unroll
-                        for (int u = 0; u < NSUB; ++u)
-                            tma_load_3d(sb + L::mask_off(u), &tm_mask, kv_full(st), j * BN, s_ld[u], itm.b);
+                        for (int u = 0; u < NSUB; ++u) {
+                            tma_load_3d(sb + L::maskb_off(u), &tm_mask, kv_full(st), j * BN, s_ld[u], itm.b);
+                            tma_load_3d(sb + L::maskb_off(u) + 2048, &tm_mask, kv_full(st), j * BN + 64, s_ld[u], itm.b);
+                        }
                     }
                     ++kv_issued[st];
                 }
@@ -216,10 +264,12 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             for (int st = 0; st < STAGES; ++st)
                 if (kv_issued[st]) mbar_wait(kv_full(st), (kv_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x004);
         }
-    } else if (warp == 1) {
+    } else if (warp == kMma) {
+        regs_decrease<L::control_regs>();
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
+            constexpr uint32_t IDESC_BIAS = idesc_bf16(BM, BN, false, true);   // B operand MN-major
             constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, false, true);
             bool ok = true;
             int tg = 0;
@@ -260,6 +310,19 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                             const uint64_t bd = smem_desc(sb + L::k_off(u) + kk * 32, 16, 512, kSw64);
                             mma_ss(tmem + u * SUBCOLS + COL_S, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
                         }
+                        if (HAS_BIAS) {
+#pragma unroll
+                            for (int kk = 0; kk < BM / 16; ++kk) {   // + r * bias[i, j]
+                                const uint64_t ad = smem_desc(base + L::ident + kk * 256, 128, 2048, kSwNone);
+                                const uint64_t bd = smem_desc(sb + L::bias_off + kk * 2048, BIAS_BOX, 1024, kSw128);
+                                mma_ss(tmem + u * SUBCOLS + COL_S, ad, bd, IDESC_BIAS, 1u);
+                            }
+                        }
+                        if (HAS_MASK) {                               // + r * mask[s, j]
+                            const uint64_t ad = smem_desc(base + L::ones, 128, 256, kSwNone);
+                            const uint64_t bd = smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128);
+                            mma_ss(tmem + u * SUBCOLS + COL_S, ad, bd, IDESC_BIAS, 1u);
+                        }
                         mma_commit(s_full(u));
                     }
                     if (ok && pending) ok = issue_pv();
@@ -276,26 +339,35 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             volatile int no_abort = 0;
             mbar_wait(bar_mma_done, 0, &no_abort, kTimeoutBase | 0x105);
         }
-    } else {
+    } else if (warp < 4 * NSUB) {
+        regs_increase<L::softmax_regs>();
         // ------------------------------------------------------------ softmax
-        const int u = (warp - 2) >> 2;
+        const int u = warp >> 2;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;          // query row within the tile = TMEM lane
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + u * SUBCOLS;
-        const uint64_t SCALE2 = f2(p.scale, p.scale);
-        const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
+        // S holds sqrt(C) * x; exponents are taken as exp2(S * sc2 - ms), sc2 = log2(e)/sqrt(C)
+        const float sc2 = p.scale * EVO_LOG2E;
+        const uint64_t SC2 = f2(sc2, sc2);
         bool ok = true;
         int tg = 0;
         for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
             const Item itm = decode(p, item);
             const int s = itm.sg * NSUB + u;
-            const int qb = k & 1;
+            const int i = itm.i0 + r;
+            const bool row_ok = s < p.S && i < p.N;
+            (void)k;
+            uint4 gw[HD / 8];
             // ms: running max in log2 units (the value subtracted inside exp2);
-            // l: running sum of exp2(x*log2e - ms)
+            // l: running sum of exp2(S * sc2 - ms)
             float ms = -INFINITY, l = 0.f;
             for (int j = 0; j < p.n_kv; ++j, ++tg) {
-                const int st = tg % STAGES;
-                const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
+                if (j == p.n_kv - 1 && row_ok) {
+                    // the gate row is only needed at the end of the item: fetch it during the last tile
+                    const uint4* gp = reinterpret_cast<const uint4*>(p.g + p.in.off(itm.b, s, i, itm.h));
+#pragma unroll
+                    for (int q = 0; q < HD / 8; ++q) gw[q] = __ldg(gp + q);
+                }
                 ok = mbar_wait(s_full(u), tg & 1, abort_flag, kTimeoutBase | 0x201);
                 if (!ok) break;
                 tc_fence_after();
@@ -304,54 +376,25 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_free(u));
-                ok = mbar_wait(kv_full(st), (tg / STAGES) & 1, abort_flag, kTimeoutBase | 0x202);
-                if (!ok) break;
 
-                // x = S/sqrt(C) + pair_bias[i, j] + mask_bias[s, j] (natural-log units), two columns per op
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int q = 0; q < BN / 8; ++q) {
-                    uint32_t bw[4] = {0u, 0u, 0u, 0u}, mw[4] = {0u, 0u, 0u, 0u};
-                    if (HAS_BIAS) {
-                        const uint32_t chunk = (uint32_t)(q & 7) ^ (uint32_t)(r & 7);
-                        const uint4 w = lds128(sb + L::bias_off + (q >> 3) * BIAS_BOX + r * 128 + (chunk << 4));
-                        bw[0] = w.x; bw[1] = w.y; bw[2] = w.z; bw[3] = w.w;
-                    }
-                    if (HAS_MASK) {
-                        const uint4 w = lds128(sb + L::mask_off(u) + q * 16);
-                        mw[0] = w.x; mw[1] = w.y; mw[2] = w.z; mw[3] = w.w;
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = q * 8 + 2 * e;
-                        uint64_t add2 = 0;
-                        if (HAS_BIAS && HAS_MASK) add2 = fadd2(bf16x2_to_f2(bw[e]), bf16x2_to_f2(mw[e]));
-                        else if (HAS_BIAS) add2 = bf16x2_to_f2(bw[e]);
-                        else if (HAS_MASK) add2 = bf16x2_to_f2(mw[e]);
-                        const uint64_t x2 = ffma2(f2(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), SCALE2, add2);
-                        const float x0 = f2lo(x2), x1 = f2hi(x2);
-                        xr[c] = __float_as_uint(x0);
-                        xr[c + 1] = __float_as_uint(x1);
-                        float m3;
-                        asm("max.f32 %0, %1, %2, %3;" : "=f"(m3) : "f"(mx[e]), "f"(x0), "f"(x1));
-                        mx[e] = m3;
-                    }
-                }
-                float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                 const int valid = p.N - j * BN;      // keys beyond N are padding: exclude them
                 if (valid < BN) {
-                    mloc = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) {
+                    for (int c = 0; c < BN; ++c)
                         if (c >= valid) xr[c] = __float_as_uint(-INFINITY);
-                        mloc = fmaxf(mloc, __uint_as_float(xr[c]));
-                    }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(kv_empty(st));   // done reading bias / mask of this stage
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < BN; c += 2) {
+                    float m3;
+                    asm("max.f32 %0, %1, %2, %3;" : "=f"(m3)
+                        : "f"(mx[(c >> 1) & 3]), "f"(__uint_as_float(xr[c])), "f"(__uint_as_float(xr[c + 1])));
+                    mx[(c >> 1) & 3] = m3;
+                }
+                const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 
                 // lazy rescale: move the running max only when this tile's max exceeds it by > 2^8
-                const float mcand = mloc * EVO_LOG2E;
+                const float mcand = mloc * sc2;
                 const bool move = mcand > ms + RESCALE_THRESHOLD;
                 const float ms_new = move ? mcand : ms;
                 const float alpha = move ? ex2(ms - ms_new) : 1.0f;   // 0 on an item's first tile
@@ -370,20 +413,24 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 }
                 const uint64_t NEG_MS2 = f2(-ms_new, -ms_new);
                 uint64_t rs2[2] = {0, 0};
-                uint32_t pk[BN / 2];
 #pragma unroll
-                for (int c = 0; c < BN / 2; ++c) {
-                    const uint64_t y2 = ffma2(f2(__uint_as_float(xr[2 * c]), __uint_as_float(xr[2 * c + 1])), L2E2, NEG_MS2);
-                    const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
-                    const uint64_t pp = f2(p0, p1);
-                    rs2[c & 1] = (c < 2) ? pp : fadd2(rs2[c & 1], pp);
-                    pk[c] = pack_bf16(p0, p1);
+                for (int half = 0; half < 2; ++half) {     // P stored 32 columns (64 keys) at a time
+                    uint32_t pk[BN / 4];
+#pragma unroll
+                    for (int cc = 0; cc < BN / 4; ++cc) {
+                        const int c = half * (BN / 4) + cc;
+                        const uint64_t y2 =
+                            ffma2(f2(__uint_as_float(xr[2 * c]), __uint_as_float(xr[2 * c + 1])), SC2, NEG_MS2);
+                        const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
+                        const uint64_t pp = f2(p0, p1);
+                        rs2[c & 1] = (c < 2) ? pp : fadd2(rs2[c & 1], pp);
+                        pk[cc] = pack_bf16(p0, p1);
+                    }
+                    tmem_st32(lane_addr + COL_P + half * 32, pk);
                 }
                 const uint64_t rsum = fadd2(rs2[0], rs2[1]);
                 l = fmaf(l, alpha, f2lo(rsum) + f2hi(rsum));
                 ms = ms_new;
-                tmem_st32(lane_addr + COL_P, pk);
-                tmem_st32(lane_addr + COL_P + 32, pk + 32);
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -392,20 +439,15 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             if (!ok) break;
             // ---------------------------------------------------------- epilogue of this item
             ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x204);
-            if (ok) ok = mbar_wait(q_full(qb), (k >> 1) & 1, abort_flag, kTimeoutBase | 0x205);
             if (!ok) break;
             tc_fence_after();
             uint32_t o[HD];
             tmem_ld32_sync(lane_addr + COL_O, o);
-            const int i = itm.i0 + r;
-            if (s < p.S && i < p.N) {
-                // gate row r of the g tile (64-byte rows, 64B swizzle: chunk ^= (row >> 1) & 3)
-                const uint32_t grow = base + L::gbuf(qb, u) + r * 64;
+            if (row_ok) {
                 __nv_bfloat16* op = p.out + p.os.off(itm.b, s, i, itm.h);
 #pragma unroll
                 for (int q = 0; q < HD / 8; ++q) {
-                    const uint4 gw = lds128(grow + ((((uint32_t)q) ^ ((uint32_t)(r >> 1) & 3u)) << 4));
-                    const uint32_t gv[4] = {gw.x, gw.y, gw.z, gw.w};
+                    const uint32_t gv[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
                     uint32_t ov[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -420,15 +462,15 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 }
                 p.lse[((int64_t)(itm.b * p.S + s) * p.H + itm.h) * p.N + i] = (ms + __log2f(l)) * EVO_LN2;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(q_empty(qb));   // gate tile consumed, O read out
         }
     }
 
+    else {
+        regs_decrease<L::control_regs>();
+    }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMma) {
         tc_fence_after();
         tmem_dealloc(tmem, L::tmem_cols);
     }

@@ -77,12 +77,12 @@ inline bool square_bf16(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, 
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// bf16 mask_bias [B,S,1,1,N] viewed as (j, s, b); box (128, 1, 1).
-inline bool mask_bf16(CUtensorMap* m, const void* ptr, const evo_shape_t& sh) {
+// bf16 mask_bias [B,S,1,1,N] viewed as (j, s, b); box (keys, 1, 1).
+inline bool mask_bf16(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, uint32_t keys = 128) {
     const uint64_t N = (uint64_t)sh.N, S = (uint64_t)sh.S;
     const uint64_t dims[3] = {N, S, (uint64_t)sh.B};
     const uint64_t str[2] = {N * 2, S * N * 2};
-    const uint32_t box[3] = {128, 1, 1};
+    const uint32_t box[3] = {keys, 1, 1};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
