@@ -102,8 +102,15 @@ evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p,
     auto kern = evo::fwd::fwd_bf16_kernel<NSUB, HM, HB>;
     static cudaError_t attr = set_smem(kern, L::bytes);
     if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    // The kernel's setmaxnreg split assumes exactly L::launch_regs registers per
+    // thread at launch; any other count could make the increase wait forever.
+    static int regs = [&] {
+        cudaFuncAttributes fa{};
+        return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
+    }();
+    if (regs != L::launch_regs) return EVO_ERR_UNSUPPORTED;
     const int grid = std::min(p.n_items, sm_count());
-    kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+    kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
@@ -121,15 +128,14 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
     const int64_t n_sg = (sh.S + kFwdNsub - 1) / kFwdNsub;
     const int64_t n_items = sh.B * sh.H * n_sg * n_it;
     if (n_items > (int64_t)1 << 30) return EVO_ERR_UNSUPPORTED;
-    CUtensorMap maps[6];
+    CUtensorMap maps[5];
     std::memset(maps, 0, sizeof(maps));
     if (!evo::tma::rows_bf16(&maps[0], q, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !evo::tma::rows_bf16(&maps[1], k, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !evo::tma::rows_bf16(&maps[3], g, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B))
+        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B))
         return EVO_ERR_CUDA;
-    if (bias && !evo::tma::square_bf16(&maps[4], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
-    if (mask && !evo::tma::mask_bf16(&maps[5], mask, sh)) return EVO_ERR_CUDA;
+    if (bias && !evo::tma::square_bf16(&maps[3], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
+    if (mask && !evo::tma::mask_bf16(&maps[4], mask, sh, 64)) return EVO_ERR_CUDA;
     evo::fwd::Params p{};
     p.B = (int)sh.B; p.S = (int)sh.S; p.N = (int)sh.N; p.H = (int)sh.H;
     p.n_kv = (int)((sh.N + evo::fwd::BN - 1) / evo::fwd::BN);
@@ -137,6 +143,9 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
     p.n_sg = (int)n_sg;
     p.n_items = (int)n_items;
     p.scale = 1.0f / sqrtf((float)sh.C);
+    p.r_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)sh.C)));
+    p.g = static_cast<const __nv_bfloat16*>(g);
+    p.in = to_strides(in);
     p.out = static_cast<__nv_bfloat16*>(out);
     p.os = to_strides(os);
     p.lse = lse;
