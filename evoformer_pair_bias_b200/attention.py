@@ -32,7 +32,10 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 
 #: Every symbol include/evo_attn.h declares.
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
-           "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count")
+           "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc")
+
+#: Size of the library's fixed scratch area used by evo_attn_bwd_noalloc (bytes).
+NOALLOC_WORKSPACE_BYTES = 32 << 20
 
 
 class EvoError(RuntimeError):
@@ -74,6 +77,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_attn_device_status.restype = ctypes.c_int
     lib.evo_attn_version.restype = ctypes.c_int
     lib.evo_attn_launch_count.restype = ctypes.c_uint64
+    lib.evo_attn_bwd_noalloc.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, stp, vp,
+                                         vp, vp, vp, vp, stp, vp, vp]
+    lib.evo_attn_bwd_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -169,6 +175,36 @@ def evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, w
                           _ptr(grads["d_pair_bias"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
                           _stream(q.device))
     _check("evo_attn_bwd", rc)
+    return grads
+
+
+def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None):
+    """Backward pass through evo_attn_bwd_noalloc: no workspace is passed or allocated.
+
+    For callers that must not allocate device memory: the library uses its own
+    fixed scratch area (NOALLOC_WORKSPACE_BYTES per device), shared by every call,
+    so calls must not overlap on the GPU.  Output tensors may be passed in
+    ``grads``; any that are missing are allocated here by torch, as plumbing.
+    """
+    lib = load_library()
+    _same_strides(q, k, v, g)
+    _same_strides(out, dout)
+    sh = _shape(q)
+    B, S, N, H, C = q.shape
+    grads = dict(grads or {})
+    for n in ("dq", "dk", "dv", "dg"):
+        if grads.get(n) is None:
+            grads[n] = empty_like_rows(q)
+    if grads.get("d_pair_bias") is None:
+        grads["d_pair_bias"] = torch.empty((B, 1, H, N, N), dtype=torch.float32, device=q.device)
+    _same_strides(grads["dq"], grads["dk"], grads["dv"], grads["dg"])
+    rc = lib.evo_attn_bwd_noalloc(ctypes.byref(sh), DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                  ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out),
+                                  _ptr(dout), ctypes.byref(_strides(out)), _ptr(lse), _ptr(grads["dq"]),
+                                  _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
+                                  ctypes.byref(_strides(grads["dq"])), _ptr(grads["d_pair_bias"]),
+                                  _stream(q.device))
+    _check("evo_attn_bwd_noalloc", rc)
     return grads
 
 

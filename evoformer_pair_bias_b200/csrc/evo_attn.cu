@@ -14,6 +14,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "evo_attn.h"
 #include "common.cuh"
@@ -320,6 +321,46 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
     const evo_status_t rs = evo::bwd::run(c, s, &launched);
     g_launches += (uint64_t)launched;
     return rs;
+}
+
+// ---------------------------------------------------------------- no-allocation backward
+// Scratch area of evo_attn_bwd_noalloc.  Host code must not pass the array's
+// name to a kernel: on the host it is only a stand-in for the device object,
+// whose address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_evo_noalloc_ws[EVO_ATTN_NOALLOC_WORKSPACE_BYTES];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_addr[256] = {};
+
+static evo_status_t noalloc_workspace(void** addr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return EVO_ERR_CUDA;
+    if (dev < 0 || dev >= 256) return EVO_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {            // once per device, with that device current
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_evo_noalloc_ws) != cudaSuccess || !a) return EVO_ERR_CUDA;
+        g_noalloc_addr[dev] = a;
+    }
+    *addr = g_noalloc_addr[dev];
+    return EVO_OK;
+}
+
+evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
+                                  const void* v, const void* g, const evo_strides_t* in_str, const void* mask_bias,
+                                  const void* pair_bias, const void* out, const void* dout,
+                                  const evo_strides_t* out_str, const float* lse, void* dq, void* dk, void* dv,
+                                  void* dg, const evo_strides_t* grad_str, float* d_pair_bias, void* stream) {
+    const evo_status_t st = check_shape(shape);
+    if (st != EVO_OK) return st;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_F32) return EVO_ERR_INVALID_ARG;
+    if (evo_attn_bwd_workspace_bytes(shape, dtype) > EVO_ATTN_NOALLOC_WORKSPACE_BYTES)
+        return EVO_ERR_WORKSPACE_TOO_SMALL;
+    void* ws = nullptr;
+    const evo_status_t wst = noalloc_workspace(&ws);
+    if (wst != EVO_OK) return wst;
+    return evo_attn_bwd(shape, dtype, q, k, v, g, in_str, mask_bias, pair_bias, out, dout, out_str, lse, dq, dk,
+                        dv, dg, grad_str, d_pair_bias, ws, EVO_ATTN_NOALLOC_WORKSPACE_BYTES, stream);
 }
 
 }  // extern "C"

@@ -140,6 +140,43 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype,
                           float* d_pair_bias,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Backward pass that allocates nothing and takes no workspace argument.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot call cudaMalloc and have no device buffer of their own to lend
+ * as workspace -- for example a plug-in that runs inside a host framework
+ * which owns all device memory and forbids its extensions to allocate, or a
+ * service whose device memory footprint is fixed when it starts.
+ *
+ * Same arguments and results as evo_attn_bwd, minus the workspace.  Instead
+ * the library uses a fixed scratch area of EVO_ATTN_NOALLOC_WORKSPACE_BYTES
+ * (32 MiB) in device memory that exists from the moment the library is loaded
+ * on a device until the process exits; every GPU that loads the library holds
+ * it.  A shape whose workspace (evo_attn_bwd_workspace_bytes) is larger than
+ * that is rejected with EVO_ERR_WORKSPACE_TOO_SMALL before anything is
+ * enqueued -- for instance bf16 with B=1, S=32, N=256, H=4, C=32 fits, the
+ * 128-row, 8-head MSA-row shape at N=256 does not.
+ *
+ * The first call on a device looks up the scratch area's device address (a
+ * one-time, host-side query; it allocates nothing); make that first call
+ * before any stream capture on that device.  All calls share the one scratch
+ * area and it keeps the last call's contents; every part of it that must
+ * start at zero is cleared by the call itself.  Calls whose kernels overlap
+ * on the GPU (different streams, or different host threads, with no ordering
+ * between them) race on the scratch area and corrupt each other's results:
+ * order them on one stream, or use evo_attn_bwd with separate workspaces.
+ */
+#define EVO_ATTN_NOALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
+evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype,
+                                  const void* q, const void* k, const void* v, const void* g,
+                                  const evo_strides_t* in_str,
+                                  const void* mask_bias, const void* pair_bias,
+                                  const void* out, const void* dout, const evo_strides_t* out_str,
+                                  const float* lse,
+                                  void* dq, void* dk, void* dv, void* dg, const evo_strides_t* grad_str,
+                                  float* d_pair_bias, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* evo_status_string(evo_status_t status);
 
