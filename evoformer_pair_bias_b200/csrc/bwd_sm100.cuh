@@ -46,22 +46,33 @@ constexpr int BK = 128;   // key tile (TMEM lanes)
 constexpr int HD = 32;
 constexpr int TILE_BYTES = 128 * HD * 2;          // 8 KB, 64-byte rows, 64B swizzle
 constexpr int BT_BOX = 128 * 64 * 2;              // 16 KB: 128 key rows x 64 queries, 128B swizzle
-constexpr int KVB = 2 * TILE_BYTES + 1024;        // K, V, mask row (256 B), padded to 1 KB
-// Q, dOa (bf16 hi part), dOa (lo part), biasT, nl (512 B), -D (512 B)
-constexpr int STB = 3 * TILE_BYTES + 2 * BT_BOX + 1024;
+constexpr int RT_BYTES = 4096;                    // 16 x 128 bf16 rank-term block, 128B swizzle
+constexpr int CONST_BYTES = 4096;                 // 128 x 16 bf16 constant block, no swizzle
+// per row s (double-buffered): K, V, mask block (row 0 = mask row of s; MN-major A operand)
+constexpr int KV_K = 0, KV_V = TILE_BYTES, KV_MASK = 2 * TILE_BYTES, KVB = 2 * TILE_BYTES + RT_BYTES;
+// per step (double-buffered): Q, dOa high / low parts, transposed bias tile,
+// nl block (rows 0,1 = high/low of -lse*sqrt(C)) and -D block (rows 0,1 = high/low of -D)
 constexpr int ST_Q = 0, ST_DOH = TILE_BYTES, ST_DOL = 2 * TILE_BYTES, ST_BT = 3 * TILE_BYTES;
-constexpr int ST_NL = 3 * TILE_BYTES + 2 * BT_BOX, ST_ND = ST_NL + 512;
+constexpr int ST_NL = ST_BT + 2 * BT_BOX, ST_ND = ST_NL + RT_BYTES, STB = ST_ND + RT_BYTES;
 constexpr int OFF_KV = 0;
 constexpr int OFF_ST = 2 * KVB;
-constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tiles (2 buffers), each 2 boxes of 128 rows x 128 B
+constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tile, 2 boxes of 128 rows x 128 B
 constexpr int DS_BYTES = 2 * BT_BOX;
-constexpr int OFF_BAR = OFF_DS + 2 * DS_BYTES;
-// kv_full[2] kv_empty[2] q_full[2] q_empty[2] sdp_full sdp_free ds_full ds_free[2]
+constexpr int OFF_ONES = OFF_DS + DS_BYTES;        // A operand: columns 0 and 1 equal to 1
+constexpr int OFF_RROW = OFF_ONES + CONST_BYTES;   // B operand: row 0 equal to r = bf16(sqrt(C))
+constexpr int OFF_BAR = OFF_RROW + CONST_BYTES;
+// kv_full[2] kv_empty[2] q_full[2] q_empty[2] sdp_full sdp_free ds_full pt_free[2] ds_free
 // dq_full dq_free dkv_full dkv_free mma_done
-constexpr int NBARS = 18;
+constexpr int NBARS = 19;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-constexpr int THREADS = 320;                       // warp 0 TMA, warp 1 MMA, warps 2..9 dS
+// Warps 0..7: two dS warpgroups (queries 0..63 / 64..127 of the tile); warp 8 TMA,
+// warp 9 MMA, warps 10, 11 idle.  The last warpgroup hands registers to the dS
+// warpgroups: 2*128*208 + 128*88 = 384*168, the launch's register pool.
+constexpr int THREADS = 384;
+constexpr int LAUNCH_REGS = 168;
+constexpr uint32_t DS_REGS = 208, CONTROL_REGS = 88;
+static_assert((2 * DS_REGS + CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
 // TMEM columns: S^T, dP^T, two P^T buffers (bf16 pairs), dV, dK, dQ accumulators
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 384, TM_DK = 416, TM_DQ = 448, TM_COLS = 512;
 
@@ -81,10 +92,10 @@ inline int num_groups(int64_t B, int64_t S, int64_t N, int64_t H) {
 struct MainParams {
     int B, S, N, H;
     int n_it;            // query tiles
-    int n_pad;           // n_it * BQ: row length of the padded row-term arrays
     int gsz;             // rows s per group
     float sc2;           // log2(e) / sqrt(C)
     float rs;            // 1 / sqrt(C)
+    float r_bf16;        // bf16(sqrt(C))
     float* part;         // [G,B,H,N,N] partials, or d_pair_bias when G == 1
     float* dq_acc;       // [B,S,N,H,C] fp32, contiguous
     __nv_bfloat16* dk;
@@ -98,16 +109,16 @@ template <bool HAS_MASK, bool HAS_BIAS>
 __global__ void __launch_bounds__(THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_doa,
-                    const __grid_constant__ CUtensorMap tm_dol,
-                    const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_mask,
-                    const __grid_constant__ CUtensorMap tm_nl, const __grid_constant__ CUtensorMap tm_d,
-                    const MainParams p) {
+                    const __grid_constant__ CUtensorMap tm_dol, const __grid_constant__ CUtensorMap tm_bt,
+                    const __grid_constant__ CUtensorMap tm_mask, const __grid_constant__ CUtensorMap tm_nl,
+                    const __grid_constant__ CUtensorMap tm_d, const MainParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kProducer = 8, kMma = 9;
     const int j0 = blockIdx.x * BK;
     const int grp = blockIdx.y;
     const int b = blockIdx.z / p.H, h = blockIdx.z % p.H;
@@ -123,25 +134,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto q_empty = [&](int x) { return bar0 + 8u * (6 + x); };
     const uint32_t sdp_full = bar0 + 8u * 8, sdp_free = bar0 + 8u * 9;
     const uint32_t ds_full = bar0 + 8u * 10;
-    auto ds_free = [&](int x) { return bar0 + 8u * (11 + x); };
-    const uint32_t dq_full = bar0 + 8u * 13, dq_free = bar0 + 8u * 14;
-    const uint32_t dkv_full = bar0 + 8u * 15, dkv_free = bar0 + 8u * 16;
-    const uint32_t mma_done = bar0 + 8u * 17;
+    auto pt_free = [&](int x) { return bar0 + 8u * (11 + x); };
+    const uint32_t ds_free = bar0 + 8u * 13;
+    const uint32_t dq_full = bar0 + 8u * 14, dq_free = bar0 + 8u * 15;
+    const uint32_t dkv_full = bar0 + 8u * 16, dkv_free = bar0 + 8u * 17;
+    const uint32_t mma_done = bar0 + 8u * 18;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(kv_full(x), 1);
-            mbar_init(kv_empty(x), 1 + 8);
+            mbar_init(kv_empty(x), 1);
             mbar_init(q_full(x), 1);
             mbar_init(q_empty(x), 1 + 8);
+            mbar_init(pt_free(x), 1);
         }
         mbar_init(sdp_full, 1);
         mbar_init(sdp_free, 8);
         mbar_init(ds_full, 8);
-        mbar_init(ds_free(0), 1);
-        mbar_init(ds_free(1), 1);
+        mbar_init(ds_free, 1);
         mbar_init(dq_full, 1);
         mbar_init(dq_free, 8);
         mbar_init(dkv_full, 1);
@@ -150,23 +162,50 @@ __global__ void __launch_bounds__(THREADS, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == kProducer && lane == 0) {
         prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_doa);
-        prefetch_tmap(&tm_dol);
-        prefetch_tmap(&tm_nl); prefetch_tmap(&tm_d);
+        prefetch_tmap(&tm_dol); prefetch_tmap(&tm_nl); prefetch_tmap(&tm_d);
         if (HAS_BIAS) prefetch_tmap(&tm_bt);
         if (HAS_MASK) prefetch_tmap(&tm_mask);
     }
-    if (warp == 1) {
+    if (warp == kMma) {
         tmem_alloc(base + OFF_MISC, TM_COLS);
         tmem_relinquish();
+    }
+    if (warp < 8) {
+        // Constant operands and the zero rows of the rank-term blocks (the TMA
+        // writes only rows 0..1 of the nl / -D blocks and row 0 of a mask block).
+        // No-swizzle K-major element (row, k): (row%8)*16 + (row/8)*256 + (k/8)*128 + (k%8)*2.
+        const int t = threadIdx.x;
+        auto zero = [&](int off, int bytes) {
+            for (int o = t * 16; o < bytes; o += 256 * 16)
+                *reinterpret_cast<uint4*>(gbase + off + o) = make_uint4(0u, 0u, 0u, 0u);
+        };
+        zero(OFF_ONES, CONST_BYTES);
+        zero(OFF_RROW, CONST_BYTES);
+        for (int x = 0; x < 2; ++x) {
+            zero(OFF_KV + x * KVB + KV_MASK, RT_BYTES);
+            zero(OFF_ST + x * STB + ST_NL, RT_BYTES);
+            zero(OFF_ST + x * STB + ST_ND, RT_BYTES);
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (t < 128) {
+            const uint16_t one = 0x3F80u;
+            const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
+            uint8_t* o = gbase + OFF_ONES + (t % 8) * 16 + (t / 8) * 256;
+            reinterpret_cast<uint16_t*>(o)[0] = one;   // k = 0
+            reinterpret_cast<uint16_t*>(o)[1] = one;   // k = 1
+            *reinterpret_cast<uint16_t*>(gbase + OFF_RROW + (t % 8) * 16 + (t / 8) * 256) = rb;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == kProducer) {
+        regs_decrease<CONTROL_REGS>();
         // ---------------------------------------------------------------- producer
         if (lane == 0 && T > 0) {
             int kv_issued[2] = {0, 0}, q_issued[2] = {0, 0};
@@ -177,16 +216,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (si >= 2) ok = mbar_wait(kv_empty(x), ((si >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01);
                 if (!ok) break;
                 mbar_arrive_expect_tx(kv_full(x), 2 * TILE_BYTES + (HAS_MASK ? 256 : 0));
-                tma_load_5d(kb, &tm_k, kv_full(x), 0, j0, h, s, b);
-                tma_load_5d(kb + TILE_BYTES, &tm_v, kv_full(x), 0, j0, h, s, b);
-                if (HAS_MASK) tma_load_3d(kb + 2 * TILE_BYTES, &tm_mask, kv_full(x), j0, s, b);
+                tma_load_5d(kb + KV_K, &tm_k, kv_full(x), 0, j0, h, s, b);
+                tma_load_5d(kb + KV_V, &tm_v, kv_full(x), 0, j0, h, s, b);
+                if (HAS_MASK) {   // mask row of s into row 0 of the two 64-key atoms of the A block
+                    tma_load_3d(kb + KV_MASK, &tm_mask, kv_full(x), j0, s, b);
+                    tma_load_3d(kb + KV_MASK + 2048, &tm_mask, kv_full(x), j0 + 64, s, b);
+                }
                 ++kv_issued[x];
                 for (int it = 0; it < ni; ++it) {
                     const int t = si * ni + it, st = t & 1, i0 = it * BQ;
                     const uint32_t sb = base + OFF_ST + st * STB;
                     if (t >= 2) ok = mbar_wait(q_empty(st), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(q_full(st), 3 * TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 1024);
+                    mbar_arrive_expect_tx(q_full(st), 3 * TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 4 * 256);
                     tma_load_5d(sb + ST_Q, &tm_q, q_full(st), 0, i0, h, s, b);
                     tma_load_5d(sb + ST_DOH, &tm_doa, q_full(st), 0, i0, h, s, b);
                     tma_load_5d(sb + ST_DOL, &tm_dol, q_full(st), 0, i0, h, s, b);
@@ -194,8 +236,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_4d(sb + ST_BT, &tm_bt, q_full(st), i0, j0, h, b);
                         tma_load_4d(sb + ST_BT + BT_BOX, &tm_bt, q_full(st), i0 + 64, j0, h, b);
                     }
-                    tma_load_4d(sb + ST_NL, &tm_nl, q_full(st), i0, h, s, b);
-                    tma_load_4d(sb + ST_ND, &tm_d, q_full(st), i0, h, s, b);
+                    // rows 0..1 (high, low) of the two 64-query atoms of the nl and -D blocks
+                    tma_load_5d(sb + ST_NL, &tm_nl, q_full(st), i0, 0, h, s, b);
+                    tma_load_5d(sb + ST_NL + 2048, &tm_nl, q_full(st), i0 + 64, 0, h, s, b);
+                    tma_load_5d(sb + ST_ND, &tm_d, q_full(st), i0, 0, h, s, b);
+                    tma_load_5d(sb + ST_ND + 2048, &tm_d, q_full(st), i0 + 64, 0, h, s, b);
                     ++q_issued[st];
                 }
             }
@@ -205,10 +250,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (q_issued[x]) mbar_wait(q_full(x), (q_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMma) {
+        regs_decrease<CONTROL_REGS>();
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0 && T > 0) {
             constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // S^T, dP^T
+            constexpr uint32_t ID_RT = idesc_bf16(BK, BQ, false, true);    // ones x rank-term block
+            constexpr uint32_t ID_MK = idesc_bf16(BK, BQ, true, false);    // mask block x r-row
             constexpr uint32_t ID_KV = idesc_bf16(BK, HD, false, true);    // dV, dK (B MN-major)
             constexpr uint32_t ID_Q = idesc_bf16(BQ, HD, true, true);      // dQ (A and B MN-major)
             bool ok = true;
@@ -219,21 +267,27 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (t > 0 && !mbar_wait(sdp_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x13)) return false;
                 tc_fence_after();
                 const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
+                // S^T = K Q^T - lse*sqrt(C) (+ r * mask_j)
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    mma_ss(tmem + TM_ST, smem_desc(kb + kk * 32, 16, 512, kSw64), smem_desc(sb + kk * 32, 16, 512, kSw64),
-                           ID_SS, kk > 0);
-                }
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    mma_ss(tmem + TM_ST, smem_desc(kb + KV_K + kk * 32, 16, 512, kSw64),
+                           smem_desc(sb + ST_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                mma_ss(tmem + TM_ST, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                       smem_desc(sb + ST_NL, 2048, 1024, kSw128), ID_RT, 1u);
+                if (HAS_MASK)
+                    mma_ss(tmem + TM_ST, smem_desc(kb + KV_MASK, 2048, 1024, kSw128),
+                           smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
+                // dP^T = V (dOa_hi + dOa_lo)^T - D
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    mma_ss(tmem + TM_DPT, smem_desc(kb + TILE_BYTES + kk * 32, 16, 512, kSw64),
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
                            smem_desc(sb + ST_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-                }
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    mma_ss(tmem + TM_DPT, smem_desc(kb + TILE_BYTES + kk * 32, 16, 512, kSw64),
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
                            smem_desc(sb + ST_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
-                }
+                mma_ss(tmem + TM_DPT, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                       smem_desc(sb + ST_ND, 2048, 1024, kSw128), ID_RT, 1u);
                 mma_commit(sdp_full);
                 return true;
             };
@@ -247,29 +301,29 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
-                const int db = t & 1;                    // dS^T / P^T buffer of this step
-                const uint32_t ds = base + OFF_DS + db * DS_BYTES;
-                const uint32_t pt = TM_PT + db * 64;
+                const int pb = t & 1;                    // P^T buffer of this step
+                const uint32_t ds = base + OFF_DS;
 #pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk) {   // dV_j += P^T dOa_i
-                    mma_ts(tmem + TM_DV, tmem + pt + kk * 8, smem_desc(sb + ST_DOH + kk * 1024, TILE_BYTES, 512, kSw64),
-                           ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < BQ / 16; ++kk)     // dV_j += P^T dOa_hi
+                    mma_ts(tmem + TM_DV, tmem + TM_PT + pb * 64 + kk * 8,
+                           smem_desc(sb + ST_DOH + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(pt_free(pb));
 #pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk) {   // dK_j += dS^T Q_i
+                for (int kk = 0; kk < BQ / 16; ++kk) {   // dK_j += dS^T Q
                     const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
-                    mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128), smem_desc(sb + ST_Q + kk * 1024, TILE_BYTES, 512, kSw64),
-                           ID_KV, (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128),
+                           smem_desc(sb + ST_Q + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
+                           (it > 0 || kk > 0) ? 1u : 0u);
                 }
                 if (t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x16);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {   // dQ_i = dS K_j
+                for (int kk = 0; kk < BK / 16; ++kk)     // dQ_i = dS K_j
                     mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
-                           smem_desc(kb + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(ds_free(db));
+                           smem_desc(kb + KV_K + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
+                mma_commit(ds_free);
                 mma_commit(dq_full);
                 mma_commit(q_empty(st));
                 if (it == ni - 1) {
@@ -281,9 +335,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait(mma_done, 0, &no_abort, kTimeoutBase | 0x17);
         }
-    } else if (T > 0) {
+    } else if (warp < 8) {
+        regs_increase<DS_REGS>();
+        if (T > 0) {
         // ---------------------------------------------------------------- dS warpgroups
-        const int wg = (warp - 2) >> 2;          // 0: queries 0..63 of the tile, 1: 64..127
+        const int wg = warp >> 2;                // 0: queries 0..63 of the tile, 1: 64..127
         const int quad = warp & 3;
         const int r = quad * 32 + lane;          // key row within the tile = TMEM lane
         const int j = j0 + r;
@@ -294,7 +350,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         // this group's slab of the partial sums (the output itself when there is one group)
         float* part = p.part + ((int64_t)grp * p.B * p.H + (int64_t)b * p.H + h) * p.N * p.N;
         bool ok = true;
-        uint64_t RB2 = 0;                        // per-key term: mask*log2e, or -inf for padded keys
 
         auto drain_dq = [&](int t) -> bool {     // dQ rows of step t: lanes = queries
             if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) return false;
@@ -346,17 +401,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
             const int i0 = it * BQ;
             if (it == 0) {
-                ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x23);
-                if (!ok) break;
-                float rb = 0.f;
-                if (HAS_MASK) {
-                    const uint16_t mb = *reinterpret_cast<const uint16_t*>(gbase + OFF_KV + x * KVB + 2 * TILE_BYTES + r * 2);
-                    rb = __uint_as_float((uint32_t)mb << 16) * EVO_LOG2E;
-                }
-                if (!jvalid) rb = -INFINITY;
-                RB2 = f2(rb, rb);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(kv_empty(x));
+                // the mask block of this row is read by the MMA only; no thread waits on kv_full
+                (void)x;
             }
             ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
             if (!ok) break;
@@ -367,16 +413,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sdp_free);
+            if (!jvalid) {                       // padded key rows: P = 0
+#pragma unroll
+                for (int c = 0; c < 64; ++c) sv[c] = __float_as_uint(-INFINITY);
+            }
 
             ok = mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x25);
-            const int db = t & 1;                // dS^T / P^T buffer of this step
-            if (ok && t >= 2) ok = mbar_wait(ds_free(db), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
+            const int pb = t & 1;                // P^T buffer of this step
+            if (ok && t >= 2) ok = mbar_wait(pt_free(pb), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
             if (!ok) break;
+            tc_fence_after();
             const uint32_t sb = base + OFF_ST + st * STB;
-            const uint32_t nl_addr = sb + ST_NL + wg * 256;
-            const uint32_t nd_addr = sb + ST_ND + wg * 256;
             const uint32_t bt_addr = sb + ST_BT + wg * BT_BOX + r * 128;
-            const uint32_t ds_row = base + OFF_DS + db * DS_BYTES + wg * BT_BOX + r * 128;
+            const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * 32;
             // d_pair_bias partial (zeroed before the launch).  Each address of this
             // group's slab is updated by exactly one thread, in row order s, with
             // fire-and-forget atomic adds; same-thread atomics to one address are
@@ -384,8 +433,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int ivalid = jvalid ? p.N - i0 - wg * 64 : 0;   // queries of this half inside N
             float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
             const int64_t rstride = p.N;
-            // P = exp2(S*scale*log2e + bias*log2e + nl_i + rb_j), dS = P * (dP - D_i), two columns per op
-            uint32_t pk[32];
+            // P = exp2(S^T * sc2 + bias * log2e) (S^T already holds -lse and the mask),
+            // dS = P * dP^T (dP^T already holds -D); two columns per op
+            uint32_t dk2[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {                      // 8 columns at a time
                 uint32_t bw[4] = {0u, 0u, 0u, 0u};
@@ -393,35 +443,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint4 w = lds128(bt_addr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
                     bw[0] = w.x; bw[1] = w.y; bw[2] = w.z; bw[3] = w.w;
                 }
-                const uint4 n0 = lds128(nl_addr + q * 32), n1 = lds128(nl_addr + q * 32 + 16);
-                const uint4 d0 = lds128(nd_addr + q * 32), d1 = lds128(nd_addr + q * 32 + 16);
-                const uint64_t nl2[4] = {f2(__uint_as_float(n0.x), __uint_as_float(n0.y)),
-                                         f2(__uint_as_float(n0.z), __uint_as_float(n0.w)),
-                                         f2(__uint_as_float(n1.x), __uint_as_float(n1.y)),
-                                         f2(__uint_as_float(n1.z), __uint_as_float(n1.w))};
-                const uint64_t nd2[4] = {f2(__uint_as_float(d0.x), __uint_as_float(d0.y)),
-                                         f2(__uint_as_float(d0.z), __uint_as_float(d0.w)),
-                                         f2(__uint_as_float(d1.x), __uint_as_float(d1.y)),
-                                         f2(__uint_as_float(d1.z), __uint_as_float(d1.w))};
                 float dsq[8];
-                uint32_t dkq[4];
+                uint32_t pk4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = q * 8 + 2 * e;
-                    uint64_t t2 = HAS_BIAS ? ffma2(bf16x2_to_f2(bw[e]), L2E2, nl2[e]) : nl2[e];
-                    t2 = fadd2(t2, RB2);
-                    const uint64_t x2 = ffma2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), SC2, t2);
-                    const float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));
-                    const uint64_t dd = fadd2(f2(__uint_as_float(sv[64 + c]), __uint_as_float(sv[65 + c])), nd2[e]);
-                    const uint64_t ds2 = fmul2(f2(p0, p1), dd);
+                    uint64_t y2 = fmul2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), SC2);
+                    if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[e]), L2E2, y2);
+                    const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
+                    const uint64_t ds2 = fmul2(f2(p0, p1), f2(__uint_as_float(sv[64 + c]), __uint_as_float(sv[65 + c])));
                     dsq[2 * e] = f2lo(ds2);
                     dsq[2 * e + 1] = f2hi(ds2);
-                    pk[q * 4 + e] = pack_bf16(p0, p1);
-                    dkq[e] = pack_bf16(dsq[2 * e], dsq[2 * e + 1]);
+                    pk4[e] = pack_bf16(p0, p1);
+                    dk2[q * 4 + e] = pack_bf16(dsq[2 * e], dsq[2 * e + 1]);
                 }
-                const uint32_t addr = ds_row + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dkq[0]), "r"(dkq[1]),
-                             "r"(dkq[2]), "r"(dkq[3])
+                asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt_addr + q * 4),
+                             "r"(pk4[0]), "r"(pk4[1]), "r"(pk4[2]), "r"(pk4[3])
                              : "memory");
                 if (ivalid >= 64) {
 #pragma unroll
@@ -439,9 +476,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(q_empty(st));           // bias / nl / D of this stage consumed
-            tc_fence_after();
-            tmem_st32(lane_addr + TM_PT + db * 64 + wg * 32, pk);
+            if (lane == 0) mbar_arrive(q_empty(st));           // bias tile of this stage consumed
+            if (t > 0) ok = mbar_wait(ds_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x27);
+            if (!ok) break;
+            const uint32_t ds_row = base + OFF_DS + wg * BT_BOX + r * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t addr = ds_row + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk2[4 * q]),
+                             "r"(dk2[4 * q + 1]), "r"(dk2[4 * q + 2]), "r"(dk2[4 * q + 3])
+                             : "memory");
+            }
             tc_wait_st();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
@@ -459,11 +504,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (ok) ok = drain_dq(T - 1);
         if (ok) ok = drain_dkv(ns - 1);
+        }
+    } else {
+        regs_decrease<CONTROL_REGS>();
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMma) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
     }
@@ -472,29 +520,39 @@ __global__ void __launch_bounds__(THREADS, 1)
 // ------------------------------------------------------------------ elementwise kernels
 struct PreParams {
     int B, S, N, H, n_pad;
+    float sqrt_c;
     const __nv_bfloat16* out; const __nv_bfloat16* dout; Strides os;
     const __nv_bfloat16* g; Strides in;
     const float* lse;
     __nv_bfloat16* dg; Strides gs;
     __nv_bfloat16* doa_hi;  // contiguous [B,S,N,H,C]
     __nv_bfloat16* doa_lo;  // contiguous [B,S,N,H,C]: dOa - float(doa_hi), rounded
-    float* nd;              // [B,S,H,n_pad]: -D_i, 0 on padding
-    float* nl;              // [B,S,H,n_pad]: -lse_i * log2(e), -inf on padding
+    __nv_bfloat16* nl;      // [B,S,H,2,n_pad]: high / low rows of -lse*sqrt(C); padding -1e30 / 0
+    __nv_bfloat16* nd;      // [B,S,H,2,n_pad]: high / low rows of -D; padding 0
     float* dq_acc;          // contiguous [B,S,N,H,C] fp32
 };
+
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    *hi = h;
+    *lo = __float2bfloat16_rn(v - __bfloat162float(h));
+}
 
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
     const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
     const int64_t pads = (int64_t)p.B * p.S * p.H * (p.n_pad - p.N);
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows + pads;
          t += (int64_t)gridDim.x * blockDim.x) {
-        if (t >= rows) {   // padded query slots of the row-term arrays
+        if (t >= rows) {   // padded query slots of the rank-term rows: P must come out 0
             const int64_t u = t - rows;
             const int w = p.n_pad - p.N;
             const int64_t bsh = u / w;
             const int i = p.N + (int)(u % w);
-            p.nl[bsh * p.n_pad + i] = -INFINITY;
-            p.nd[bsh * p.n_pad + i] = 0.f;
+            const int64_t o = bsh * 2 * p.n_pad + i;
+            p.nl[o] = __float2bfloat16_rn(-1e30f);
+            p.nl[o + p.n_pad] = __float2bfloat16_rn(0.f);
+            p.nd[o] = __float2bfloat16_rn(0.f);
+            p.nd[o + p.n_pad] = __float2bfloat16_rn(0.f);
             continue;
         }
         const int h = (int)(t % p.H);
@@ -531,8 +589,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
             lo4[q] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
         const int64_t bsh = ((int64_t)b * p.S + s) * p.H + h;
-        p.nd[bsh * p.n_pad + i] = -D;
-        p.nl[bsh * p.n_pad + i] = -p.lse[bsh * p.N + i] * EVO_LOG2E;
+        const int64_t o = bsh * 2 * p.n_pad + i;
+        split_bf16(-D, p.nd + o, p.nd + o + p.n_pad);
+        split_bf16(-p.lse[bsh * p.N + i] * p.sqrt_c, p.nl + o, p.nl + o + p.n_pad);
         float4* acc = reinterpret_cast<float4*>(p.dq_acc + t * HD);
 #pragma unroll
         for (int q = 0; q < HD / 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -624,7 +683,14 @@ inline cudaError_t launch_main(const CUtensorMap* m, const MainParams& mp, dim3 
     auto kern = bwd_main_kernel<HM, HB>;
     static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (attr != cudaSuccess) return attr;
-    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[8], m[4], m[5], m[6], m[7], mp);
+    // The setmaxnreg split assumes exactly LAUNCH_REGS registers per thread at
+    // launch; with any other count an increase could wait forever.
+    static int regs = [&] {
+        cudaFuncAttributes fa{};
+        return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
+    }();
+    if (regs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], mp);
     return cudaGetLastError();
 }
 
@@ -643,8 +709,8 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
 
     const int B = (int)sh.B, S = (int)sh.S, N = (int)sh.N, H = (int)sh.H;
     const int n_pad = (N + BQ - 1) / BQ * BQ;
-    float* nd = reinterpret_cast<float*>(c.ws + c.d_off);
-    float* nl = reinterpret_cast<float*>(c.ws + c.nl_off);
+    __nv_bfloat16* nd = reinterpret_cast<__nv_bfloat16*>(c.ws + c.d_off);
+    __nv_bfloat16* nl = reinterpret_cast<__nv_bfloat16*>(c.ws + c.nl_off);
     __nv_bfloat16* doa = reinterpret_cast<__nv_bfloat16*>(c.ws + c.doa_off);
     __nv_bfloat16* dol = reinterpret_cast<__nv_bfloat16*>(c.ws + c.dol_off);
     float* dq_acc = reinterpret_cast<float*>(c.ws + c.dqacc_off);
@@ -654,11 +720,12 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     const int64_t rows = (int64_t)B * S * N * H;
     PreParams pp{};
     pp.B = B; pp.S = S; pp.N = N; pp.H = H; pp.n_pad = n_pad;
+    pp.sqrt_c = sqrtf((float)HD);
     pp.out = static_cast<const __nv_bfloat16*>(c.out); pp.dout = static_cast<const __nv_bfloat16*>(c.dout);
     pp.os = Strides{c.os.b, c.os.s, c.os.n, c.os.h};
     pp.g = static_cast<const __nv_bfloat16*>(c.g); pp.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
     pp.lse = c.lse; pp.dg = static_cast<__nv_bfloat16*>(c.dg); pp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
-    pp.doa_hi = doa; pp.doa_lo = dol; pp.nd = nd; pp.nl = nl; pp.dq_acc = dq_acc;
+    pp.doa_hi = doa; pp.doa_lo = dol; pp.nl = nl; pp.nd = nd; pp.dq_acc = dq_acc;
     bwd_pre_kernel<<<grid_for(rows + (int64_t)B * S * H * (n_pad - N), 256), 256, 0, stream>>>(pp);
     ++*launched;
     if (c.bias) {
@@ -671,7 +738,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     const size_t part_bytes = (size_t)c.groups * B * H * N * N * sizeof(float);
     if (cudaMemsetAsync(part, 0, part_bytes, stream) != cudaSuccess) return EVO_ERR_CUDA;
 
-    // tensor maps
+    // tensor maps: q, k, v, dOa high, dOa low, transposed bias, mask, nl rows, -D rows
     const evo_strides_t contig{(int64_t)S * N * H * HD, (int64_t)N * H * HD, (int64_t)H * HD, (int64_t)HD};
     CUtensorMap m[9];
     std::memset(m, 0, sizeof(m));
@@ -680,20 +747,20 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
         !tma::rows_bf16(&m[1], c.k, s5, c.in, BK, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !tma::rows_bf16(&m[2], c.v, s5, c.in, BK, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !tma::rows_bf16(&m[3], doa, s5, contig, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !tma::rows_bf16(&m[8], dol, s5, contig, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !tma::rowscalar_f32(&m[6], nl, s5, n_pad) || !tma::rowscalar_f32(&m[7], nd, s5, n_pad))
+        !tma::rows_bf16(&m[4], dol, s5, contig, BQ, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !tma::rowterm_bf16(&m[7], nl, s5, n_pad) || !tma::rowterm_bf16(&m[8], nd, s5, n_pad))
         return EVO_ERR_CUDA;
-    if (c.bias && !tma::square_bf16(&m[4], biasT, s5, BK)) return EVO_ERR_CUDA;
-    if (c.mask && !tma::mask_bf16(&m[5], c.mask, s5)) return EVO_ERR_CUDA;
+    if (c.bias && !tma::square_bf16(&m[5], biasT, s5, BK)) return EVO_ERR_CUDA;
+    if (c.mask && !tma::mask_bf16(&m[6], c.mask, s5, 64)) return EVO_ERR_CUDA;
 
     MainParams mp{};
     mp.B = B; mp.S = S; mp.N = N; mp.H = H;
     mp.n_it = (N + BQ - 1) / BQ;
-    mp.n_pad = n_pad;
     const int G = c.groups;
     mp.gsz = (S + G - 1) / G;
     mp.sc2 = EVO_LOG2E / sqrtf((float)HD);
     mp.rs = 1.0f / sqrtf((float)HD);
+    mp.r_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)HD)));
     mp.part = part;
     mp.dq_acc = dq_acc;
     mp.dk = static_cast<__nv_bfloat16*>(c.dk);
@@ -705,6 +772,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     else if (c.mask) e = launch_main<true, false>(m, mp, grid, stream);
     else if (c.bias) e = launch_main<false, true>(m, mp, grid, stream);
     else e = launch_main<false, false>(m, mp, grid, stream);
+    if (e == cudaErrorInvalidConfiguration) return EVO_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return EVO_ERR_CUDA;
     ++*launched;
 

@@ -95,5 +95,16 @@ inline bool rowscalar_f32(CUtensorMap* m, const void* ptr, const evo_shape_t& sh
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// bf16 rank-term rows [B,S,H,2,n_row] (a high and a low row per (b,s,h))
+// viewed as (i, row, h, s, b); box (64 queries, 2 rows, 1, 1, 1) with 128B
+// swizzle, so each box lands as rows 0..1 of one 128B-swizzled operand atom.
+inline bool rowterm_bf16(CUtensorMap* m, const void* ptr, const evo_shape_t& sh, int64_t n_row) {
+    const uint64_t N = (uint64_t)n_row, H = (uint64_t)sh.H, S = (uint64_t)sh.S;
+    const uint64_t dims[5] = {N, 2, H, S, (uint64_t)sh.B};
+    const uint64_t str[4] = {N * 2, 2 * N * 2, H * 2 * N * 2, S * H * 2 * N * 2};
+    const uint32_t box[5] = {64, 2, 1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 }  // namespace tma
 }  // namespace evo
