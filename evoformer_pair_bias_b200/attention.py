@@ -32,7 +32,8 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 
 #: Every symbol include/evo_attn.h declares.
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
-           "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc")
+           "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc",
+           "evo_attn_timing_enable", "evo_attn_timing_collect")
 
 #: Size of the library's fixed scratch area used by evo_attn_bwd_noalloc (bytes).
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -50,6 +51,14 @@ class Shape(ctypes.Structure):
 
 class Strides(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in ("b", "s", "n", "h")]
+
+
+#: Timing phases (evo_timing_t indices).
+PHASES = ("fwd_main", "bwd_main", "bwd_all")
+
+
+class Timing(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_uint64 * len(PHASES)), ("ms", ctypes.c_double * len(PHASES))]
 
 
 _lib = None
@@ -80,6 +89,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_attn_bwd_noalloc.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, stp, vp,
                                          vp, vp, vp, vp, stp, vp, vp]
     lib.evo_attn_bwd_noalloc.restype = ctypes.c_int
+    lib.evo_attn_timing_enable.argtypes = [ctypes.c_int]
+    lib.evo_attn_timing_enable.restype = ctypes.c_int
+    lib.evo_attn_timing_collect.argtypes = [ctypes.POINTER(Timing)]
+    lib.evo_attn_timing_collect.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -211,6 +224,18 @@ def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads
 def launch_count() -> int:
     """Kernels the library has enqueued in this process so far."""
     return int(load_library().evo_attn_launch_count())
+
+
+def timing_enable(on: bool = True) -> None:
+    """Switch the library's per-kernel event timing on or off."""
+    _check("evo_attn_timing_enable", load_library().evo_attn_timing_enable(1 if on else 0))
+
+
+def timing_collect() -> dict:
+    """Wait for the recorded phases; {phase: (calls, total ms)} since the last collect."""
+    t = Timing()
+    _check("evo_attn_timing_collect", load_library().evo_attn_timing_collect(ctypes.byref(t)))
+    return {name: (int(t.calls[i]), float(t.ms[i])) for i, name in enumerate(PHASES)}
 
 
 def device_status(clear: bool = True) -> int:

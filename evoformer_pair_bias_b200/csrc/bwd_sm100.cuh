@@ -690,7 +690,10 @@ inline cudaError_t launch_main(const CUtensorMap* m, const MainParams& mp, dim3 
         return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
     }();
     if (regs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], mp);
+    {
+        timing::Scope t(EVO_PHASE_BWD_MAIN, stream);
+        kern<<<grid, THREADS, SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8], mp);
+    }
     return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@
 #include "simt.cuh"
 #include "sm100.cuh"
 #include "tma_maps.cuh"
+#include "timing.cuh"
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
 
@@ -85,7 +86,10 @@ evo_status_t fwd_f32(const evo_shape_t& sh, const void* q, const void* k, const 
     a.mask = mask; a.bias = bias; a.out_w = out; a.os = to_strides(os); a.lse = lse;
     dim3 grid((unsigned)((sh.N + evo::simt::kRowsPerCta - 1) / evo::simt::kRowsPerCta), (unsigned)sh.S,
               (unsigned)(sh.B * sh.H));
-    evo::simt::fwd_kernel<float><<<grid, evo::simt::kWarps * 32, 0, stream>>>(a);
+    {
+        evo::timing::Scope t(EVO_PHASE_FWD_MAIN, stream);
+        evo::simt::fwd_kernel<float><<<grid, evo::simt::kWarps * 32, 0, stream>>>(a);
+    }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
@@ -111,7 +115,10 @@ evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p,
     }();
     if (regs != L::launch_regs) return EVO_ERR_UNSUPPORTED;
     const int grid = std::min(p.n_items, sm_count());
-    kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    {
+        evo::timing::Scope t(EVO_PHASE_FWD_MAIN, stream);
+        kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
@@ -228,6 +235,10 @@ int evo_attn_version(void) { return EVO_VERSION; }
 
 uint64_t evo_attn_launch_count(void) { return g_launches.load(); }
 
+evo_status_t evo_attn_timing_enable(int on) { return evo::timing::enable(on); }
+
+evo_status_t evo_attn_timing_collect(evo_timing_t* out) { return evo::timing::collect(out); }
+
 evo_status_t evo_attn_device_status(int clear) {
     if (cudaDeviceSynchronize() != cudaSuccess) return EVO_ERR_CUDA;
     unsigned int v = 0;
@@ -306,6 +317,7 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
                               (const void*)dg})
             if (!aligned(p, 4)) return EVO_ERR_INVALID_ARG;
         if (shape->S > 65535 || shape->N > 65535) return EVO_ERR_UNSUPPORTED;
+        evo::timing::Scope t(EVO_PHASE_BWD_ALL, s);
         return bwd_f32(*shape, a, s);
     }
     evo::bwd::Call c{};
@@ -318,7 +330,11 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
     c.dqacc_off = ws.dqacc_off;
     c.biast_off = ws.biast_off; c.part_off = ws.part_off; c.groups = ws.groups;
     int launched = 0;
-    const evo_status_t rs = evo::bwd::run(c, s, &launched);
+    evo_status_t rs;
+    {
+        evo::timing::Scope t(EVO_PHASE_BWD_ALL, s);
+        rs = evo::bwd::run(c, s, &launched);
+    }
     g_launches += (uint64_t)launched;
     return rs;
 }

@@ -195,6 +195,36 @@ int evo_attn_version(void);
  * (all devices, all streams).  Host-side counter; never synchronises. */
 uint64_t evo_attn_launch_count(void);
 
+/*
+ * Per-kernel device timing (off by default).  While switched on, each
+ * evo_attn_fwd / evo_attn_bwd call records a pair of CUDA events on its own
+ * `stream` around its main kernel, and evo_attn_bwd a second pair around all
+ * of its kernels, so that a caller can see how a step's device time splits
+ * between the kernels without a profiler.  The events come from a pool kept
+ * by the library (created on first use, reused afterwards); recording them
+ * adds no kernel and no synchronisation.  Recording is best-effort: if an
+ * event cannot be created or recorded that call simply goes untimed.
+ *
+ * evo_attn_timing_collect blocks until every phase recorded since the last
+ * collect has completed, adds up the elapsed times per phase into *out
+ * (calls and milliseconds) and forgets them.  It returns EVO_ERR_INVALID_ARG
+ * for a NULL `out` and EVO_ERR_CUDA if an event could not be waited on or
+ * read (that phase is then left out of the sums).  Both functions are safe to
+ * call from several host threads.
+ */
+#define EVO_TIMING_PHASES 3
+enum {
+    EVO_PHASE_FWD_MAIN = 0,   /* the forward kernel                         */
+    EVO_PHASE_BWD_MAIN = 1,   /* the backward's main (tensor-core) kernel    */
+    EVO_PHASE_BWD_ALL = 2     /* every kernel and memset of one evo_attn_bwd */
+};
+typedef struct {
+    uint64_t calls[EVO_TIMING_PHASES];
+    double ms[EVO_TIMING_PHASES];
+} evo_timing_t;
+evo_status_t evo_attn_timing_enable(int on);
+evo_status_t evo_attn_timing_collect(evo_timing_t* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,6 +77,15 @@ def test_host_argument_errors_need_no_gpu(lib):
     assert rc == 1
 
 
+def test_timing_hooks_answer_without_a_gpu(lib):
+    m = re.search(r"#define EVO_TIMING_PHASES (\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == len(A.PHASES)
+    assert lib.evo_attn_timing_collect(None) == 1
+    A.timing_enable(True)
+    A.timing_enable(False)
+    assert A.timing_collect() == {p: (0, 0.0) for p in A.PHASES}   # nothing recorded, nothing waited on
+
+
 def test_product_path_never_touches_the_oracle():
     """The package must not import, load or mention the CPU oracle."""
     pkg = os.path.join(ROOT, "evoformer_pair_bias_b200")
