@@ -53,32 +53,87 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """SM clocks, power and clock-event (throttle) reasons sampled during the timed region.
 
+    Polls NVML (the library nvidia-smi reads) every 5 ms from a thread, plus one
+    sample on entry and one on exit, so that even a timed region of a few
+    milliseconds is covered.  Falls back to ``nvidia-smi -lms 200`` if NVML
+    cannot be loaded.
+    """
+
+    # NVML clocks-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, uuid: str):
-        self.uuid = uuid
+    def __init__(self, uuid: str, period_s: float = 0.005):
+        self.uuid, self.period = uuid, period_s
+        self.samples = []          # (sm_mhz, max_mhz, power_w, reason bits)
+        self.smi_lines = []
+        self.nvml = None
         self.proc = None
-        self.lines = []
+        self.stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if not self.uuid or u == self.uuid:
+                return pynvml, h
+        raise RuntimeError("GPU not found through NVML")
+
+    def _sample(self):
+        nv, h = self.nvml
+        try:
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except AttributeError:
+            rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                             nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM),
+                             nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(rs)))
+
+    def _poll(self):
+        while not self.stop.wait(self.period):
+            try:
+                self._sample()
+            except Exception:
+                return
+
+    def _read_smi(self):
+        for line in self.proc.stdout:
+            self.smi_lines.append(line.strip())
 
     def __enter__(self):
         try:
+            self.nvml = self._nvml_handle()
+            self._sample()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
+        try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
+        if self.nvml is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
+            try:
+                self._sample()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -87,9 +142,16 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if self.nvml is not None and self.samples:
+            reasons = set()
+            for *_, bits in self.samples:
+                reasons.update(n for b, n in self.REASONS.items() if bits & b)
+            return {"sm_mhz": statistics.median(x[0] for x in self.samples), "sm_max_mhz": self.samples[-1][1],
+                    "power_w_max": max(x[2] for x in self.samples), "reasons": sorted(reasons),
+                    "samples": len(self.samples), "source": "NVML, 5 ms"}
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.smi_lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9 or (self.uuid and self.uuid not in parts[0]):
                 continue
@@ -102,7 +164,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 def gpu_uuid(dev) -> str:
@@ -179,39 +241,57 @@ def roofline(w, kt, pk, timed_s: float):
 
 
 def cpu_oracle_sample(w, target_s: float = 12.0, max_rows=None):
-    """Time the fp64 oracle (fwd + bwd) on the first r rows s of the workload, r sized for ~target_s."""
+    """Time the fp64 oracle (fwd + bwd) on the first r rows s of the workload, r (and a repeat
+    count) sized for about target_s seconds of CPU work."""
     import oracle
     oracle.build()
-    inp = make_inputs(w.with_(S=min(w.S, 64)), device="cpu")
+    inp = make_inputs(w, device="cpu")
 
-    def run(r):
-        x = {k: (None if v is None else (v[:, :r] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v)
-                 ).double().numpy() if v is not None else None for k, v in inp.items()}
+    def rows(r):
+        return {k: (None if v is None else (v[:, :r] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v)
+                    ).double().numpy() if v is not None else None for k, v in inp.items()}
+
+    def run(x):
         t0 = time.perf_counter()
         oracle.forward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"])
         oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"], x["dout"])
         return time.perf_counter() - t0
 
-    t1 = run(1)
-    r = max(1, min(inp["q"].shape[1], int(target_s / max(t1, 1e-3))))
+    t1 = run(rows(1))
+    r = max(1, min(w.S, int(target_s / max(t1, 1e-3))))
     if max_rows:
         r = min(r, max_rows)
-    t = run(r) if r > 1 else t1
-    L = w.B * r * w.H * w.N * w.N
+    x = rows(r)
+    t, reps = 0.0, 0
+    while reps == 0 or t < 0.7 * target_s:
+        t += run(x)
+        reps += 1
+    L = w.B * r * w.H * w.N * w.N * reps
     fl = 14 * L * w.C
-    return dict(value=fl / t / 1e12, unit="TFLOP/s", cores=os.cpu_count(), kind="oracle",
-                sample=f"{r} of {w.S} rows s (all {w.H} heads, N={w.N}), fwd+bwd, fp64, {t:.2f} s",
+    return dict(value=fl / t / 1e12, unit="TFLOP/s", cores=oracle_threads(), kind="oracle",
+                sample=f"{r} of {w.S} rows s (all {w.H} heads, N={w.N}) x{reps}, fwd+bwd, fp64, {t:.2f} s",
                 seconds=t)
+
+
+def oracle_threads() -> int:
+    """Threads the OpenMP oracle runs with on this host."""
+    v = os.environ.get("OMP_NUM_THREADS")
+    if v and v.isdigit():
+        return int(v)
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
 
 
 def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
     steps, warm = args.steps, args.warmup
-    info = cpu_oracle_sample(w, target_s=max(1.0, 60.0 / max(1, steps + warm)), max_rows=None)
+    info = cpu_oracle_sample(w, target_s=max(0.5, 60.0 / max(1, steps + warm)), max_rows=None)
     rows = int(info["sample"].split()[0])
     import oracle
-    inp = make_inputs(w.with_(S=min(w.S, 64)), device="cpu")
+    inp = make_inputs(w, device="cpu")
     x = {k: (None if v is None else (v[:, :rows] if k in ("q", "k", "v", "g", "dout", "mask_bias") else v)
              ).double().numpy() if v is not None else None for k, v in inp.items()}
     times = []
@@ -229,7 +309,7 @@ def run_reference(args, w, rank, world):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "B": w.B, "N_seq": w.S, "N_res": w.N, "H": w.H, "c": w.C,
                        "sample_rows": rows, "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
                              "sample": f"{rows} of {w.S} rows s per step, fwd+bwd, fp64"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -239,7 +319,7 @@ def run_reference(args, w, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -24,10 +24,12 @@
 //   warp 4*NSUB           TMA producer: per item Q (double-buffered by item
 //            parity), then per key tile K, V and the mask row (per row s) and
 //            the pair-bias tile into a 2-stage ring that runs across items.
-//   warp 4*NSUB+1         TMEM owner and MMA issuer (one lane): S_u as above
-//            (M=128, N=128), then O_u += P_u V_u (M=128, N=32, K=128, P read
-//            from TMEM).  The S MMAs of the next tile are issued before the PV
-//            of the current one, so they overlap the softmax.
+//   warps 4*NSUB+1+u      MMA issuer of row group u (one lane; the first also
+//            owns TMEM): S_u as above (M=128, N=128), then O_u += P_u V_u
+//            (M=128, N=32, K=128, P read from TMEM).  The S MMA of the next
+//            tile is issued before the PV of the current one, so it overlaps
+//            the softmax; one issuer per row group keeps the groups' pipelines
+//            independent of each other.
 //   softmax: thread = query row.  Load S
 //            from TMEM, online max and sum in fp32 with a lazy rescale (the
 //            running max moves only when a tile's max exceeds it by more than
@@ -71,8 +73,8 @@ struct Layout {
     static constexpr int maskb_off(int u) { return bias_off + BIAS_BYTES + u * MASKB_BYTES; }
     static constexpr int stage_bytes = round_up(bias_off + BIAS_BYTES + NSUB * MASKB_BYTES, 1024);
     static constexpr int bars = stage0 + STAGES * stage_bytes;
-    // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[u], s_free[u], p_full[u], o_full[u], mma_done
-    static constexpr int nbars = 4 + 2 * STAGES + 4 * NSUB + 1;
+    // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[u], s_free[u], p_full[u], o_full[u], mma_done[u]
+    static constexpr int nbars = 4 + 2 * STAGES + 5 * NSUB;
     static constexpr int misc = bars + nbars * 8;   // tmem base (u32), abort flag (u32)
     static constexpr int bytes = misc + 16 + 1024;  // + slack to align the base to 1024
     static constexpr uint32_t tmem_cols = NSUB == 1 ? 256 : 512;
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = 4 * NSUB, kMma = 4 * NSUB + 1;
+    constexpr int kProducer = 4 * NSUB, kMma = 4 * NSUB + 1;   // MMA issuers: warps kMma .. kMma+NSUB-1
 
     const uint32_t bar0 = base + L::bars;
     auto q_full = [&](int x) { return bar0 + 8u * (0 + x); };
@@ -143,26 +145,26 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     auto s_free = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + NSUB + u); };
     auto p_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 2 * NSUB + u); };
     auto o_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 3 * NSUB + u); };
-    const uint32_t bar_mma_done = bar0 + 8u * (4 + 2 * STAGES + 4 * NSUB);
+    auto mma_done = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 4 * NSUB + u); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::misc + 4);
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(q_full(x), 1);
-            mbar_init(q_empty(x), 1);
+            mbar_init(q_empty(x), NSUB);           // one commit per MMA issuer
         }
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(kv_full(st), 1);
-            mbar_init(kv_empty(st), 1);
+            mbar_init(kv_empty(st), NSUB);
         }
         for (int u = 0; u < NSUB; ++u) {
             mbar_init(s_full(u), 1);
             mbar_init(s_free(u), 4);
             mbar_init(p_full(u), 4);
             mbar_init(o_full(u), 1);
+            mbar_init(mma_done(u), 1);
         }
-        mbar_init(bar_mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -264,31 +266,30 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             for (int st = 0; st < STAGES; ++st)
                 if (kv_issued[st]) mbar_wait(kv_full(st), (kv_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x004);
         }
-    } else if (warp == kMma) {
+    } else if (warp >= kMma && warp < kMma + NSUB) {
         regs_decrease<L::control_regs>();
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ MMA issuer of row group u
+        const int u = warp - kMma;
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
             constexpr uint32_t IDESC_BIAS = idesc_bf16(BM, BN, false, true);   // B operand MN-major
             constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, false, true);
+            const uint32_t t_s = tmem + u * SUBCOLS + COL_S, t_p = tmem + u * SUBCOLS + COL_P,
+                           t_o = tmem + u * SUBCOLS + COL_O;
             bool ok = true;
             int tg = 0;
             int prev_st = 0, prev_j = 0;      // the tile whose PV is still to be issued
             bool pending = false;
             auto issue_pv = [&]() -> bool {   // PV of tile tg-1
                 const uint32_t sb = base + L::stage0 + prev_st * L::stage_bytes;
+                if (!mbar_wait(p_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x104)) return false;
+                tc_fence_after();
 #pragma unroll
-                for (int u = 0; u < NSUB; ++u) {
-                    if (!mbar_wait(p_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x104)) return false;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint64_t bd = smem_desc(sb + L::v_off(u) + kk * 1024, KV_BYTES, 512, kSw64);
-                        mma_ts(tmem + u * SUBCOLS + COL_O, tmem + u * SUBCOLS + COL_P + kk * 8, bd, IDESC_PV,
-                               (prev_j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(o_full(u));
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t bd = smem_desc(sb + L::v_off(u) + kk * 1024, KV_BYTES, 512, kSw64);
+                    mma_ts(t_o, t_p + kk * 8, bd, IDESC_PV, (prev_j > 0 || kk > 0) ? 1u : 0u);
                 }
+                mma_commit(o_full(u));
                 mma_commit(kv_empty(prev_st));
                 return true;
             };
@@ -299,33 +300,30 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     const int st = tg % STAGES;
                     const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
                     ok = mbar_wait(kv_full(st), (tg / STAGES) & 1, abort_flag, kTimeoutBase | 0x102);
+                    if (ok && tg > 0) ok = mbar_wait(s_free(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x103);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
-                    for (int u = 0; u < NSUB && ok; ++u) {
-                        if (tg > 0) ok = mbar_wait(s_free(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x103);
-                        if (!ok) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            const uint64_t ad = smem_desc(base + L::qbuf(qb, u) + kk * 32, 16, 512, kSw64);
-                            const uint64_t bd = smem_desc(sb + L::k_off(u) + kk * 32, 16, 512, kSw64);
-                            mma_ss(tmem + u * SUBCOLS + COL_S, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-                        }
-                        if (HAS_BIAS) {
-#pragma unroll
-                            for (int kk = 0; kk < BM / 16; ++kk) {   // + r * bias[i, j]
-                                const uint64_t ad = smem_desc(base + L::ident + kk * 256, 128, 2048, kSwNone);
-                                const uint64_t bd = smem_desc(sb + L::bias_off + kk * 2048, BIAS_BOX, 1024, kSw128);
-                                mma_ss(tmem + u * SUBCOLS + COL_S, ad, bd, IDESC_BIAS, 1u);
-                            }
-                        }
-                        if (HAS_MASK) {                               // + r * mask[s, j]
-                            const uint64_t ad = smem_desc(base + L::ones, 128, 256, kSwNone);
-                            const uint64_t bd = smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128);
-                            mma_ss(tmem + u * SUBCOLS + COL_S, ad, bd, IDESC_BIAS, 1u);
-                        }
-                        mma_commit(s_full(u));
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint64_t ad = smem_desc(base + L::qbuf(qb, u) + kk * 32, 16, 512, kSw64);
+                        const uint64_t bd = smem_desc(sb + L::k_off(u) + kk * 32, 16, 512, kSw64);
+                        mma_ss(t_s, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
                     }
-                    if (ok && pending) ok = issue_pv();
+                    if (HAS_BIAS) {
+#pragma unroll
+                        for (int kk = 0; kk < BM / 16; ++kk) {   // + r * bias[i, j]
+                            const uint64_t ad = smem_desc(base + L::ident + kk * 256, 128, 2048, kSwNone);
+                            const uint64_t bd = smem_desc(sb + L::bias_off + kk * 2048, BIAS_BOX, 1024, kSw128);
+                            mma_ss(t_s, ad, bd, IDESC_BIAS, 1u);
+                        }
+                    }
+                    if (HAS_MASK) {                               // + r * mask[s, j]
+                        const uint64_t ad = smem_desc(base + L::ones, 128, 256, kSwNone);
+                        const uint64_t bd = smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128);
+                        mma_ss(t_s, ad, bd, IDESC_BIAS, 1u);
+                    }
+                    mma_commit(s_full(u));
+                    if (pending) ok = issue_pv();
                     prev_st = st;
                     prev_j = j;
                     pending = true;
@@ -335,9 +333,9 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             }
             if (ok && pending) ok = issue_pv();
             // Drain: every MMA issued by this thread has finished before TMEM is released.
-            mma_commit(bar_mma_done);
+            mma_commit(mma_done(u));
             volatile int no_abort = 0;
-            mbar_wait(bar_mma_done, 0, &no_abort, kTimeoutBase | 0x105);
+            mbar_wait(mma_done(u), 0, &no_abort, kTimeoutBase | 0x105);
         }
     } else if (warp < 4 * NSUB) {
         regs_increase<L::softmax_regs>();
