@@ -10,9 +10,10 @@
 //   bwd_pre        per logit row: D_i = sum_c dout*out, dOa = dout*sigmoid(g)
 //                  split into a bf16 high part and a bf16 low part (their sum
 //                  carries ~16 mantissa bits into dP), dg = dout*out*(1-sigmoid(g)),
-//                  nl_i = -lse_i*log2(e); zeroes the fp32 dq accumulator.  The
-//                  row terms nl and -D are stored with the query axis padded to
-//                  whole tiles, padding nl = -inf, so padded queries get P = 0.
+//                  nl_i = -lse_i*sqrt(C); zeroes the fp32 dq accumulator.  Four
+//                  threads per row, 16-byte accesses.  The row terms nl and -D
+//                  are stored with the query axis padded to whole tiles, padding
+//                  nl = -1e30, so padded queries get P = 0.
 //   transpose_bias pair_bias[b,h,i,j] -> biasT[b,h,j,i] (bf16), so that the
 //                  main kernel reads bias rows along its TMEM lanes (keys).
 //   bwd_main       CTA = (key tile j, row group g, b*H + h); loops over the
@@ -538,63 +539,66 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bflo
     *lo = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
+constexpr int PRE_LANES = HD / 8;   // threads per logit row, 8 channels (16 bytes) each
+
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
     const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
     const int64_t pads = (int64_t)p.B * p.S * p.H * (p.n_pad - p.N);
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows + pads;
-         t += (int64_t)gridDim.x * blockDim.x) {
+    const int part = threadIdx.x % PRE_LANES;
+    const int64_t step = (int64_t)gridDim.x * (blockDim.x / PRE_LANES);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / PRE_LANES) + threadIdx.x / PRE_LANES; t < rows + pads;
+         t += step) {
         if (t >= rows) {   // padded query slots of the rank-term rows: P must come out 0
-            const int64_t u = t - rows;
-            const int w = p.n_pad - p.N;
-            const int64_t bsh = u / w;
-            const int i = p.N + (int)(u % w);
-            const int64_t o = bsh * 2 * p.n_pad + i;
-            p.nl[o] = __float2bfloat16_rn(-1e30f);
-            p.nl[o + p.n_pad] = __float2bfloat16_rn(0.f);
-            p.nd[o] = __float2bfloat16_rn(0.f);
-            p.nd[o + p.n_pad] = __float2bfloat16_rn(0.f);
+            if (part == 0) {
+                const int64_t u = t - rows;
+                const int w = p.n_pad - p.N;
+                const int64_t bsh = u / w;
+                const int i = p.N + (int)(u % w);
+                const int64_t o = bsh * 2 * p.n_pad + i;
+                p.nl[o] = __float2bfloat16_rn(-1e30f);
+                p.nl[o + p.n_pad] = __float2bfloat16_rn(0.f);
+                p.nd[o] = __float2bfloat16_rn(0.f);
+                p.nd[o + p.n_pad] = __float2bfloat16_rn(0.f);
+            }
             continue;
         }
         const int h = (int)(t % p.H);
         const int i = (int)((t / p.H) % p.N);
         const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
         const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
-        const uint4* o4 = reinterpret_cast<const uint4*>(p.out + p.os.off(b, s, i, h));
-        const uint4* d4 = reinterpret_cast<const uint4*>(p.dout + p.os.off(b, s, i, h));
-        const uint4* g4 = reinterpret_cast<const uint4*>(p.g + p.in.off(b, s, i, h));
-        uint4* dg4 = reinterpret_cast<uint4*>(p.dg + p.gs.off(b, s, i, h));
-        uint4* hi4 = reinterpret_cast<uint4*>(p.doa_hi + t * HD);
-        uint4* lo4 = reinterpret_cast<uint4*>(p.doa_lo + t * HD);
+        const uint4 ow = reinterpret_cast<const uint4*>(p.out + p.os.off(b, s, i, h))[part];
+        const uint4 dw = reinterpret_cast<const uint4*>(p.dout + p.os.off(b, s, i, h))[part];
+        const uint4 gw = reinterpret_cast<const uint4*>(p.g + p.in.off(b, s, i, h))[part];
+        const uint32_t ov[4] = {ow.x, ow.y, ow.z, ow.w}, dv[4] = {dw.x, dw.y, dw.z, dw.w},
+                       gv[4] = {gw.x, gw.y, gw.z, gw.w};
+        uint32_t dgv[4], hv[4], lv[4];
         float D = 0.f;
 #pragma unroll
-        for (int q = 0; q < HD / 8; ++q) {
-            const uint4 ow = o4[q], dw = d4[q], gw = g4[q];
-            const uint32_t ov[4] = {ow.x, ow.y, ow.z, ow.w}, dv[4] = {dw.x, dw.y, dw.z, dw.w},
-                           gv[4] = {gw.x, gw.y, gw.z, gw.w};
-            uint32_t dgv[4], hv[4], lv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float o0 = bf16lo(ov[e]), o1 = bf16hi(ov[e]);
-                const float d0 = bf16lo(dv[e]), d1 = bf16hi(dv[e]);
-                const float s0 = 1.0f / (1.0f + __expf(-bf16lo(gv[e]))), s1 = 1.0f / (1.0f + __expf(-bf16hi(gv[e])));
-                D = fmaf(d0, o0, D);
-                D = fmaf(d1, o1, D);
-                dgv[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
-                const float a0 = d0 * s0, a1 = d1 * s1;
-                hv[e] = pack_bf16(a0, a1);
-                lv[e] = pack_bf16(a0 - bf16lo(hv[e]), a1 - bf16hi(hv[e]));
-            }
-            dg4[q] = make_uint4(dgv[0], dgv[1], dgv[2], dgv[3]);
-            hi4[q] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            lo4[q] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        for (int e = 0; e < 4; ++e) {
+            const float o0 = bf16lo(ov[e]), o1 = bf16hi(ov[e]);
+            const float d0 = bf16lo(dv[e]), d1 = bf16hi(dv[e]);
+            const float s0 = 1.0f / (1.0f + __expf(-bf16lo(gv[e]))), s1 = 1.0f / (1.0f + __expf(-bf16hi(gv[e])));
+            D = fmaf(d0, o0, D);
+            D = fmaf(d1, o1, D);
+            dgv[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
+            const float a0 = d0 * s0, a1 = d1 * s1;
+            hv[e] = pack_bf16(a0, a1);
+            lv[e] = pack_bf16(a0 - bf16lo(hv[e]), a1 - bf16hi(hv[e]));
         }
-        const int64_t bsh = ((int64_t)b * p.S + s) * p.H + h;
-        const int64_t o = bsh * 2 * p.n_pad + i;
-        split_bf16(-D, p.nd + o, p.nd + o + p.n_pad);
-        split_bf16(-p.lse[bsh * p.N + i] * p.sqrt_c, p.nl + o, p.nl + o + p.n_pad);
-        float4* acc = reinterpret_cast<float4*>(p.dq_acc + t * HD);
+        reinterpret_cast<uint4*>(p.dg + p.gs.off(b, s, i, h))[part] = make_uint4(dgv[0], dgv[1], dgv[2], dgv[3]);
+        reinterpret_cast<uint4*>(p.doa_hi + t * HD)[part] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        reinterpret_cast<uint4*>(p.doa_lo + t * HD)[part] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        float4* acc = reinterpret_cast<float4*>(p.dq_acc + t * HD) + 2 * part;
+        acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < HD / 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 1; m < PRE_LANES; m <<= 1) D += __shfl_xor_sync(0xffffffffu, D, m);
+        if (part == 0) {
+            const int64_t bsh = ((int64_t)b * p.S + s) * p.H + h;
+            const int64_t o = bsh * 2 * p.n_pad + i;
+            split_bf16(-D, p.nd + o, p.nd + o + p.n_pad);
+            split_bf16(-p.lse[bsh * p.N + i] * p.sqrt_c, p.nl + o, p.nl + o + p.n_pad);
+        }
     }
 }
 
@@ -729,7 +733,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     pp.g = static_cast<const __nv_bfloat16*>(c.g); pp.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
     pp.lse = c.lse; pp.dg = static_cast<__nv_bfloat16*>(c.dg); pp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
     pp.doa_hi = doa; pp.doa_lo = dol; pp.nl = nl; pp.nd = nd; pp.dq_acc = dq_acc;
-    bwd_pre_kernel<<<grid_for(rows + (int64_t)B * S * H * (n_pad - N), 256), 256, 0, stream>>>(pp);
+    bwd_pre_kernel<<<grid_for((rows + (int64_t)B * S * H * (n_pad - N)) * PRE_LANES, 256), 256, 0, stream>>>(pp);
     ++*launched;
     if (c.bias) {
         transpose_bias_kernel<<<dim3((N + 31) / 32, (N + 31) / 32, B * H), dim3(32, 8), 0, stream>>>(
