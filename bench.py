@@ -284,6 +284,21 @@ def oracle_threads() -> int:
         return os.cpu_count()
 
 
+def max_over_ranks(vals, world: int, device) -> list:
+    """Element-wise maximum of per-rank timings (device time: the slowest rank decides)."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's time."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
@@ -395,19 +410,13 @@ def main():
     fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     tot_ms = sum(fwd_ms) + sum(bwd_ms)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([tot_ms, sum(fwd_ms), sum(bwd_ms)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, fsum, bsum = t.tolist()
-    else:
-        fsum, bsum = sum(fwd_ms), sum(bwd_ms)
+    tot_ms, fsum, bsum = max_over_ranks([tot_ms, sum(fwd_ms), sum(bwd_ms)], world, dev)
     if A.device_status(clear=True) != 0:
         raise RuntimeError("a kernel reported a timed-out wait during the timed region")
 
     ff, bf = flops(w)
     pk = peaks()
-    value = (ff + bf) * K * world / (tot_ms * 1e-3) / 1e12
+    value = job_throughput(ff + bf, K, world, tot_ms)
     fwd_tf = ff * K / (fsum * 1e-3) / 1e12
     bwd_tf = bf * K / (bsum * 1e-3) / 1e12
 
@@ -452,12 +461,8 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         et = e0.elapsed_time(e1)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([et], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            et = t.item()
-        e2e = {"value": (ff + bf) * K * world / (et * 1e-3) / 1e12, "unit": "TFLOP/s",
+        et = max_over_ranks([et], world, dev)[0]
+        e2e = {"value": job_throughput(ff + bf, K, world, et), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": et / K}
 
     cpu = None
