@@ -7,16 +7,16 @@
 // flash-style, online-softmax treatment EvoFlash-3D gives this op in the
 // MegaFold summary, section "EvoFlash-3D").
 //
-// The biases are added by the tensor core, not by the softmax threads:
-//   S_u = Q_u K_u^T + (r I) B + (r e_0) m_u^T,        r = bf16(sqrt(C))
-// accumulates, in fp32 TMEM, the logits scaled by sqrt(C): I is a constant
-// identity tile, B the pair-bias tile (TMA-loaded once per key tile and shared
-// by all NSUB rows s -- it is the same for every s), and the last term is one
-// 16-deep K step whose B block carries the mask row of row s in its first
-// row.  Products with the exact bf16 inputs are exact in fp32, so the biases
-// enter with only the relative error of r/sqrt(C) (1.1e-4 for C = 32; exact
-// for C = 16 or 64).  The softmax threads then need one fused multiply-add
-// per logit before the exponential.
+// The mask row is added by the tensor core:
+//   S_u = Q_u K_u^T + (r e_0) m_u^T,        r = bf16(sqrt(C))
+// accumulates, in fp32 TMEM, sqrt(C) times the logit without the pair bias:
+// the last term is one 16-deep K step whose B block carries the mask row of
+// row s in its first row (exact products in fp32; the mask enters with the
+// relative error of r/sqrt(C), 1.1e-4 for C = 32).  The pair-bias tile
+// (TMA-loaded once per key tile and shared by all NSUB rows s -- it is the
+// same for every s) is added by the softmax threads from shared memory, one
+// fused multiply-add per logit pair, while the other row group has its turn
+// on the exponentials (see below).
 //
 // Warp roles (128*NSUB + 128 threads; the last warpgroup gives up registers
 // to the softmax warpgroups with setmaxnreg):
@@ -30,12 +30,15 @@
 //            tile is issued before the PV of the current one, so it overlaps
 //            the softmax; one issuer per row group keeps the groups' pipelines
 //            independent of each other.
-//   softmax: thread = query row.  Load S
-//            from TMEM, online max and sum in fp32 with a lazy rescale (the
+//   softmax: thread = query row.  Load S from TMEM and add the pair-bias
+//            row, online max and sum in fp32 with a lazy rescale (the
 //            running max moves only when a tile's max exceeds it by more than
 //            2^8), P (bf16) back to TMEM, and at the end of the item
-//            out = sigmoid(g) * O / l, lse = log(l) + max.
-// TMEM per row s: S 128 columns, P 64 columns (bf16 pairs), O 32 columns.
+//            out = sigmoid(g) * O / l, lse = log(l) + max.  The two row
+//            groups take turns on the exponentials (the MUFU unit is the
+//            scarce resource at C = 32): each group's loads, bias adds and
+//            maxima overlap the other group's exponentials.
+// TMEM per row s: S 128 columns, P 64 columns (bf16 pairs), O 2 x 32 columns.
 #pragma once
 
 #include "sm100.cuh"
@@ -54,18 +57,25 @@ constexpr int KV_BYTES = BN * HD * 2;   // 8 KB each for K and V
 constexpr int BIAS_BOX = BM * 64 * 2;   // 16 KB: 128 rows x 64 keys, 128B swizzle
 constexpr int BIAS_BYTES = 2 * BIAS_BOX;
 constexpr int MASKB_BYTES = 4096;       // 16 x 128 bf16 B block (row 0 = mask row), 128B swizzle
-constexpr int IDENT_BYTES = 128 * 128 * 2;   // r * I, K-major, no swizzle
 constexpr int ONES_BYTES = 128 * 16 * 2;     // r * e_0 column, K-major, no swizzle
+// per row group: S, P, and two O accumulators (items alternate between them,
+// so an item's epilogue can run after the next item's first tile)
 constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192, SUBCOLS = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+// Every POLY_EVERY-th pair of exponentials of a row runs on the FMA pipe
+// (exp2_poly2) instead of the MUFU unit, which at C = 32 is the scarcest unit;
+// 0 keeps every exponential on MUFU.
+#ifndef EVO_FWD_POLY_EVERY
+#define EVO_FWD_POLY_EVERY 0
+#endif
+constexpr int POLY_EVERY = EVO_FWD_POLY_EVERY;
 
 __host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / a * a; }
 
 template <int NSUB>
 struct Layout {
     static constexpr int qbuf(int k, int u) { return (k * NSUB + u) * Q_BYTES; }   // per item parity k
-    static constexpr int ident = 2 * NSUB * Q_BYTES;
-    static constexpr int ones = ident + IDENT_BYTES;
+    static constexpr int ones = 2 * NSUB * Q_BYTES;
     static constexpr int stage0 = round_up(ones + ONES_BYTES, 1024);
     static constexpr int k_off(int u) { return u * KV_BYTES; }
     static constexpr int v_off(int u) { return (NSUB + u) * KV_BYTES; }
@@ -73,8 +83,9 @@ struct Layout {
     static constexpr int maskb_off(int u) { return bias_off + BIAS_BYTES + u * MASKB_BYTES; }
     static constexpr int stage_bytes = round_up(bias_off + BIAS_BYTES + NSUB * MASKB_BYTES, 1024);
     static constexpr int bars = stage0 + STAGES * stage_bytes;
-    // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[u], s_free[u], p_full[u], o_full[u], mma_done[u]
-    static constexpr int nbars = 4 + 2 * STAGES + 5 * NSUB;
+    // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[u], s_free[u], p_full[u], o_full[u],
+    // mma_done[u], exp_turn[u]
+    static constexpr int nbars = 4 + 2 * STAGES + 6 * NSUB;
     static constexpr int misc = bars + nbars * 8;   // tmem base (u32), abort flag (u32)
     static constexpr int bytes = misc + 16 + 1024;  // + slack to align the base to 1024
     static constexpr uint32_t tmem_cols = NSUB == 1 ? 256 : 512;
@@ -94,7 +105,7 @@ struct Params {
     int n_sg;                 // row groups of NSUB rows
     int n_items;              // B * H * n_sg * n_it
     float scale;              // 1/sqrt(C)
-    float r_bf16;             // bf16(sqrt(C)), the diagonal of the identity tile
+    float r_bf16;             // bf16(sqrt(C)), the nonzero of the mask MMA column
     const __nv_bfloat16* g;   // gate, strides `in`
     Strides in;
     __nv_bfloat16* out;       // strides `os`
@@ -146,6 +157,8 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     auto p_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 2 * NSUB + u); };
     auto o_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 3 * NSUB + u); };
     auto mma_done = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 4 * NSUB + u); };
+    // exp_turn[u]: row group u may start the exponentials of its next tile
+    auto exp_turn = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 5 * NSUB + u); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::misc + 4);
 
@@ -164,6 +177,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             mbar_init(p_full(u), 4);
             mbar_init(o_full(u), 1);
             mbar_init(mma_done(u), 1);
+            mbar_init(exp_turn(u), 4);             // one arrival per warp of the other group
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -180,15 +194,13 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         tmem_relinquish();
     }
     if (warp < 4 * NSUB) {
-        // Constant MMA operands (element (row, k) of a no-swizzle K-major tile is
+        // Constant MMA operand (element (row, k) of a no-swizzle K-major tile is
         // at (row % 8) * 16 + (row / 8) * SBO + (k / 8) * 128 + (k % 8) * 2):
-        //   identity r*I (SBO 2048), column r*e_0 (SBO 256), and rows 1..15 of
-        //   every mask block zero (the TMA writes row 0 each stage).
+        //   column r*e_0 (SBO 256), and rows 1..15 of every mask block zero
+        //   (the TMA writes row 0 each stage).
         const int t = threadIdx.x;
         const int nt = 128 * NSUB;
         const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
-        for (int o = t * 16; o < IDENT_BYTES; o += nt * 16)
-            *reinterpret_cast<uint4*>(gbase + L::ident + o) = make_uint4(0u, 0u, 0u, 0u);
         for (int o = t * 16; o < ONES_BYTES; o += nt * 16)
             *reinterpret_cast<uint4*>(gbase + L::ones + o) = make_uint4(0u, 0u, 0u, 0u);
         for (int st = 0; st < STAGES; ++st)
@@ -200,8 +212,6 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");
         if (t < 128) {
             const int rr = t;
-            *reinterpret_cast<uint16_t*>(gbase + L::ident + (rr % 8) * 16 + (rr / 8) * 2048 + (rr / 8) * 128 +
-                                         (rr % 8) * 2) = rb;
             *reinterpret_cast<uint16_t*>(gbase + L::ones + (rr % 8) * 16 + (rr / 8) * 256) = rb;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -272,13 +282,13 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         const int u = warp - kMma;
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
-            constexpr uint32_t IDESC_BIAS = idesc_bf16(BM, BN, false, true);   // B operand MN-major
+            constexpr uint32_t IDESC_MASK = idesc_bf16(BM, BN, false, true);   // B operand MN-major
             constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, false, true);
             const uint32_t t_s = tmem + u * SUBCOLS + COL_S, t_p = tmem + u * SUBCOLS + COL_P,
                            t_o = tmem + u * SUBCOLS + COL_O;
             bool ok = true;
             int tg = 0;
-            int prev_st = 0, prev_j = 0;      // the tile whose PV is still to be issued
+            int prev_st = 0, prev_j = 0, prev_k = 0;   // the tile whose PV is still to be issued
             bool pending = false;
             auto issue_pv = [&]() -> bool {   // PV of tile tg-1
                 const uint32_t sb = base + L::stage0 + prev_st * L::stage_bytes;
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bd = smem_desc(sb + L::v_off(u) + kk * 1024, KV_BYTES, 512, kSw64);
-                    mma_ts(t_o, t_p + kk * 8, bd, IDESC_PV, (prev_j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(t_o + (uint32_t)(prev_k & 1) * HD, t_p + kk * 8, bd, IDESC_PV, (prev_j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(o_full(u));
                 mma_commit(kv_empty(prev_st));
@@ -309,23 +319,16 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                         const uint64_t bd = smem_desc(sb + L::k_off(u) + kk * 32, 16, 512, kSw64);
                         mma_ss(t_s, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
                     }
-                    if (HAS_BIAS) {
-#pragma unroll
-                        for (int kk = 0; kk < BM / 16; ++kk) {   // + r * bias[i, j]
-                            const uint64_t ad = smem_desc(base + L::ident + kk * 256, 128, 2048, kSwNone);
-                            const uint64_t bd = smem_desc(sb + L::bias_off + kk * 2048, BIAS_BOX, 1024, kSw128);
-                            mma_ss(t_s, ad, bd, IDESC_BIAS, 1u);
-                        }
-                    }
                     if (HAS_MASK) {                               // + r * mask[s, j]
                         const uint64_t ad = smem_desc(base + L::ones, 128, 256, kSwNone);
                         const uint64_t bd = smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128);
-                        mma_ss(t_s, ad, bd, IDESC_BIAS, 1u);
+                        mma_ss(t_s, ad, bd, IDESC_MASK, 1u);
                     }
                     mma_commit(s_full(u));
                     if (pending) ok = issue_pv();
                     prev_st = st;
                     prev_j = j;
+                    prev_k = k;
                     pending = true;
                     ++tg;
                 }
@@ -344,27 +347,72 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;          // query row within the tile = TMEM lane
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + u * SUBCOLS;
-        // S holds sqrt(C) * x; exponents are taken as exp2(S * sc2 - ms), sc2 = log2(e)/sqrt(C)
+        // S holds sqrt(C) * (q.k / sqrt(C) + mask); the logit in log2 units is
+        // y = S * sc2 + bias * log2(e), sc2 = log2(e)/sqrt(C); exponents are exp2(y - ms)
         const float sc2 = p.scale * EVO_LOG2E;
         const uint64_t SC2 = f2(sc2, sc2);
+        const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
         bool ok = true;
         int tg = 0;
+        // The epilogue of an item (out = sigmoid(g) * O / l, lse) is deferred to
+        // after the first tile of the next item: by then the item's last PV is
+        // complete (that tile waited for it), so no thread idles on it.
+        struct Epi {
+            bool pending, row_ok;
+            int b, s, i, h, obuf;
+            float l, ms;
+        } epi;
+        epi.pending = false;
+        auto run_epilogue = [&]() {
+            // the gate row (prefetched into L2 during the item's last tile)
+            uint4 gw[HD / 8];
+            if (epi.row_ok) {
+                const uint4* gp = reinterpret_cast<const uint4*>(p.g + p.in.off(epi.b, epi.s, epi.i, epi.h));
+#pragma unroll
+                for (int q = 0; q < HD / 8; ++q) gw[q] = __ldg(gp + q);
+            }
+            uint32_t o[HD];
+            tmem_ld32_sync(lane_addr + COL_O + (uint32_t)epi.obuf * HD, o);
+            if (epi.row_ok) {
+                __nv_bfloat16* op = p.out + p.os.off(epi.b, epi.s, epi.i, epi.h);
+#pragma unroll
+                for (int q = 0; q < HD / 8; ++q) {
+                    const uint32_t gv[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
+                    uint32_t ov[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // out = O / (l * (1 + exp(-g))): the backward's D = sum(dout * out)
+                        // feeds a cancellation, so the gate is computed accurately
+                        // (exp on the FMA pipe, relative error < 8e-5; arguments
+                        // clamped to the exponent range, exp(-g) <= 2^126).
+                        const uint64_t ng = f2(fminf(-EVO_LOG2E * bf16lo(gv[e]), 126.0f),
+                                               fminf(-EVO_LOG2E * bf16hi(gv[e]), 126.0f));
+                        const uint64_t eg = exp2_poly2(ng);
+                        const float e0 = f2lo(eg), e1 = f2hi(eg);
+                        const float o0 = __fdividef(__uint_as_float(o[q * 8 + 2 * e]), epi.l * (1.0f + e0));
+                        const float o1 = __fdividef(__uint_as_float(o[q * 8 + 2 * e + 1]), epi.l * (1.0f + e1));
+                        ov[e] = pack_bf16(o0, o1);
+                    }
+                    *reinterpret_cast<uint4*>(op + q * 8) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+                }
+                p.lse[((int64_t)(epi.b * p.S + epi.s) * p.H + epi.h) * p.N + epi.i] =
+                    (epi.ms + __log2f(epi.l)) * EVO_LN2;
+            }
+            epi.pending = false;
+        };
         for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
             const Item itm = decode(p, item);
             const int s = itm.sg * NSUB + u;
             const int i = itm.i0 + r;
             const bool row_ok = s < p.S && i < p.N;
-            (void)k;
-            uint4 gw[HD / 8];
+            const uint32_t col_o = COL_O + (uint32_t)(k & 1) * HD;
             // ms: running max in log2 units (the value subtracted inside exp2);
             // l: running sum of exp2(S * sc2 - ms)
             float ms = -INFINITY, l = 0.f;
             for (int j = 0; j < p.n_kv; ++j, ++tg) {
                 if (j == p.n_kv - 1 && row_ok) {
-                    // the gate row is only needed at the end of the item: fetch it during the last tile
-                    const uint4* gp = reinterpret_cast<const uint4*>(p.g + p.in.off(itm.b, s, i, itm.h));
-#pragma unroll
-                    for (int q = 0; q < HD / 8; ++q) gw[q] = __ldg(gp + q);
+                    // the gate row is only needed by the item's epilogue: start bringing it into L2
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.g + p.in.off(itm.b, s, i, itm.h)));
                 }
                 ok = mbar_wait(s_full(u), tg & 1, abort_flag, kTimeoutBase | 0x201);
                 if (!ok) break;
@@ -375,6 +423,34 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_free(u));
 
+                // y = S * sc2 + bias * log2(e): the pair-bias row of this query from
+                // the stage's tile (two 64-key boxes, 128B swizzle: 16-byte chunk c
+                // of row r sits at chunk c ^ (r & 7)), two logits per instruction
+                if (HAS_BIAS) {
+                    // acquire the TMA writes of this stage (already complete: S used them)
+                    ok = mbar_wait(kv_full(tg % STAGES), (tg / STAGES) & 1, abort_flag, kTimeoutBase | 0x206);
+                    if (!ok) break;
+                }
+                {
+                    const int st = tg % STAGES;
+                    const uint8_t* brow = gbase + L::stage0 + st * L::stage_bytes + L::bias_off + r * 128;
+#pragma unroll
+                    for (int q = 0; q < BN / 8; ++q) {
+                        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                        if (HAS_BIAS)
+                            w = *reinterpret_cast<const uint4*>(brow + (q >> 3) * BIAS_BOX +
+                                                                ((((uint32_t)q & 7u) ^ (uint32_t)(r & 7)) << 4));
+                        const uint32_t bw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int c = q * 8 + 2 * e;
+                            uint64_t y2 = fmul2(f2(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), SC2);
+                            if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[e]), L2E2, y2);
+                            xr[c] = __float_as_uint(f2lo(y2));
+                            xr[c + 1] = __float_as_uint(f2hi(y2));
+                        }
+                    }
+                }
                 const int valid = p.N - j * BN;      // keys beyond N are padding: exclude them
                 if (valid < BN) {
 #pragma unroll
@@ -392,7 +468,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 
                 // lazy rescale: move the running max only when this tile's max exceeds it by > 2^8
-                const float mcand = mloc * sc2;
+                const float mcand = mloc;
                 const bool move = mcand > ms + RESCALE_THRESHOLD;
                 const float ms_new = move ? mcand : ms;
                 const float alpha = move ? ex2(ms - ms_new) : 1.0f;   // 0 on an item's first tile
@@ -404,10 +480,19 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 }
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
                     uint32_t o[HD];
-                    tmem_ld32_sync(lane_addr + COL_O, o);
+                    tmem_ld32_sync(lane_addr + col_o, o);
 #pragma unroll
                     for (int c = 0; c < HD; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st32(lane_addr + COL_O, o);
+                    tmem_st32(lane_addr + col_o, o);
+                }
+                // The two row groups take turns on the exponentials (MUFU): group 1
+                // runs tile t after group 0's tile t, group 0 runs tile t+1 after
+                // group 1's tile t, so one group's exponentials overlap the other's
+                // loads, maxima and waits instead of competing with its exponentials.
+                if (NSUB == 2) {
+                    if (u == 1) ok = mbar_wait(exp_turn(1), tg & 1, abort_flag, kTimeoutBase | 0x205);
+                    else if (tg > 0) ok = mbar_wait(exp_turn(0), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x205);
+                    if (!ok) break;
                 }
                 const uint64_t NEG_MS2 = f2(-ms_new, -ms_new);
                 uint64_t rs2[2] = {0, 0};
@@ -418,13 +503,21 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     for (int cc = 0; cc < BN / 4; ++cc) {
                         const int c = half * (BN / 4) + cc;
                         const uint64_t y2 =
-                            ffma2(f2(__uint_as_float(xr[2 * c]), __uint_as_float(xr[2 * c + 1])), SC2, NEG_MS2);
-                        const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
-                        const uint64_t pp = f2(p0, p1);
+                            fadd2(f2(__uint_as_float(xr[2 * c]), __uint_as_float(xr[2 * c + 1])), NEG_MS2);
+                        uint64_t pp;
+                        if (POLY_EVERY > 0 && c % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1)
+                            pp = exp2_poly2(y2);
+                        else
+                            pp = f2(ex2(f2lo(y2)), ex2(f2hi(y2)));
+                        const float p0 = f2lo(pp), p1 = f2hi(pp);
                         rs2[c & 1] = (c < 2) ? pp : fadd2(rs2[c & 1], pp);
                         pk[cc] = pack_bf16(p0, p1);
                     }
                     tmem_st32(lane_addr + COL_P + half * 32, pk);
+                }
+                if (NSUB == 2) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(exp_turn(1 - u));
                 }
                 const uint64_t rsum = fadd2(rs2[0], rs2[1]);
                 l = fmaf(l, alpha, f2lo(rsum) + f2hi(rsum));
@@ -433,32 +526,21 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full(u));
+                // the previous item's epilogue: its last PV finished before this
+                // tile's P was written (the o_full wait above)
+                if (j == 0 && epi.pending) run_epilogue();
             }
             if (!ok) break;
-            // ---------------------------------------------------------- epilogue of this item
+            epi.pending = true;
+            epi.row_ok = row_ok;
+            epi.b = itm.b; epi.s = s; epi.i = i; epi.h = itm.h; epi.obuf = k & 1;
+            epi.l = l; epi.ms = ms;
+        }
+        if (ok && epi.pending) {   // the last item: wait for its last PV
             ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x204);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t o[HD];
-            tmem_ld32_sync(lane_addr + COL_O, o);
-            if (row_ok) {
-                __nv_bfloat16* op = p.out + p.os.off(itm.b, s, i, itm.h);
-#pragma unroll
-                for (int q = 0; q < HD / 8; ++q) {
-                    const uint32_t gv[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
-                    uint32_t ov[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        // out = O / (l * (1 + exp(-g))): the backward's D = sum(dout * out)
-                        // feeds a cancellation, so the gate is computed accurately.
-                        const float e0 = ex2(-EVO_LOG2E * bf16lo(gv[e])), e1 = ex2(-EVO_LOG2E * bf16hi(gv[e]));
-                        const float o0 = __fdividef(__uint_as_float(o[q * 8 + 2 * e]), l * (1.0f + e0));
-                        const float o1 = __fdividef(__uint_as_float(o[q * 8 + 2 * e + 1]), l * (1.0f + e1));
-                        ov[e] = pack_bf16(o0, o1);
-                    }
-                    *reinterpret_cast<uint4*>(op + q * 8) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-                }
-                p.lse[((int64_t)(itm.b * p.S + s) * p.H + itm.h) * p.N + i] = (ms + __log2f(l)) * EVO_LN2;
+            if (ok) {
+                tc_fence_after();
+                run_epilogue();
             }
         }
     }

@@ -249,6 +249,30 @@ __device__ __forceinline__ void tmem_ld32x4_sync(uint32_t a0, uint32_t a1, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3)
         : "memory");
 }
+// Two back-to-back x32 loads (columns from a0 and from a1), then one wait.
+__device__ __forceinline__ void tmem_ld32x2_sync(uint32_t a0, uint32_t a1, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(a0), "r"(a1)
+        : "memory");
+}
+// 16x256b shape, .x2: a warp reads 16 TMEM lanes (from the address's lane) x
+// 16 columns.  Thread t receives, for lanes L = t/4 and L + 8 and columns
+// c = 2*(t%4), 2*(t%4)+1 (then the same 8 columns further on):
+//   r[0], r[1] = (L, c), (L, c+1)        r[2], r[3] = (L+8, c), (L+8, c+1)
+//   r[4], r[5] = (L, c+8), (L, c+9)      r[6], r[7] = (L+8, c+8), (L+8, c+9)
+// so four consecutive threads hold 8 consecutive columns (32 bytes) of a lane.
+__device__ __forceinline__ void tmem_ld16x256b_x2_sync(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
         ::"r"(taddr),
@@ -338,6 +362,30 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for a pair of arguments on the FMA pipe instead of the MUFU unit.
+// Method: split x = n + f with n = round(x) by the classic float-rounding
+// constant 1.5 * 2^23 (adding it leaves round(x) in the low mantissa bits),
+// f = x - n in [-1/2, 1/2]; 2^f from a cubic fitted (weighted least squares
+// toward minimax, on [-1/2, 1/2]) with relative error below 8e-5; 2^n is
+// added to the exponent field of the result as an integer.  Arguments are
+// clamped at -125 so every result is a normal float (2^-125 stands in for an
+// underflow, e.g. a masked key's exp2(-inf)); valid for x <= 126.
+constexpr float kExp2Round = 12582912.0f;                       // 1.5 * 2^23
+constexpr float kExp2C0 = 0.9999284744f, kExp2C1 = 0.6932614446f, kExp2C2 = 0.2426052243f,
+                kExp2C3 = 0.0551665500f;
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    const uint64_t xc = f2(fmaxf(f2lo(x2), -125.0f), fmaxf(f2hi(x2), -125.0f));
+    const uint64_t r = fadd2(xc, f2(kExp2Round, kExp2Round));                 // round(x) in the low bits
+    const uint64_t n = fadd2(r, f2(-kExp2Round, -kExp2Round));
+    const uint64_t f = ffma2(n, f2(-1.0f, -1.0f), xc);                        // x - round(x)
+    uint64_t p = ffma2(f2(kExp2C3, kExp2C3), f, f2(kExp2C2, kExp2C2));
+    p = ffma2(p, f, f2(kExp2C1, kExp2C1));
+    p = ffma2(p, f, f2(kExp2C0, kExp2C0));
+    const uint32_t lo = __float_as_uint(f2lo(p)) + (__float_as_uint(f2lo(r)) << 23);
+    const uint32_t hi = __float_as_uint(f2hi(p)) + (__float_as_uint(f2hi(r)) << 23);
+    return f2(__uint_as_float(lo), __uint_as_float(hi));
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
