@@ -7,15 +7,17 @@
 // forward and the backward passes).
 //
 // Kernels (one stream, in order):
-//   bwd_pre        per logit row: D_i = sum_c dout*out, dOa = dout*sigmoid(g)
+//   bwd_prep       one launch, by block range:
+//                  per logit row: D_i = sum_c dout*out, dOa = dout*sigmoid(g)
 //                  split into a bf16 high part and a bf16 low part (their sum
 //                  carries ~16 mantissa bits into dP), dg = dout*out*(1-sigmoid(g)),
 //                  nl_i = -lse_i*sqrt(C); zeroes the fp32 dq accumulator.  Four
 //                  threads per row, 16-byte accesses.  The row terms nl and -D
 //                  are stored with the query axis padded to whole tiles, padding
-//                  nl = -1e30, so padded queries get P = 0.
-//   transpose_bias pair_bias[b,h,i,j] -> biasT[b,h,j,i] (bf16), so that the
-//                  main kernel reads bias rows along its TMEM lanes (keys).
+//                  nl = -1e30, so padded queries get P = 0;
+//                  pair_bias[b,h,i,j] -> biasT[b,h,j,i] (bf16), so that the
+//                  main kernel reads bias rows along its TMEM lanes (keys);
+//                  the d_pair_bias partial slabs cleared.
 //   bwd_main       CTA = (key tile j, row group g, b*H + h); loops over the
 //                  group's rows s (outer) and query tiles i (inner):
 //                    S^T  = K_j Q_i^T      dP^T = V_j (dOa_hi + dOa_lo)_i^T  (TMEM)
@@ -28,8 +30,8 @@
 //                  The dS^T smem tile and the P^T TMEM tile are double-buffered
 //                  by step parity, so the dS warps write step t while the MMAs of
 //                  step t-1 still read the other buffer.
-//   bwd_post       dq = bf16(accumulator); d_pair_bias = sum over g of the
-//                  partials in index order (skipped when there is one group).
+//   bwd_post       one launch: dq = bf16(accumulator); d_pair_bias = sum over
+//                  g of the partials in index order (when there are several).
 // The result of d_pair_bias is therefore bitwise reproducible; dq's last bits
 // depend on the order of the atomic adds.
 #pragma once
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t sb = base + OFF_ST + st * STB;
-            const uint32_t bt_addr = sb + ST_BT + wg * BT_BOX + r * 128;
+            const uint8_t* bt_ptr = gbase + (sb - base) + ST_BT + wg * BT_BOX + r * 128;
             const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * 32;
             // d_pair_bias partial (zeroed before the launch).  Each address of this
             // group's slab is updated by exactly one thread, in row order s, with
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int q = 0; q < 8; ++q) {                      // 8 columns at a time
                 uint32_t bw[4] = {0u, 0u, 0u, 0u};
                 if (HAS_BIAS) {
-                    const uint4 w = lds128(bt_addr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
+                    const uint4 w = *reinterpret_cast<const uint4*>(bt_ptr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
                     bw[0] = w.x; bw[1] = w.y; bw[2] = w.z; bw[3] = w.w;
                 }
                 float dsq[8];
@@ -459,21 +461,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                     dk2[q * 4 + e] = pack_bf16(dsq[2 * e], dsq[2 * e + 1]);
                 }
                 asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt_addr + q * 4),
-                             "r"(pk4[0]), "r"(pk4[1]), "r"(pk4[2]), "r"(pk4[3])
-                             : "memory");
+                             "r"(pk4[0]), "r"(pk4[1]), "r"(pk4[2]), "r"(pk4[3]));
+                // (no "memory" clobber: nothing in this kernel reads the slab)
                 if (ivalid >= 64) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (q * 8 + e) * rstride),
-                                     "f"(dsq[e])
-                                     : "memory");
+                                     "f"(dsq[e]));
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         if (q * 8 + e < ivalid)
                             asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (q * 8 + e) * rstride),
-                                         "f"(dsq[e])
-                                         : "memory");
+                                         "f"(dsq[e]));
                 }
             }
             __syncwarp();
@@ -541,12 +541,12 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bflo
 
 constexpr int PRE_LANES = HD / 8;   // threads per logit row, 8 channels (16 bytes) each
 
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
+__device__ __forceinline__ void pre_rows(const PreParams& p, int blk, int nblk) {
     const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
     const int64_t pads = (int64_t)p.B * p.S * p.H * (p.n_pad - p.N);
     const int part = threadIdx.x % PRE_LANES;
-    const int64_t step = (int64_t)gridDim.x * (blockDim.x / PRE_LANES);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / PRE_LANES) + threadIdx.x / PRE_LANES; t < rows + pads;
+    const int64_t step = (int64_t)nblk * (blockDim.x / PRE_LANES);
+    for (int64_t t = (int64_t)blk * (blockDim.x / PRE_LANES) + threadIdx.x / PRE_LANES; t < rows + pads;
          t += step) {
         if (t >= rows) {   // padded query slots of the rank-term rows: P must come out 0
             if (part == 0) {
@@ -602,21 +602,54 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const PreParams p) {
     }
 }
 
-// biasT[b,h,j,i] = pair_bias[b,h,i,j]  (32x32 tiles through shared memory)
-__global__ void __launch_bounds__(256) transpose_bias_kernel(const __nv_bfloat16* __restrict__ src,
-                                                             __nv_bfloat16* __restrict__ dst, int N) {
-    __shared__ __nv_bfloat16 tile[32][33];
-    const int64_t plane = (int64_t)blockIdx.z * N * N;
-    const int bx = blockIdx.x * 32, by = blockIdx.y * 32;
-    for (int y = threadIdx.y; y < 32; y += 8) {
-        const int i = by + y, jj = bx + threadIdx.x;
-        if (i < N && jj < N) tile[y][threadIdx.x] = src[plane + (int64_t)i * N + jj];
+// biasT[b,h,j,i] = pair_bias[b,h,i,j]: one 32x32 tile through shared memory
+// (256 threads as 32 x 8).
+__device__ __forceinline__ void transpose_tile(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                               int N, int tile) {
+    __shared__ __nv_bfloat16 buf[32][33];
+    const int nt = (N + 31) / 32;
+    const int64_t plane = (int64_t)(tile / (nt * nt)) * N * N;
+    const int bx = (tile % nt) * 32, by = ((tile / nt) % nt) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int y = ty; y < 32; y += 8) {
+        const int i = by + y, jj = bx + tx;
+        if (i < N && jj < N) buf[y][tx] = src[plane + (int64_t)i * N + jj];
     }
     __syncthreads();
-    for (int y = threadIdx.y; y < 32; y += 8) {
-        const int jj = bx + y, i = by + threadIdx.x;
-        if (i < N && jj < N) dst[plane + (int64_t)jj * N + i] = tile[threadIdx.x][y];
+    for (int y = ty; y < 32; y += 8) {
+        const int jj = bx + y, i = by + tx;
+        if (i < N && jj < N) dst[plane + (int64_t)jj * N + i] = buf[tx][y];
     }
+}
+
+// The backward's preparation in one launch, by block range: the per-row pass
+// (pre_rows), the pair-bias transpose (one tile per block) and the clearing of
+// the d_pair_bias partial slabs.
+struct PrepParams {
+    PreParams pre;
+    int nb_pre;
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* biast;
+    int nb_tr;                // transpose tiles (0 without a pair bias)
+    float4* zero;             // partial slabs to clear
+    int64_t n_zero4;
+};
+
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams pp) {
+    int blk = blockIdx.x;
+    if (blk < pp.nb_pre) {
+        pre_rows(pp.pre, blk, pp.nb_pre);
+        return;
+    }
+    blk -= pp.nb_pre;
+    if (blk < pp.nb_tr) {
+        transpose_tile(pp.bias, pp.biast, pp.pre.N, blk);
+        return;
+    }
+    blk -= pp.nb_tr;
+    const int nb_zero = (int)gridDim.x - pp.nb_pre - pp.nb_tr;
+    for (int64_t t = (int64_t)blk * blockDim.x + threadIdx.x; t < pp.n_zero4; t += (int64_t)nb_zero * blockDim.x)
+        pp.zero[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 struct PostParams {
@@ -627,35 +660,36 @@ struct PostParams {
     float* dbias;
 };
 
-// dq (bf16, caller strides) from the fp32 accumulator: one thread per row.
-__global__ void __launch_bounds__(256) dq_convert_kernel(const PostParams p) {
+// The backward's finishing pass in one launch: dq (bf16, caller strides) from
+// the fp32 accumulator, four threads per row converting 8 channels each; then
+// (several row groups only) d_pair_bias = sum over groups g = 0, 1, ... of the
+// partial slabs, in that order, 4 elements per thread.
+__global__ void __launch_bounds__(256) bwd_post_kernel(const PostParams p) {
     const int64_t rows = (int64_t)p.B * p.S * p.N * p.H;
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < rows; t += (int64_t)gridDim.x * blockDim.x) {
-        const int h = (int)(t % p.H);
-        const int i = (int)((t / p.H) % p.N);
-        const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
-        const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
-        const float4* a = reinterpret_cast<const float4*>(p.dq_acc + t * HD);
-        uint4* o = reinterpret_cast<uint4*>(p.dq + p.gs.off(b, s, i, h));
-#pragma unroll
-        for (int q = 0; q < HD / 8; ++q) {
-            const float4 x = a[2 * q], y = a[2 * q + 1];
-            o[q] = make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
-        }
-    }
-}
-
-// d_pair_bias = sum over groups g = 0, 1, ... of the partials, in that order.
-__global__ void __launch_bounds__(256) dbias_reduce_kernel(const PostParams p) {
-    const int64_t n4 = (int64_t)p.B * p.H * p.N * p.N / 4;
+    const int64_t nq = rows * PRE_LANES;
+    const int64_t n4 = p.groups > 1 ? (int64_t)p.B * p.H * p.N * p.N / 4 : 0;
     const int64_t stride = (int64_t)p.B * p.H * p.N * p.N;
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n4; t += (int64_t)gridDim.x * blockDim.x) {
-        float4 acc = reinterpret_cast<const float4*>(p.part)[t];
-        for (int g = 1; g < p.groups; ++g) {
-            const float4 v = reinterpret_cast<const float4*>(p.part + g * stride)[t];
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < nq + n4; g += (int64_t)gridDim.x * blockDim.x) {
+        if (g < nq) {
+            const int64_t t = g / PRE_LANES;
+            const int part = (int)(g % PRE_LANES);
+            const int h = (int)(t % p.H);
+            const int i = (int)((t / p.H) % p.N);
+            const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
+            const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
+            const float4* a = reinterpret_cast<const float4*>(p.dq_acc + t * HD) + 2 * part;
+            const float4 x = a[0], y = a[1];
+            reinterpret_cast<uint4*>(p.dq + p.gs.off(b, s, i, h))[part] =
+                make_uint4(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w), pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
+        } else {
+            const int64_t t = g - nq;
+            float4 acc = reinterpret_cast<const float4*>(p.part)[t];
+            for (int k = 1; k < p.groups; ++k) {
+                const float4 v = reinterpret_cast<const float4*>(p.part + k * stride)[t];
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            reinterpret_cast<float4*>(p.dbias)[t] = acc;
         }
-        reinterpret_cast<float4*>(p.dbias)[t] = acc;
     }
 }
 
@@ -733,17 +767,20 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     pp.g = static_cast<const __nv_bfloat16*>(c.g); pp.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
     pp.lse = c.lse; pp.dg = static_cast<__nv_bfloat16*>(c.dg); pp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
     pp.doa_hi = doa; pp.doa_lo = dol; pp.nl = nl; pp.nd = nd; pp.dq_acc = dq_acc;
-    bwd_pre_kernel<<<grid_for((rows + (int64_t)B * S * H * (n_pad - N)) * PRE_LANES, 256), 256, 0, stream>>>(pp);
+    // one launch: per-row pass, pair-bias transpose, and clearing of the partial
+    // slabs (or of the output itself), which accumulate by atomic adds from zero
+    PrepParams prep{};
+    prep.pre = pp;
+    prep.nb_pre = grid_for((rows + (int64_t)B * S * H * (n_pad - N)) * PRE_LANES, 256);
+    prep.bias = static_cast<const __nv_bfloat16*>(c.bias);
+    prep.biast = biasT;
+    const int nt = (N + 31) / 32;
+    prep.nb_tr = c.bias ? nt * nt * B * H : 0;
+    prep.zero = reinterpret_cast<float4*>(part);
+    prep.n_zero4 = (int64_t)c.groups * B * H * N * N / 4;   // N % 8 == 0: whole float4s
+    const int nb_zero = grid_for(prep.n_zero4, 256);
+    bwd_prep_kernel<<<prep.nb_pre + prep.nb_tr + nb_zero, 256, 0, stream>>>(prep);
     ++*launched;
-    if (c.bias) {
-        transpose_bias_kernel<<<dim3((N + 31) / 32, (N + 31) / 32, B * H), dim3(32, 8), 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(c.bias), biasT, N);
-        ++*launched;
-    }
-
-    // the partial slabs (or the output itself) accumulate by atomic adds from zero
-    const size_t part_bytes = (size_t)c.groups * B * H * N * N * sizeof(float);
-    if (cudaMemsetAsync(part, 0, part_bytes, stream) != cudaSuccess) return EVO_ERR_CUDA;
 
     // tensor maps: q, k, v, dOa high, dOa low, transposed bias, mask, nl rows, -D rows
     const evo_strides_t contig{(int64_t)S * N * H * HD, (int64_t)N * H * HD, (int64_t)H * HD, (int64_t)HD};
@@ -787,12 +824,8 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     qp.B = B; qp.S = S; qp.N = N; qp.H = H;
     qp.dq_acc = dq_acc; qp.dq = static_cast<__nv_bfloat16*>(c.dq); qp.gs = mp.gs;
     qp.part = part; qp.groups = G; qp.dbias = c.dbias;
-    dq_convert_kernel<<<grid_for(rows, 256), 256, 0, stream>>>(qp);
+    bwd_post_kernel<<<grid_for(rows * PRE_LANES + (G > 1 ? (int64_t)B * H * N * N / 4 : 0), 256), 256, 0, stream>>>(qp);
     ++*launched;
-    if (G > 1) {
-        dbias_reduce_kernel<<<grid_for((int64_t)B * H * N * N / 4, 256), 256, 0, stream>>>(qp);
-        ++*launched;
-    }
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
