@@ -184,8 +184,10 @@ def flops(w):
 # profiles/ summary, together with the SHA-256 of the kernel's source file at
 # that time.  Reported only while the source is unchanged.
 TRAFFIC = {
-    ("bwd_main", "msa_row_256"): (176.93e6, "bwd_sm100.cuh",
-                                "2cf8499a7d0684cb246472a6f7f7abfd5361aa1a10807f21ddd21e9678c2e052"),
+    ("bwd_main", "msa_row_256"): (178.88e6, "bwd_sm100.cuh",
+                                "b8b80b5dac49ab2b8777761e2246889ec13f7608b74d22a3292eddd15711f7f3"),
+    ("fwd_main", "msa_row_256"): (75.56e6, "fwd_sm100.cuh",
+                                "ccbab72209fc7ef6501f95e939be78536073bbefc7e9c99387ac6f81f106e9be"),
 }
 
 
