@@ -45,7 +45,12 @@ MUTANTS = {
     5: "pair bias read transposed (b_ji instead of b_ij)",
     6: "sign of D = sum_j P dP flipped in backward",
     7: "dk missing its 1/sqrt(C) factor",
+    8: "LayerNorm divides by the variance instead of its square root",
+    9: "projection output columns shifted by one",
 }
+#: Which function each planted mistake breaks.
+ATTENTION_MUTANTS = (1, 2, 3, 4, 5, 6, 7)
+LN_LINEAR_MUTANTS = (8, 9)
 
 
 class _Dims(ctypes.Structure):
@@ -80,6 +85,8 @@ def _lib(mutant: int = 0) -> ctypes.CDLL:
         lib.evo_ref_backward.argtypes = [ctypes.POINTER(_Dims)] + [p] * 12
         lib.evo_ref_backward.restype = ctypes.c_int
         lib.evo_ref_mutant.restype = ctypes.c_int
+        lib.evo_ref_ln_linear.argtypes = [ctypes.c_int64] * 3 + [p] * 3 + [ctypes.c_double] + [p] * 3
+        lib.evo_ref_ln_linear.restype = ctypes.c_int
         _LIBS[mutant] = lib
     return _LIBS[mutant]
 
@@ -158,6 +165,31 @@ def backward(q, k, v, g, mask_bias, pair_bias, dout, *, mutant: int = 0,
     if rc != 0:
         raise ValueError("evo_ref_backward rejected its arguments")
     return res
+
+
+def ln_linear(x, ln_w, ln_b, eps, w, bias=None, *, mutant: int = 0):
+    """LayerNorm over the last axis of x, then y = LN(x) @ w + bias, in fp64.
+
+    x: [..., c_in]; ln_w, ln_b: [c_in] (None = ones / zeros); w: [c_in, n_out];
+    bias: [n_out] or None.  Returns y with shape x.shape[:-1] + (n_out,).
+    This is the fused pre-attention projection (MegaFold summary, section
+    "EvoFusion"): q, k, v, g are column blocks of y, and the pair bias is y
+    of the pair representation with n_out = H, read as [b, h, i, j].
+    """
+    x = _f64(x)
+    lead, c_in = x.shape[:-1], x.shape[-1]
+    w = _f64(w)
+    if w.shape[0] != c_in:
+        raise ValueError(f"w {w.shape} does not match c_in {c_in}")
+    n_out = w.shape[1]
+    x2 = x.reshape(-1, c_in)
+    y = np.empty((x2.shape[0], n_out), np.float64)
+    lw, lb, bb = _f64(ln_w), _f64(ln_b), _f64(bias)
+    rc = _lib(mutant).evo_ref_ln_linear(x2.shape[0], c_in, n_out, _ptr(x2), _ptr(lw), _ptr(lb), float(eps),
+                                        _ptr(w), _ptr(bb), _ptr(y))
+    if rc != 0:
+        raise ValueError("evo_ref_ln_linear rejected its arguments")
+    return y.reshape(lead + (n_out,))
 
 
 def mutant_id(mutant: int) -> int:

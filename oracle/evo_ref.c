@@ -40,6 +40,9 @@
  * Nq may differ from Nk so that a caller can evaluate the definition at a
  * subset of query rows (a smaller, equally valid problem).
  *
+ * The file also holds the fused pre-attention projection (LayerNorm + linear,
+ * evo_ref_ln_linear below) that produces q, k, v, g and the pair bias.
+ *
  * Planted mistakes (mutation testing of the pins): building with
  * -DEVO_REF_MUTANT=n swaps in one deliberate error, see mutant_* below.
  */
@@ -263,6 +266,61 @@ int evo_ref_backward(const evo_ref_dims* d, const double* q, const double* k, co
             }
             free(p); free(ds); free(A); free(dA);
         }
+    }
+    return 0;
+}
+
+/*
+ * Fused pre-attention projection: the LayerNorm of every row of a
+ * representation (MSA or pair) followed by its linear projections, the pair
+ * of operators that EvoFusion computes without writing the normalised tensor
+ * to memory (MegaFold summary, section "EvoFusion : Pile d'Operateurs
+ * Fusionnes").  For each row r of x [rows, c_in]:
+ *
+ *   mu      = (1/c_in) sum_k x[r,k]
+ *   var     = (1/c_in) sum_k (x[r,k] - mu)^2            (biased, as LayerNorm)
+ *   n[k]    = (x[r,k] - mu) / sqrt(var + eps) * ln_w[k] + ln_b[k]
+ *   y[r,o]  = sum_k n[k] * w[k,o] + bias[o]               (w: [c_in, n_out])
+ *
+ * ln_w NULL means ones, ln_b and bias NULL mean zeros.  Returns 0, or -1 for
+ * a bad size.
+ */
+int evo_ref_ln_linear(int64_t rows, int64_t c_in, int64_t n_out, const double* x, const double* ln_w,
+                      const double* ln_b, double eps, const double* w, const double* bias, double* y) {
+    if (rows < 0 || c_in <= 0 || n_out <= 0) return -1;
+#pragma omp parallel
+    {
+        double* n = (double*)malloc(sizeof(double) * (size_t)c_in);
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < rows; ++r) {
+            const double* xr = x + r * c_in;
+            double mu = 0.0;
+            for (int64_t k = 0; k < c_in; ++k) mu += xr[k];
+            mu /= (double)c_in;
+            double var = 0.0;
+            for (int64_t k = 0; k < c_in; ++k) var += (xr[k] - mu) * (xr[k] - mu);
+            var /= (double)c_in;
+#if EVO_REF_MUTANT == 8
+            const double inv = 1.0 / var;          /* mutant: missing square root */
+#else
+            const double inv = 1.0 / sqrt(var + eps);
+#endif
+            for (int64_t k = 0; k < c_in; ++k)
+                n[k] = (xr[k] - mu) * inv * (ln_w ? ln_w[k] : 1.0) + (ln_b ? ln_b[k] : 0.0);
+            double* yr = y + r * n_out;
+            for (int64_t o = 0; o < n_out; ++o) yr[o] = bias ? bias[o] : 0.0;
+            for (int64_t k = 0; k < c_in; ++k) {
+                const double nk = n[k];
+                const double* wk = w + k * n_out;
+#if EVO_REF_MUTANT == 9
+                /* mutant: output columns shifted by one */
+                for (int64_t o = 0; o < n_out; ++o) yr[o] += nk * wk[(o + 1) % n_out];
+#else
+                for (int64_t o = 0; o < n_out; ++o) yr[o] += nk * wk[o];
+#endif
+            }
+        }
+        free(n);
     }
     return 0;
 }
