@@ -17,6 +17,13 @@ ranks.
 
 ``--impl reference`` times the fp64 CPU oracle (the correctness reference)
 on a bounded sample of the same workload, on this host's cores.
+
+``--workload msa_proj_256 | pair_proj_256`` benchmarks the fused pre-attention
+projection instead (MegaFold summary, section "EvoFusion"): one step is
+y = LayerNorm(x) @ [w_q | w_k | w_v | w_g] + bias over every row of the MSA
+(or pair) representation, and for the pair representation also the
+pair-bias projection LayerNorm(z) @ w_b + b_b.  Metric: TFLOP/s of the
+projection GEMMs (2 * rows * c_in * n_out), with the same timing rules.
 """
 from __future__ import annotations
 
@@ -35,9 +42,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from evoformer_pair_bias_b200 import attention as A  # noqa: E402
-from evoformer_pair_bias_b200.workloads import WORKLOADS, DEFAULT_BENCH, logical_view, make_inputs  # noqa: E402
+from evoformer_pair_bias_b200.workloads import (WORKLOADS, DEFAULT_BENCH, PROJ_WORKLOADS, logical_view,  # noqa: E402
+                                                make_inputs, make_pair_bias_params, make_proj_inputs)
 
 METRIC = "Evoformer pair-bias attention fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
+PROJ_METRIC = "fused LayerNorm + linear pre-attention projection TFLOP/s"
+PROJ_EPS = 1e-5
 NOMINAL_BF16_TFLOPS = 2250.0
 
 
@@ -333,12 +343,236 @@ def run_reference(args, w, rank, world):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# Fused pre-attention projection (LayerNorm + linear)
+
+
+def proj_parts(pw):
+    """The projections one step runs: the q, k, v, g projection, plus the pair bias for the pair representation."""
+    return ("qkvg", "pair_bias") if pw.name.startswith("pair") else ("qkvg",)
+
+
+def proj_algorithmic(pw, part: str):
+    """(FLOPs, bytes) of one launch: x read once, w and the LayerNorm/bias vectors read once, y written once."""
+    n_out = pw.n_out if part == "qkvg" else pw.H
+    fl = 2 * pw.rows * pw.c_in * n_out
+    by = pw.rows * pw.c_in * 2 + pw.c_in * n_out * 2 + (2 * pw.c_in + n_out) * 4 + pw.rows * n_out * 2
+    return fl, by
+
+
+def proj_roofline(pw, part, us, pk, timed_s):
+    fl, by = proj_algorithmic(pw, part)
+    sec = us * 1e-6
+    sustained = timed_s > 1.0
+    tflops_peak = pk["bf16_sustained"] if sustained else pk["bf16"]
+    t_tensor, t_hbm = fl / (tflops_peak * 1e12), by / (pk["hbm"] * 1e9)
+    tr = TRAFFIC.get((part, pw.name))
+    traffic = tr[0] if tr is not None and _source_sha(tr[1]) == tr[2] else None
+    kernel = {"qkvg": "proj::ln_linear_kernel", "pair_bias": "proj::pair_bias_kernel"}[part]
+    common = {"kernel": kernel, "us_per_launch": us, "flops_per_launch": fl, "algorithmic_bytes_per_launch": by,
+              "traffic": traffic, "tensor_floor_us": t_tensor * 1e6, "hbm_floor_us": t_hbm * 1e6}
+    if t_tensor >= t_hbm:
+        a = fl / sec / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": tflops_peak, "unit": "TFLOP/s", "frac": a / tflops_peak,
+                "peak_source": f"{pk['source']} bf16 {'sustained' if sustained else 'burst'}", **common}
+    a = by / sec / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": pk["hbm"], "unit": "GB/s", "frac": a / pk["hbm"],
+            "peak_source": f"{pk['source']} HBM copy", "tensor_frac": fl / sec / 1e12 / tflops_peak, **common}
+
+
+def proj_oracle_sample(pw, target_s: float = 12.0):
+    """Time the fp64 oracle projection on the first r rows of the workload, sized for about target_s."""
+    import oracle
+    oracle.build()
+    d = make_proj_inputs(pw)
+    pb = make_pair_bias_params(pw) if "pair_bias" in proj_parts(pw) else None
+    x_all = d["x"].reshape(-1, pw.c_in)
+    f = {k: d[k].double().numpy() for k in ("w", "ln_w", "ln_b", "bias")}
+    fb = None if pb is None else {k: v.double().numpy() for k, v in pb.items()}
+
+    def run(r):
+        x = x_all[:r].double().numpy()
+        t0 = time.perf_counter()
+        oracle.ln_linear(x, f["ln_w"], f["ln_b"], PROJ_EPS, f["w"], f["bias"])
+        if fb is not None:
+            oracle.ln_linear(x, fb["ln_w"], fb["ln_b"], PROJ_EPS, fb["w"], fb["bias"])
+        return time.perf_counter() - t0
+
+    t1 = run(64) / 64
+    r = max(64, min(pw.rows, int(target_s / max(t1, 1e-9))))
+    t, reps = 0.0, 0
+    while reps == 0 or t < 0.7 * target_s:
+        t += run(r)
+        reps += 1
+    fl = sum(proj_algorithmic(pw, p)[0] for p in proj_parts(pw)) * r / pw.rows * reps
+    return dict(value=fl / t / 1e12, unit="TFLOP/s", cores=oracle_threads(), kind="oracle",
+                sample=f"{r} of {pw.rows} rows x{reps}, {'+'.join(proj_parts(pw))}, fp64, {t:.2f} s",
+                seconds=t, rows=r)
+
+
+def run_projection(args, pw, rank, world, local):
+    parts = proj_parts(pw)
+    fl_step = sum(proj_algorithmic(pw, p)[0] for p in parts)
+    base_cfg = {"workload": pw.name, "B": pw.B, "rows_per_batch": pw.S, "N_res": pw.N, "c_in": pw.c_in,
+                "H": pw.H, "c": pw.C, "n_out": pw.n_out, "projections": list(parts), "eps": PROJ_EPS}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps, warm = args.steps, args.warmup
+        info = proj_oracle_sample(pw, target_s=max(0.5, 60.0 / max(1, steps + warm)))
+        r = info["rows"]
+        import oracle
+        d = make_proj_inputs(pw)
+        x = d["x"].reshape(-1, pw.c_in)[:r].double().numpy()
+        f = {k: d[k].double().numpy() for k in ("w", "ln_w", "ln_b", "bias")}
+        fb = ({k: v.double().numpy() for k, v in make_pair_bias_params(pw).items()}
+              if "pair_bias" in parts else None)
+        times = []
+        for i in range(warm + steps):
+            t0 = time.perf_counter()
+            oracle.ln_linear(x, f["ln_w"], f["ln_b"], PROJ_EPS, f["w"], f["bias"])
+            if fb is not None:
+                oracle.ln_linear(x, fb["ln_w"], fb["ln_b"], PROJ_EPS, fb["w"], fb["bias"])
+            if i >= warm:
+                times.append(time.perf_counter() - t0)
+        t = sum(times)
+        val = fl_step * r / pw.rows * steps / t / 1e12
+        line = {"metric": PROJ_METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps,
+                "warmup": warm, "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {**base_cfg, "sample_rows": r, "l2": "n/a (CPU)"},
+                "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": f"{r} of {pw.rows} rows per step, fp64"},
+                "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import datetime
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    A.load_library()
+    hin = make_proj_inputs(pw)
+    d = {k: v.to(dev) for k, v in hin.items()}
+    pbp = {k: v.to(dev) for k, v in make_pair_bias_params(pw).items()} if "pair_bias" in parts else None
+    y = torch.empty(pw.B, pw.S, pw.N, pw.n_out, dtype=torch.bfloat16, device=dev)
+    pb = torch.empty(pw.B, 1, pw.H, pw.N, pw.N, dtype=torch.bfloat16, device=dev) if pbp else None
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(x):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+        ev[0].record()
+        A.ln_linear(x, d["ln_w"], d["ln_b"], PROJ_EPS, d["w"], d["bias"], y=y)
+        ev[1].record()
+        if pbp is not None:
+            A.ln_pair_bias(x, pbp["ln_w"], pbp["ln_b"], PROJ_EPS, pbp["w"], pbp["bias"], out=pb)
+            ev[2].record()
+        return ev
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(d["x"])
+    torch.cuda.synchronize()
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported an error during warm-up")
+    K = args.steps
+    evs = []
+    with ClockSampler(gpu_uuid(dev)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        n0 = A.launch_count()
+        for _ in range(K):
+            flush.zero_()
+            evs.append(step(d["x"]))
+        torch.cuda.synchronize()
+        barrier()
+        launches = A.launch_count() - n0
+    per_part = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(len(parts))]
+    tot = sum(per_part)
+    tot, *per_part = max_over_ranks([tot] + per_part, world, dev)
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported an error during the timed region")
+    value = job_throughput(fl_step, K, world, tot)
+    pk = peaks()
+
+    e2e = None
+    if not args.no_e2e:
+        hx = hin["x"].pin_memory()
+        hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        hpb = torch.empty(pb.shape, dtype=pb.dtype).pin_memory() if pb is not None else None
+        dx = torch.empty_like(hx, device=dev)
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            step(dx)
+            hy.copy_(y, non_blocking=True)
+            if hpb is not None:
+                hpb.copy_(pb, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        et = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+        e2e = {"value": job_throughput(fl_step, K, world, et), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": hx.numel() * hx.element_size(),
+               "d2h_bytes_per_step": hy.numel() * hy.element_size() + (0 if hpb is None else
+                                                                       hpb.numel() * hpb.element_size()),
+               "ms_per_step": et / K}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            cpu = proj_oracle_sample(pw)
+            cpu.pop("seconds", None)
+            cpu.pop("rows", None)
+        except Exception as exc:  # the baseline is reported, never required
+            cpu = {"error": repr(exc)}
+
+    if rank == 0:
+        us = {p: 1e3 * per_part[j] / K for j, p in enumerate(parts)}
+        top = max(parts, key=lambda p: us[p])
+        line = {
+            "metric": PROJ_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": tot / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**base_cfg, "l2": "flushed (256 MB write) before every step",
+                       "parallelism": f"replicas x{world}, rows independent, no collective"},
+            "roofline": proj_roofline(pw, top, us[top], pk, timed_s=tot * 1e-3),
+            "kernels": {p: {"launches": K, "us_per_launch": us[p],
+                            "roofline": proj_roofline(pw, p, us[p], pk, timed_s=tot * 1e-3)} for p in parts},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS) + sorted(PROJ_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -348,6 +582,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in PROJ_WORKLOADS:
+        return run_projection(args, PROJ_WORKLOADS[args.workload], rank, world, local)
     w = WORKLOADS[args.workload]
 
     if args.impl == "reference":

@@ -33,7 +33,7 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 #: Every symbol include/evo_attn.h declares.
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
            "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc",
-           "evo_attn_timing_enable", "evo_attn_timing_collect")
+           "evo_attn_timing_enable", "evo_attn_timing_collect", "evo_ln_linear", "evo_ln_pair_bias")
 
 #: Size of the library's fixed scratch area used by evo_attn_bwd_noalloc (bytes).
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -54,7 +54,7 @@ class Strides(ctypes.Structure):
 
 
 #: Timing phases (evo_timing_t indices).
-PHASES = ("fwd_main", "bwd_main", "bwd_all")
+PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj")
 
 
 class Timing(ctypes.Structure):
@@ -93,6 +93,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_attn_timing_enable.restype = ctypes.c_int
     lib.evo_attn_timing_collect.argtypes = [ctypes.POINTER(Timing)]
     lib.evo_attn_timing_collect.restype = ctypes.c_int
+    i64, f32 = ctypes.c_int64, ctypes.c_float
+    lib.evo_ln_linear.argtypes = [i64, i64, i64, vp, vp, vp, f32, vp, vp, vp, i64, vp]
+    lib.evo_ln_linear.restype = ctypes.c_int
+    lib.evo_ln_pair_bias.argtypes = [i64, i64, i64, i64, vp, vp, vp, f32, vp, vp, vp, vp]
+    lib.evo_ln_pair_bias.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -224,6 +229,69 @@ def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads
 def launch_count() -> int:
     """Kernels the library has enqueued in this process so far."""
     return int(load_library().evo_attn_launch_count())
+
+
+def _opt_f32(t, n, device):
+    if t is None:
+        return None
+    t = t.to(device=device, dtype=torch.float32).contiguous()
+    if t.numel() != n:
+        raise ValueError(f"expected {n} values, got {t.numel()}")
+    return t
+
+
+def ln_linear(x, ln_w, ln_b, eps, w, bias=None, y=None):
+    """Fused LayerNorm + linear: y = LayerNorm(x) @ w + bias (bf16 in and out).
+
+    x: bf16 [..., c_in] (rows contiguous); ln_w, ln_b, bias: any float tensors
+    (None = ones / zeros / zeros); w: bf16 [c_in, n_out].  Returns y with shape
+    x.shape[:-1] + (n_out,).  With w = [w_q | w_k | w_v | w_g], qkvg_views(y, H)
+    gives q, k, v, g as attention inputs without a copy.
+    """
+    lib = load_library()
+    c_in = x.shape[-1]
+    xc = x.contiguous().view(-1, c_in)
+    n_out = w.shape[1]
+    if w.shape[0] != c_in:
+        raise ValueError(f"w {tuple(w.shape)} does not match c_in {c_in}")
+    wc = w.contiguous()
+    if y is None:
+        y = torch.empty(x.shape[:-1] + (n_out,), dtype=torch.bfloat16, device=x.device)
+    lw, lb, bb = (_opt_f32(t, n, x.device) for t, n in ((ln_w, c_in), (ln_b, c_in), (bias, n_out)))
+    rc = lib.evo_ln_linear(xc.shape[0], c_in, n_out, _ptr(xc), _ptr(lw), _ptr(lb), float(eps), _ptr(wc),
+                           _ptr(bb), _ptr(y), n_out, _stream(x.device))
+    _check("evo_ln_linear", rc)
+    return y
+
+
+def qkvg_views(y, H: int):
+    """q, k, v, g as [B, S, N, H, C] views of a ln_linear output [B, S, N, 4*H*C]."""
+    B, S, N, F = y.shape
+    C = F // (4 * H)
+    if 4 * H * C != F:
+        raise ValueError(f"last axis {F} is not 4 * H * C")
+    y5 = y.view(B, S, N, 4, H, C)
+    return tuple(y5[:, :, :, m] for m in range(4))
+
+
+def ln_pair_bias(z, ln_w, ln_b, eps, w, bias=None, out=None):
+    """Pair-bias projection: pair_bias[b, 0, h, i, j] = LayerNorm(z[b, i, j]) @ w[:, h] + bias[h].
+
+    z: bf16 [B, N, N, c_z]; w: bf16 [c_z, H].  Returns bf16 [B, 1, H, N, N].
+    """
+    lib = load_library()
+    B, N, N2, c_z = z.shape
+    if N2 != N or w.shape[0] != c_z:
+        raise ValueError("z must be [B, N, N, c_z] and w [c_z, H]")
+    H = w.shape[1]
+    zc, wc = z.contiguous(), w.contiguous()
+    if out is None:
+        out = torch.empty((B, 1, H, N, N), dtype=torch.bfloat16, device=z.device)
+    lw, lb, bb = (_opt_f32(t, n, z.device) for t, n in ((ln_w, c_z), (ln_b, c_z), (bias, H)))
+    rc = lib.evo_ln_pair_bias(B, N, c_z, H, _ptr(zc), _ptr(lw), _ptr(lb), float(eps), _ptr(wc), _ptr(bb),
+                              _ptr(out), _stream(z.device))
+    _check("evo_ln_pair_bias", rc)
+    return out
 
 
 def timing_enable(on: bool = True) -> None:

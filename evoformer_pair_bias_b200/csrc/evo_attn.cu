@@ -24,6 +24,7 @@
 #include "timing.cuh"
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
+#include "proj_sm100.cuh"
 
 #define EVO_VERSION 10000
 
@@ -215,6 +216,22 @@ evo_status_t bwd_f32(const evo_shape_t& sh, evo::simt::Args a, cudaStream_t stre
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- fused pre-attention projection
+template <int BNO>
+evo_status_t launch_ln_linear(const CUtensorMap* maps, const evo::proj::LnParams& p, cudaStream_t stream) {
+    using L = evo::proj::PLayout<BNO>;
+    auto kern = evo::proj::ln_linear_kernel<BNO>;
+    static cudaError_t attr = set_smem(kern, L::bytes);
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    const dim3 grid((unsigned)((p.rows + evo::proj::BM - 1) / evo::proj::BM), (unsigned)(p.n_out / BNO));
+    {
+        evo::timing::Scope t(EVO_PHASE_PROJ, stream);
+        kern<<<grid, evo::proj::THREADS, L::bytes, stream>>>(maps[0], maps[1], p);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -360,6 +377,60 @@ static evo_status_t noalloc_workspace(void** addr) {
     }
     *addr = g_noalloc_addr[dev];
     return EVO_OK;
+}
+
+evo_status_t evo_ln_linear(int64_t rows, int64_t c_in, int64_t n_out, const void* x, const float* ln_w,
+                           const float* ln_b, float eps, const void* w, const float* bias, void* y, int64_t ldy,
+                           void* stream) {
+    if (rows < 0 || c_in <= 0 || n_out <= 0 || ldy < n_out || !(eps >= 0.f)) return EVO_ERR_INVALID_ARG;
+    if (rows == 0) return EVO_OK;
+    if (!x || !w || !y) return EVO_ERR_INVALID_ARG;
+    if (c_in % evo::proj::KBOX != 0 || c_in > evo::proj::MAX_CIN || n_out % 128 != 0 || ldy % 8 != 0)
+        return EVO_ERR_UNSUPPORTED;
+    for (const void* q : {x, w, (const void*)y})
+        if (!aligned(q, 16)) return EVO_ERR_UNSUPPORTED;
+    for (const void* q : {(const void*)ln_w, (const void*)ln_b, (const void*)bias})
+        if (q && !aligned(q, 4)) return EVO_ERR_INVALID_ARG;
+    CUtensorMap maps[2];
+    std::memset(maps, 0, sizeof(maps));
+    const bool wide = n_out % 256 == 0;
+    if (!evo::tma::matrix_bf16(&maps[0], x, rows, c_in, c_in, evo::proj::BM) ||
+        !evo::tma::matrix_bf16(&maps[1], w, c_in, n_out, n_out, (uint32_t)c_in))
+        return EVO_ERR_CUDA;
+    evo::proj::LnParams p{};
+    p.rows = (int)rows; p.c_in = (int)c_in; p.n_out = (int)n_out; p.eps = eps;
+    p.ln_w = ln_w; p.ln_b = ln_b; p.bias = bias;
+    p.y = static_cast<__nv_bfloat16*>(y); p.ldy = ldy;
+    if (rows > (int64_t)0x7fffffff) return EVO_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return wide ? launch_ln_linear<256>(maps, p, s) : launch_ln_linear<128>(maps, p, s);
+}
+
+evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, const void* z, const float* ln_w,
+                              const float* ln_b, float eps, const void* w, const float* bias, void* pair_bias,
+                              void* stream) {
+    if (B < 0 || N < 0 || c_z <= 0 || H <= 0 || !(eps >= 0.f)) return EVO_ERR_INVALID_ARG;
+    if (B == 0 || N == 0) return EVO_OK;
+    if (!z || !w || !pair_bias) return EVO_ERR_INVALID_ARG;
+    if (c_z % 8 != 0 || c_z > 1024 || H > evo::proj::PB_MAX_H) return EVO_ERR_UNSUPPORTED;
+    if (!aligned(z, 16) || !aligned(w, 2) || !aligned(pair_bias, 2)) return EVO_ERR_UNSUPPORTED;
+    evo::proj::PbParams p{};
+    p.B = (int)B; p.N = (int)N; p.c_z = (int)c_z; p.H = (int)H; p.eps = eps;
+    p.z = static_cast<const __nv_bfloat16*>(z); p.ln_w = ln_w; p.ln_b = ln_b;
+    p.w = static_cast<const __nv_bfloat16*>(w); p.bias = bias;
+    p.out = static_cast<__nv_bfloat16*>(pair_bias);
+    const int64_t total = B * N * N;
+    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
+    const size_t shm = (size_t)c_z * H * sizeof(float);   // <= 64 KB
+    static cudaError_t attr = set_smem(evo::proj::pair_bias_kernel, (int)(1024 * evo::proj::PB_MAX_H * sizeof(float)));
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        evo::timing::Scope t(EVO_PHASE_PROJ, s);
+        evo::proj::pair_bias_kernel<<<grid, 256, shm, s>>>(p);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
 evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,

@@ -106,5 +106,14 @@ inline bool rowterm_bf16(CUtensorMap* m, const void* ptr, const evo_shape_t& sh,
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 5, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// bf16 row-major matrix [rows, cols] with row pitch ld (elements), viewed as
+// (col, row); box (64 cols, box_rows) with 128B swizzle.
+inline bool matrix_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, uint32_t box_rows) {
+    const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+    const uint64_t str[1] = {(uint64_t)ld * 2};
+    const uint32_t box[2] = {64, box_rows};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 }  // namespace tma
 }  // namespace evo

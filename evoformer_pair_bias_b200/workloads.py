@@ -187,4 +187,75 @@ def ceil_div(a: int, b: int) -> int:
 
 __all__ = ["Workload", "WORKLOADS", "DEFAULT_BENCH", "MASK_VALUE", "make_inputs",
            "logical_view", "storage_empty", "sample_rows", "logits_bytes", "pair_rep_bytes",
-           "mask_columns", "ceil_div"]
+           "mask_columns", "ceil_div", "ProjWorkload", "PROJ_WORKLOADS", "make_proj_inputs",
+           "make_pair_bias_params"]
+
+
+# ---------------------------------------------------------------------------
+# Fused pre-attention projection (LayerNorm + linear): seeded inputs only.
+#
+# Recipe (generator seeded with ``seed``): draw x (rows x c_in) ~ N(0, 1),
+# then w ~ N(0, 1/c_in), ln_w = 1 + 0.1 N(0, 1), ln_b = 0.1 N(0, 1) and
+# bias ~ N(0, 1), in that order, in fp32; x and w are rounded to bf16 (the
+# LayerNorm parameters and the bias stay fp32).  Shapes: the MSA
+# representation (c_m = 256) projected to q, k, v, g of MSA-row attention
+# (4 x 8 heads x 32), and the pair representation (c_z = 128) projected to
+# q, k, v, g of triangle attention (4 x 4 heads x 32) and to its pair bias
+# (one output per head).
+
+
+@dataclasses.dataclass(frozen=True)
+class ProjWorkload:
+    name: str
+    B: int
+    S: int          # rows of the representation per batch (MSA sequences, or N for the pair)
+    N: int
+    c_in: int
+    H: int          # attention heads
+    C: int          # head dim
+    seed: int
+
+    @property
+    def rows(self) -> int:
+        return self.B * self.S * self.N
+
+    @property
+    def n_out(self) -> int:
+        return 4 * self.H * self.C
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.rows * self.c_in * self.n_out
+
+
+PROJ_WORKLOADS = {
+    "msa_proj_256": ProjWorkload("msa_proj_256", 1, 128, 256, 256, 8, 32, 20271),
+    "pair_proj_256": ProjWorkload("pair_proj_256", 1, 256, 256, 128, 4, 32, 20272),
+    "tiny_proj": ProjWorkload("tiny_proj", 1, 3, 50, 64, 1, 32, 20273),
+}
+
+
+def make_proj_inputs(w: ProjWorkload, n_out: int | None = None, device="cpu") -> dict:
+    """x [B, S, N, c_in] bf16, w [c_in, n_out] bf16, ln_w / ln_b [c_in] and bias [n_out] fp32."""
+    n_out = w.n_out if n_out is None else n_out
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    x = torch.randn((w.B, w.S, w.N, w.c_in), generator=g)
+    wt = torch.randn((w.c_in, n_out), generator=g) / (w.c_in ** 0.5)
+    ln_w = 1 + 0.1 * torch.randn(w.c_in, generator=g)
+    ln_b = 0.1 * torch.randn(w.c_in, generator=g)
+    bias = torch.randn(n_out, generator=g)
+    return {"x": x.to(torch.bfloat16).to(device), "w": wt.to(torch.bfloat16).to(device),
+            "ln_w": ln_w.to(device), "ln_b": ln_b.to(device), "bias": bias.to(device)}
+
+
+def make_pair_bias_params(w: ProjWorkload, device="cpu") -> dict:
+    """Parameters of the pair-bias projection of a pair representation [B, N, N, c_in]:
+    w [c_in, H] ~ N(0, 1/c_in) in bf16, ln_w = 1 + 0.1 N(0, 1), ln_b = 0.1 N(0, 1) and
+    bias ~ N(0, 1) in fp32, drawn in that order from a generator seeded with seed + 1."""
+    g = torch.Generator("cpu").manual_seed(w.seed + 1)
+    wt = torch.randn((w.c_in, w.H), generator=g) / (w.c_in ** 0.5)
+    ln_w = 1 + 0.1 * torch.randn(w.c_in, generator=g)
+    ln_b = 0.1 * torch.randn(w.c_in, generator=g)
+    bias = torch.randn(w.H, generator=g)
+    return {"w": wt.to(torch.bfloat16).to(device), "ln_w": ln_w.to(device), "ln_b": ln_b.to(device),
+            "bias": bias.to(device)}

@@ -177,6 +177,43 @@ evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype,
                                   void* dq, void* dk, void* dv, void* dg, const evo_strides_t* grad_str,
                                   float* d_pair_bias, void* stream);
 
+/*
+ * Fused pre-attention projection: y = LayerNorm(x) @ w + bias, for every row
+ * of a representation, without writing the normalised rows to memory -- the
+ * LayerNorm + linear pair that EvoFusion fuses (MegaFold summary, section
+ * "EvoFusion : Pile d'Operateurs Fusionnes").
+ *
+ *   mean_r = (1/c_in) sum_k x[r,k],  var_r = (1/c_in) sum_k (x[r,k] - mean_r)^2
+ *   y[r,o] = sum_k ((x[r,k] - mean_r) / sqrt(var_r + eps) * ln_w[k] + ln_b[k]) * w[k,o] + bias[o]
+ *
+ * x: bf16 [rows, c_in], rows contiguous (pitch c_in); ln_w, ln_b: fp32 [c_in]
+ * (NULL = ones / zeros); w: bf16 [c_in, n_out] row-major; bias: fp32 [n_out]
+ * or NULL; y: bf16 [rows, n_out] with row pitch ldy >= n_out (elements).
+ * LayerNorm statistics and the products accumulate in fp32 (tensor cores).
+ * With w = [w_q | w_k | w_v | w_g] (each H*c wide) the column blocks of y are
+ * q, k, v and g of the attention, as [B, S, N, H, c] views with row stride
+ * 4*H*c that evo_attn_fwd / evo_attn_bwd take through their strides.
+ * Supported: c_in a multiple of 64 up to 256, n_out a multiple of 128, ldy a
+ * multiple of 8, x / w / y 16-byte aligned (else EVO_ERR_UNSUPPORTED); rows
+ * == 0 is a no-op.  Stream-ordered, no allocation, no synchronisation.
+ */
+evo_status_t evo_ln_linear(int64_t rows, int64_t c_in, int64_t n_out, const void* x,
+                           const float* ln_w, const float* ln_b, float eps,
+                           const void* w, const float* bias, void* y, int64_t ldy, void* stream);
+
+/*
+ * Pair-bias projection of the pair representation: the same LayerNorm +
+ * linear with one output per head, written in the layout the attention reads,
+ *   pair_bias[b, h, i, j] = sum_k LN(z[b, i, j, :])[k] * w[k, h] + bias[h].
+ * z: bf16 [B, N, N, c_z] contiguous; ln_w, ln_b: fp32 [c_z] (NULL = ones /
+ * zeros); w: bf16 [c_z, H]; bias: fp32 [H] or NULL; pair_bias: bf16
+ * [B, 1, H, N, N] contiguous.  Supported: c_z a multiple of 8 up to 1024,
+ * H <= 16, z 16-byte aligned.  Stream-ordered, no allocation.
+ */
+evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, const void* z,
+                              const float* ln_w, const float* ln_b, float eps,
+                              const void* w, const float* bias, void* pair_bias, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* evo_status_string(evo_status_t status);
 
@@ -212,11 +249,12 @@ uint64_t evo_attn_launch_count(void);
  * read (that phase is then left out of the sums).  Both functions are safe to
  * call from several host threads.
  */
-#define EVO_TIMING_PHASES 3
+#define EVO_TIMING_PHASES 4
 enum {
     EVO_PHASE_FWD_MAIN = 0,   /* the forward kernel                         */
     EVO_PHASE_BWD_MAIN = 1,   /* the backward's main (tensor-core) kernel    */
-    EVO_PHASE_BWD_ALL = 2     /* every kernel and memset of one evo_attn_bwd */
+    EVO_PHASE_BWD_ALL = 2,    /* every kernel and memset of one evo_attn_bwd */
+    EVO_PHASE_PROJ = 3        /* evo_ln_linear / evo_ln_pair_bias kernels    */
 };
 typedef struct {
     uint64_t calls[EVO_TIMING_PHASES];

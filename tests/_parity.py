@@ -5,6 +5,7 @@ Tolerances (per output tensor, over the compared elements):
   bf16 inputs, fp32 accumulation: max|gpu - oracle| <= 2e-2 and
                                   ||gpu - oracle||_2 / ||oracle||_2 <= 5e-3
   fp32 path:                      ||gpu - oracle||_2 / ||oracle||_2 <= 1e-4
+  fused LayerNorm + linear (bf16): element-wise projection_bound() and rel-L2 <= 5e-3
 """
 from __future__ import annotations
 
@@ -51,6 +52,20 @@ def oracle_fwd_bwd(inp, want=("dq", "dk", "dv", "dg", "d_pair_bias")):
         res.update(oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"],
                                    x["dout"], want=want))
     return res
+
+
+def projection_bound(x, ln_w, ln_b, eps, w, ref):
+    """Per-element error bound of y = LN(x) @ w + bias on the bf16 tensor-core path.
+
+    The path rounds the normalised activations LN(x) to bf16 before the product
+    (relative error <= 2^-9 each, so the dot product moves by at most
+    2^-9 * sum_k |LN(x)_k| |w_kn|) and rounds y to bf16 on the store (<= 2^-9 |y|);
+    fp32 statistics and accumulation over <= 256 terms add orders of magnitude
+    less.  Both terms are doubled for slack: 2^-8 * (|y| + |LN(x)| @ |w|).
+    All arguments fp64 arrays (ln_w, ln_b may be None); ref is the oracle's y.
+    """
+    ln = oracle.ln_linear(x, ln_w, ln_b, eps, np.eye(x.shape[-1]))      # LN(x) itself
+    return 2.0 ** -8 * (np.abs(ref) + np.abs(ln) @ np.abs(w))
 
 
 def metrics(got, ref):

@@ -86,6 +86,20 @@ def test_timing_hooks_answer_without_a_gpu(lib):
     assert A.timing_collect() == {p: (0, 0.0) for p in A.PHASES}   # nothing recorded, nothing waited on
 
 
+def test_projection_host_checks_need_no_gpu(lib):
+    nul, fake = None, ctypes.c_void_p(1 << 20)            # never dereferenced: the checks fail first
+    assert lib.evo_ln_linear(0, 256, 1024, nul, nul, nul, 1e-5, nul, nul, nul, 1024, nul) == 0   # empty
+    assert lib.evo_ln_linear(-1, 256, 1024, nul, nul, nul, 1e-5, nul, nul, nul, 1024, nul) == 1
+    assert lib.evo_ln_linear(8, 256, 1024, nul, nul, nul, 1e-5, nul, nul, nul, 1024, nul) == 1   # null x
+    assert lib.evo_ln_linear(8, 256, 1024, fake, nul, nul, 1e-5, fake, nul, fake, 512, nul) == 1  # ldy < n_out
+    assert lib.evo_ln_linear(8, 48, 1024, fake, nul, nul, 1e-5, fake, nul, fake, 1024, nul) == 2  # c_in % 64
+    assert lib.evo_ln_linear(8, 320, 1024, fake, nul, nul, 1e-5, fake, nul, fake, 1024, nul) == 2  # c_in > 256
+    assert lib.evo_ln_linear(8, 256, 192, fake, nul, nul, 1e-5, fake, nul, fake, 192, nul) == 2   # n_out % 128
+    assert lib.evo_ln_pair_bias(1, 16, 128, 17, fake, nul, nul, 1e-5, fake, nul, fake, nul) == 2  # H > 16
+    assert lib.evo_ln_pair_bias(1, 16, 12, 4, fake, nul, nul, 1e-5, fake, nul, fake, nul) == 2    # c_z % 8
+    assert lib.evo_ln_pair_bias(1, 0, 128, 4, nul, nul, nul, 1e-5, nul, nul, nul, nul) == 0       # empty
+
+
 def test_product_path_never_touches_the_oracle():
     """The package must not import, load or mention the CPU oracle."""
     pkg = os.path.join(ROOT, "evoformer_pair_bias_b200")

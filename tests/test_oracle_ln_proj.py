@@ -82,3 +82,26 @@ def test_planted_mistakes_fail_the_pins(mutant):
     ref = torch_ref(x, lw, lb, 1e-5, w, b)
     assert rel(oracle.ln_linear(x, lw, lb, 1e-5, w, b, mutant=mutant), ref) > 1e-3
     assert rel(oracle.ln_linear(x, lw, lb, 1e-5, w, b), ref) < RTOL
+
+
+def test_projection_bound_covers_a_bf16_emulation_and_is_tight():
+    # the GPU tolerance (projection_bound) against a CPU emulation of the
+    # tensor-core path's two roundings: LN(x) to bf16 before the product, y to
+    # bf16 after it; every element inside the bound, and the bound not vacuous
+    from _parity import projection_bound
+    r = np.random.default_rng(11)
+    rows, c_in, n_out = 4096, 256, 256
+    x = torch.tensor(r.standard_normal((rows, c_in))).to(torch.bfloat16).double().numpy()
+    w = torch.tensor(r.standard_normal((c_in, n_out)) / 16).to(torch.bfloat16).double().numpy()
+    lw, lb, b = 1 + 0.1 * r.standard_normal(c_in), 0.1 * r.standard_normal(c_in), r.standard_normal(n_out)
+    ref = oracle.ln_linear(x, lw, lb, 1e-5, w, b)
+    ln = torch.nn.functional.layer_norm(torch.tensor(x, dtype=torch.float32), (c_in,),
+                                        torch.tensor(lw, dtype=torch.float32), torch.tensor(lb, dtype=torch.float32),
+                                        1e-5)
+    y = (ln.to(torch.bfloat16).float() @ torch.tensor(w, dtype=torch.float32) + torch.tensor(b, dtype=torch.float32))
+    emu = y.to(torch.bfloat16).double().numpy()
+    bound = projection_bound(x, lw, lb, 1e-5, w, ref)
+    err = np.abs(emu - ref)
+    assert np.all(err <= bound)
+    assert err.max() > 0.1 * bound.max()                  # the emulation comes within 10x of the bound
+    assert not np.all(np.abs(ref + 0.05 - emu) <= bound)  # a 0.05 shift of y is caught
