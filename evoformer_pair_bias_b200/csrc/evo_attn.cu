@@ -217,16 +217,50 @@ evo_status_t bwd_f32(const evo_shape_t& sh, evo::simt::Args a, cudaStream_t stre
 }
 
 // ---------------------------------------------------------------- fused pre-attention projection
-template <int BNO>
+// maps[0]: w [c_in, n_out], boxes of 64 columns x c_in rows; maps[1]: y [rows, n_out] (pitch ldy),
+// boxes of 64 columns x 32 rows.  Persistent grid: n_slices x (CTAs per slice), at most one per SM.
+template <int BNO, int CIN>
 evo_status_t launch_ln_linear(const CUtensorMap* maps, const evo::proj::LnParams& p, cudaStream_t stream) {
-    using L = evo::proj::PLayout<BNO>;
-    auto kern = evo::proj::ln_linear_kernel<BNO>;
+    using L = evo::proj::PLayout<BNO, CIN>;
+    auto kern = evo::proj::ln_linear_kernel<BNO, CIN>;
     static cudaError_t attr = set_smem(kern, L::bytes);
     if (attr != cudaSuccess) return EVO_ERR_CUDA;
-    const dim3 grid((unsigned)((p.rows + evo::proj::BM - 1) / evo::proj::BM), (unsigned)(p.n_out / BNO));
+    const int64_t nsl = p.n_out / BNO;
+    const int64_t nrb = (p.rows + evo::proj::BM - 1) / evo::proj::BM;
+    const int64_t per_slice = std::min<int64_t>(nrb, std::max<int64_t>(1, sm_count() / nsl));
+    const int64_t grid = nsl * per_slice;
+    if (grid > 0x7fffffff) return EVO_ERR_UNSUPPORTED;
     {
         evo::timing::Scope t(EVO_PHASE_PROJ, stream);
-        kern<<<grid, evo::proj::THREADS, L::bytes, stream>>>(maps[0], maps[1], p);
+        kern<<<(unsigned)grid, evo::proj::THREADS, L::bytes, stream>>>(maps[0], maps[1], p);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+template <int BNO>
+evo_status_t launch_ln_linear_cin(const CUtensorMap* maps, const evo::proj::LnParams& p, cudaStream_t stream) {
+    switch (p.c_in) {
+        case 64: return launch_ln_linear<BNO, 64>(maps, p, stream);
+        case 128: return launch_ln_linear<BNO, 128>(maps, p, stream);
+        case 192: return launch_ln_linear<BNO, 192>(maps, p, stream);
+        case 256: return launch_ln_linear<BNO, 256>(maps, p, stream);
+    }
+    return EVO_ERR_UNSUPPORTED;
+}
+
+template <int CPL, int LPR>
+evo_status_t launch_pair_bias(const evo::proj::PbParams& p, int64_t total, cudaStream_t stream) {
+    auto kern = evo::proj::pair_bias_kernel<CPL, LPR>;
+    static cudaError_t attr = set_smem(kern, evo::proj::PB_SMEM);
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    const int64_t blocks = (total + evo::proj::PB_ROWS - 1) / evo::proj::PB_ROWS;
+    const int grid = (int)std::min<int64_t>(blocks, (int64_t)sm_count() * 8);
+    const int hp = (p.H + 3) & ~3;
+    const size_t shm = (size_t)p.c_z * hp * sizeof(float) + (size_t)p.H * evo::proj::PB_ROWS * 2;
+    {
+        evo::timing::Scope t(EVO_PHASE_PROJ, stream);
+        kern<<<grid, evo::proj::PB_THREADS, shm, stream>>>(p);
     }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
@@ -387,23 +421,21 @@ evo_status_t evo_ln_linear(int64_t rows, int64_t c_in, int64_t n_out, const void
     if (!x || !w || !y) return EVO_ERR_INVALID_ARG;
     if (c_in % evo::proj::KBOX != 0 || c_in > evo::proj::MAX_CIN || n_out % 128 != 0 || ldy % 8 != 0)
         return EVO_ERR_UNSUPPORTED;
+    if (rows > (int64_t)0x7fffffff - evo::proj::BM || n_out > (int64_t)0x7fffffff) return EVO_ERR_UNSUPPORTED;
     for (const void* q : {x, w, (const void*)y})
         if (!aligned(q, 16)) return EVO_ERR_UNSUPPORTED;
     for (const void* q : {(const void*)ln_w, (const void*)ln_b, (const void*)bias})
         if (q && !aligned(q, 4)) return EVO_ERR_INVALID_ARG;
     CUtensorMap maps[2];
     std::memset(maps, 0, sizeof(maps));
-    const bool wide = n_out % 256 == 0;
-    if (!evo::tma::matrix_bf16(&maps[0], x, rows, c_in, c_in, evo::proj::BM) ||
-        !evo::tma::matrix_bf16(&maps[1], w, c_in, n_out, n_out, (uint32_t)c_in))
+    if (!evo::tma::matrix_bf16(&maps[0], w, c_in, n_out, n_out, (uint32_t)c_in) ||
+        !evo::tma::matrix_bf16(&maps[1], y, rows, n_out, ldy, 32))
         return EVO_ERR_CUDA;
     evo::proj::LnParams p{};
     p.rows = (int)rows; p.c_in = (int)c_in; p.n_out = (int)n_out; p.eps = eps;
-    p.ln_w = ln_w; p.ln_b = ln_b; p.bias = bias;
-    p.y = static_cast<__nv_bfloat16*>(y); p.ldy = ldy;
-    if (rows > (int64_t)0x7fffffff) return EVO_ERR_UNSUPPORTED;
+    p.x = static_cast<const __nv_bfloat16*>(x); p.ln_w = ln_w; p.ln_b = ln_b; p.bias = bias;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return wide ? launch_ln_linear<256>(maps, p, s) : launch_ln_linear<128>(maps, p, s);
+    return n_out % 256 == 0 ? launch_ln_linear_cin<256>(maps, p, s) : launch_ln_linear_cin<128>(maps, p, s);
 }
 
 evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, const void* z, const float* ln_w,
@@ -420,17 +452,15 @@ evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, cons
     p.w = static_cast<const __nv_bfloat16*>(w); p.bias = bias;
     p.out = static_cast<__nv_bfloat16*>(pair_bias);
     const int64_t total = B * N * N;
-    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
-    const size_t shm = (size_t)c_z * H * sizeof(float);   // <= 64 KB
-    static cudaError_t attr = set_smem(evo::proj::pair_bias_kernel, (int)(1024 * evo::proj::PB_MAX_H * sizeof(float)));
-    if (attr != cudaSuccess) return EVO_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    {
-        evo::timing::Scope t(EVO_PHASE_PROJ, s);
-        evo::proj::pair_bias_kernel<<<grid, 256, shm, s>>>(p);
-    }
-    g_launches += 1;
-    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+    const int64_t chunks = c_z / 8;
+    if (chunks > 64) return launch_pair_bias<4, 32>(p, total, s);
+    if (chunks > 32) return launch_pair_bias<2, 32>(p, total, s);
+    if (chunks > 16) return launch_pair_bias<1, 32>(p, total, s);
+    if (chunks > 8) return launch_pair_bias<1, 16>(p, total, s);
+    if (chunks > 4) return launch_pair_bias<1, 8>(p, total, s);
+    if (chunks > 2) return launch_pair_bias<1, 4>(p, total, s);
+    return launch_pair_bias<1, 2>(p, total, s);      // at least 2 lanes per row: 16 rows per warp step
 }
 
 evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
