@@ -47,10 +47,13 @@ MUTANTS = {
     7: "dk missing its 1/sqrt(C) factor",
     8: "LayerNorm divides by the variance instead of its square root",
     9: "projection output columns shifted by one",
+    10: "triangular update without its third index (elementwise product of the two edges)",
+    11: "triangular update reading the second edge as k-j instead of j-k",
 }
 #: Which function each planted mistake breaks.
 ATTENTION_MUTANTS = (1, 2, 3, 4, 5, 6, 7)
 LN_LINEAR_MUTANTS = (8, 9)
+TRI_MUL_MUTANTS = (10, 11)
 
 
 class _Dims(ctypes.Structure):
@@ -87,6 +90,8 @@ def _lib(mutant: int = 0) -> ctypes.CDLL:
         lib.evo_ref_mutant.restype = ctypes.c_int
         lib.evo_ref_ln_linear.argtypes = [ctypes.c_int64] * 3 + [p] * 3 + [ctypes.c_double] + [p] * 3
         lib.evo_ref_ln_linear.restype = ctypes.c_int
+        lib.evo_ref_tri_mul.argtypes = [ctypes.c_int64] * 3 + [p] * 2 + [ctypes.c_int, p]
+        lib.evo_ref_tri_mul.restype = ctypes.c_int
         _LIBS[mutant] = lib
     return _LIBS[mutant]
 
@@ -190,6 +195,25 @@ def ln_linear(x, ln_w, ln_b, eps, w, bias=None, *, mutant: int = 0):
     if rc != 0:
         raise ValueError("evo_ref_ln_linear rejected its arguments")
     return y.reshape(lead + (n_out,))
+
+
+def tri_mul(a, b, incoming: bool = False, *, mutant: int = 0):
+    """The contraction of the triangular multiplicative update, in fp64.
+
+    a, b: [B, N, N, C] (the pair representation's layout).  Outgoing edges
+    (default): z[b, i, j, c] = sum_k a[b, i, k, c] * b[b, j, k, c]; incoming:
+    z[b, i, j, c] = sum_k a[b, k, i, c] * b[b, k, j, c] ("Evoformer: the memory
+    wall ZeRO cannot move", section "The three operations").
+    """
+    a, b = _f64(a), _f64(b)
+    if a.ndim != 4 or a.shape != b.shape or a.shape[1] != a.shape[2]:
+        raise ValueError(f"a {a.shape} and b {b.shape} must both be [B, N, N, C]")
+    B, N, _, C = a.shape
+    z = np.empty_like(a)
+    rc = _lib(mutant).evo_ref_tri_mul(B, N, C, _ptr(a), _ptr(b), 1 if incoming else 0, _ptr(z))
+    if rc != 0:
+        raise ValueError("evo_ref_tri_mul rejected its arguments")
+    return z
 
 
 def mutant_id(mutant: int) -> int:

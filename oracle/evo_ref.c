@@ -41,7 +41,8 @@
  * subset of query rows (a smaller, equally valid problem).
  *
  * The file also holds the fused pre-attention projection (LayerNorm + linear,
- * evo_ref_ln_linear below) that produces q, k, v, g and the pair bias.
+ * evo_ref_ln_linear below) that produces q, k, v, g and the pair bias, and
+ * the contraction of the triangular multiplicative update (evo_ref_tri_mul).
  *
  * Planted mistakes (mutation testing of the pins): building with
  * -DEVO_REF_MUTANT=n swaps in one deliberate error, see mutant_* below.
@@ -321,6 +322,51 @@ int evo_ref_ln_linear(int64_t rows, int64_t c_in, int64_t n_out, const double* x
             }
         }
         free(n);
+    }
+    return 0;
+}
+
+/*
+ * Triangular multiplicative update, the contraction at its core ("Evoformer:
+ * the memory wall ZeRO cannot move", section "The three operations"): edge
+ * (i, j) is updated from every third residue k, channel by channel,
+ *
+ *   outgoing edges (i-k and j-k):  z[b,i,j,c] = sum_k a[b,i,k,c] * bb[b,j,k,c]
+ *   incoming edges (k-i and k-j):  z[b,i,j,c] = sum_k a[b,k,i,c] * bb[b,k,j,c]
+ *
+ * a, bb, z: [B, N, N, C] contiguous fp64, the layout of the pair
+ * representation.  O(N^3 C) time; the sum over k contracts as it goes.
+ * Returns 0, or -1 for a bad size.
+ */
+int evo_ref_tri_mul(int64_t B, int64_t N, int64_t C, const double* a, const double* bb, int incoming,
+                    double* z) {
+    if (B < 0 || N < 0 || C <= 0) return -1;
+    const int64_t nn = N * N;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t i = 0; i < N; ++i) {
+            const double* ab = a + b * nn * C;
+            const double* bbb = bb + b * nn * C;
+            for (int64_t j = 0; j < N; ++j) {
+                double* zr = z + ((b * N + i) * N + j) * C;
+                for (int64_t c = 0; c < C; ++c) zr[c] = 0.0;
+#if EVO_REF_MUTANT == 10
+                /* mutant: no third index -- the elementwise product of the two edges */
+                for (int64_t c = 0; c < C; ++c) zr[c] = ab[(i * N + j) * C + c] * bbb[(i * N + j) * C + c];
+#else
+                for (int64_t k = 0; k < N; ++k) {
+                    const double* ar = incoming ? ab + (k * N + i) * C : ab + (i * N + k) * C;
+#if EVO_REF_MUTANT == 11
+                    /* mutant: second operand read as the edge k-j in outgoing mode */
+                    const double* br = incoming ? bbb + (k * N + j) * C : bbb + (k * N + j) * C;
+#else
+                    const double* br = incoming ? bbb + (k * N + j) * C : bbb + (j * N + k) * C;
+#endif
+                    for (int64_t c = 0; c < C; ++c) zr[c] += ar[c] * br[c];
+                }
+#endif
+            }
+        }
     }
     return 0;
 }
