@@ -24,6 +24,12 @@ y = LayerNorm(x) @ [w_q | w_k | w_v | w_g] + bias over every row of the MSA
 (or pair) representation, and for the pair representation also the
 pair-bias projection LayerNorm(z) @ w_b + b_b.  Metric: TFLOP/s of the
 projection GEMMs (2 * rows * c_in * n_out), with the same timing rules.
+
+``--workload tri_mul_256 | tri_mul_384 | tri_mul_768`` benchmarks the
+contraction of the triangular multiplicative update ("Evoformer: the memory
+wall ZeRO cannot move", section "The three operations"): one step is the
+outgoing-edge update z[b,c,i,j] = sum_k a[b,c,i,k] b[b,c,j,k] over every channel,
+then the incoming-edge one; metric TFLOP/s (2 * B * C * N^3 per direction).
 """
 from __future__ import annotations
 
@@ -43,10 +49,12 @@ sys.path.insert(0, ROOT)
 
 from evoformer_pair_bias_b200 import attention as A  # noqa: E402
 from evoformer_pair_bias_b200.workloads import (WORKLOADS, DEFAULT_BENCH, PROJ_WORKLOADS, logical_view,  # noqa: E402
-                                                make_inputs, make_pair_bias_params, make_proj_inputs)
+                                                make_inputs, make_pair_bias_params, make_proj_inputs,
+                                                TRI_MUL_WORKLOADS, make_tri_mul_inputs)
 
 METRIC = "Evoformer pair-bias attention fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
 PROJ_METRIC = "fused LayerNorm + linear pre-attention projection TFLOP/s"
+TRI_METRIC = "triangular multiplicative update contraction TFLOP/s"
 PROJ_EPS = 1e-5
 NOMINAL_BF16_TFLOPS = 2250.0
 
@@ -468,40 +476,64 @@ def run_projection(args, pw, rank, world, local):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step(x):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
-        ev[0].record()
         A.ln_linear(x, d["ln_w"], d["ln_b"], PROJ_EPS, d["w"], d["bias"], y=y)
-        ev[1].record()
         if pbp is not None:
             A.ln_pair_bias(x, pbp["ln_w"], pbp["ln_b"], PROJ_EPS, pbp["w"], pbp["bias"], out=pb)
-            ev[2].record()
-        return ev
 
+    A.timing_enable(True)
     for _ in range(args.warmup):
         flush.zero_()
         step(d["x"])
     torch.cuda.synchronize()
+    A.timing_collect()
     if A.device_status(clear=True) != 0:
         raise RuntimeError("a kernel reported an error during warm-up")
     K = args.steps
-    evs = []
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     with ClockSampler(gpu_uuid(dev)) as clk:
         barrier()
         torch.cuda.synchronize()
         n0 = A.launch_count()
-        for _ in range(K):
+        for i in range(K):
             flush.zero_()
-            evs.append(step(d["x"]))
+            ev[i][0].record()
+            step(d["x"])
+            ev[i][1].record()
         torch.cuda.synchronize()
         barrier()
         launches = A.launch_count() - n0
-    per_part = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(len(parts))]
-    tot = sum(per_part)
-    tot, *per_part = max_over_ranks([tot] + per_part, world, dev)
+    kt = A.timing_collect()
+    A.timing_enable(False)
+    tot = max_over_ranks([sum(e0.elapsed_time(e1) for e0, e1 in ev)], world, dev)[0]
     if A.device_status(clear=True) != 0:
         raise RuntimeError("a kernel reported an error during the timed region")
     value = job_throughput(fl_step, K, world, tot)
     pk = peaks()
+    phase = {"qkvg": "proj", "pair_bias": "pair_bias"}
+    us = {p: 1e3 * kt[phase[p]][1] / max(kt[phase[p]][0], 1) for p in parts}
+
+    # the same step replayed from a CUDA graph: no host launch overhead between the kernels
+    graph_ms = None
+    try:
+        s_cap = torch.cuda.Stream()
+        s_cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_cap):
+            step(d["x"])
+        torch.cuda.current_stream().wait_stream(s_cap)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            step(d["x"])
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            gev[i][0].record()
+            gr.replay()
+            gev[i][1].record()
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in gev)], world, dev)[0] / K
+        del gr
+    except Exception as exc:  # reported, never required
+        graph_ms = repr(exc)
 
     e2e = None
     if not args.no_e2e:
@@ -544,7 +576,6 @@ def run_projection(args, pw, rank, world, local):
             cpu = {"error": repr(exc)}
 
     if rank == 0:
-        us = {p: 1e3 * per_part[j] / K for j, p in enumerate(parts)}
         top = max(parts, key=lambda p: us[p])
         line = {
             "metric": PROJ_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
@@ -553,8 +584,213 @@ def run_projection(args, pw, rank, world, local):
             "config": {**base_cfg, "l2": "flushed (256 MB write) before every step",
                        "parallelism": f"replicas x{world}, rows independent, no collective"},
             "roofline": proj_roofline(pw, top, us[top], pk, timed_s=tot * 1e-3),
-            "kernels": {p: {"launches": K, "us_per_launch": us[p],
+            "kernels": {p: {"launches": kt[phase[p]][0], "us_per_launch": us[p],
                             "roofline": proj_roofline(pw, p, us[p], pk, timed_s=tot * 1e-3)} for p in parts},
+            "graph_ms_per_step": graph_ms,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Triangular multiplicative update (its contraction)
+
+
+def tri_algorithmic(tw):
+    """(FLOPs, bytes) of one launch (one direction): a and b read once, z written once (bf16)."""
+    return tw.flops, 3 * tw.B * tw.C * tw.N * tw.N * 2
+
+
+def tri_oracle_sample(tw, target_s: float = 12.0):
+    """Time the fp64 oracle (both directions) on the first r channels of the workload."""
+    import oracle
+    oracle.build()
+    d = make_tri_mul_inputs(tw)
+    a_all = d["a"].double().permute(0, 2, 3, 1)
+    b_all = d["b"].double().permute(0, 2, 3, 1)
+
+    def run(r):
+        a = a_all[:1, :, :, :r].contiguous().numpy()
+        b = b_all[:1, :, :, :r].contiguous().numpy()
+        t0 = time.perf_counter()
+        oracle.tri_mul(a, b, False)
+        oracle.tri_mul(a, b, True)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    r = max(1, min(tw.C, int(target_s / max(t1, 1e-6) / 2)))
+    t, reps = 0.0, 0
+    while reps == 0 or t < 0.7 * target_s:
+        t += run(r)
+        reps += 1
+    fl = 2 * 2 * r * tw.N ** 3 * reps
+    return dict(value=fl / t / 1e12, unit="TFLOP/s", cores=oracle_threads(), kind="oracle",
+                sample=f"{r} of {tw.B * tw.C} channel matrices x{reps}, both directions, fp64, {t:.2f} s",
+                seconds=t, channels=r)
+
+
+def run_tri_mul(args, tw, rank, world, local):
+    fl_launch, by_launch = tri_algorithmic(tw)
+    fl_step = 2 * fl_launch
+    cfg = {"workload": tw.name, "B": tw.B, "N_res": tw.N, "C": tw.C, "layout": "channel-first [B, C, N, N]",
+           "directions": ["outgoing", "incoming"]}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps, warm = args.steps, args.warmup
+        info = tri_oracle_sample(tw, target_s=max(0.5, 60.0 / max(1, steps + warm)))
+        r = info["channels"]
+        import oracle
+        d = make_tri_mul_inputs(tw)
+        a = d["a"].double().permute(0, 2, 3, 1)[:1, :, :, :r].contiguous().numpy()
+        b = d["b"].double().permute(0, 2, 3, 1)[:1, :, :, :r].contiguous().numpy()
+        times = []
+        for i in range(warm + steps):
+            t0 = time.perf_counter()
+            oracle.tri_mul(a, b, False)
+            oracle.tri_mul(a, b, True)
+            if i >= warm:
+                times.append(time.perf_counter() - t0)
+        t = sum(times)
+        val = 2 * 2 * r * tw.N ** 3 * steps / t / 1e12
+        line = {"metric": TRI_METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps,
+                "warmup": warm, "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {**cfg, "sample_channels": r, "l2": "n/a (CPU)"},
+                "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": f"{r} of {tw.B * tw.C} channel matrices per step, fp64"},
+                "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import datetime
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    A.load_library()
+    hin = make_tri_mul_inputs(tw)
+    d = {k: v.to(dev) for k, v in hin.items()}
+    z_out = torch.empty_like(d["a"])
+    z_in = torch.empty_like(d["a"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(a, b):
+        A.tri_mul(a, b, False, z=z_out)
+        A.tri_mul(a, b, True, z=z_in)
+
+    A.timing_enable(True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(d["a"], d["b"])
+    torch.cuda.synchronize()
+    A.timing_collect()
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported an error during warm-up")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with ClockSampler(gpu_uuid(dev)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        n0 = A.launch_count()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record()
+            step(d["a"], d["b"])
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        launches = A.launch_count() - n0
+    kt = A.timing_collect()
+    A.timing_enable(False)
+    tot = max_over_ranks([sum(e0.elapsed_time(e1) for e0, e1 in ev)], world, dev)[0]
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported an error during the timed region")
+    value = job_throughput(fl_step, K, world, tot)
+    pk = peaks()
+    n_l, ms_l = kt["tri_mul"]
+    us = 1e3 * ms_l / max(n_l, 1)
+    sec = us * 1e-6
+    sustained = tot * 1e-3 > 1.0
+    tflops_peak = pk["bf16_sustained"] if sustained else pk["bf16"]
+    t_tensor, t_hbm = fl_launch / (tflops_peak * 1e12), by_launch / (pk["hbm"] * 1e9)
+    tr = TRAFFIC.get(("tri_mul", tw.name))
+    common = {"kernel": "trimul::tri_mul_kernel", "launches": n_l, "us_per_launch": us, "flops_per_launch": fl_launch,
+              "algorithmic_bytes_per_launch": by_launch,
+              "traffic": tr[0] if tr is not None and _source_sha(tr[1]) == tr[2] else None,
+              "tensor_floor_us": t_tensor * 1e6, "hbm_floor_us": t_hbm * 1e6}
+    if t_tensor >= t_hbm:
+        a_ = fl_launch / sec / 1e12
+        roof = {"bound": "tensor", "achieved": a_, "peak": tflops_peak, "unit": "TFLOP/s", "frac": a_ / tflops_peak,
+                "peak_source": f"{pk['source']} bf16 {'sustained' if sustained else 'burst'}", **common}
+    else:
+        a_ = by_launch / sec / 1e9
+        roof = {"bound": "hbm", "achieved": a_, "peak": pk["hbm"], "unit": "GB/s", "frac": a_ / pk["hbm"],
+                "peak_source": f"{pk['source']} HBM copy", "tensor_frac": fl_launch / sec / 1e12 / tflops_peak,
+                **common}
+
+    e2e = None
+    if not args.no_e2e:
+        ha, hb = hin["a"].pin_memory(), hin["b"].pin_memory()
+        hzo = torch.empty(z_out.shape, dtype=z_out.dtype).pin_memory()
+        hzi = torch.empty(z_in.shape, dtype=z_in.dtype).pin_memory()
+        da, db = torch.empty_like(ha, device=dev), torch.empty_like(hb, device=dev)
+
+        def e2e_step():
+            da.copy_(ha, non_blocking=True)
+            db.copy_(hb, non_blocking=True)
+            step(da, db)
+            hzo.copy_(z_out, non_blocking=True)
+            hzi.copy_(z_in, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        et = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+        e2e = {"value": job_throughput(fl_step, K, world, et), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 2 * ha.numel() * ha.element_size(),
+               "d2h_bytes_per_step": 2 * hzo.numel() * hzo.element_size(), "ms_per_step": et / K}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            cpu = tri_oracle_sample(tw)
+            cpu.pop("seconds", None)
+            cpu.pop("channels", None)
+        except Exception as exc:  # the baseline is reported, never required
+            cpu = {"error": repr(exc)}
+
+    if rank == 0:
+        line = {
+            "metric": TRI_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": tot / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**cfg, "l2": "flushed (256 MB write) before every step",
+                       "parallelism": f"replicas x{world}, channels independent, no collective"},
+            "roofline": roof,
+            "kernels": {"tri_mul": {"launches": n_l, "us_per_launch": us}},
+            "frac_measured_peak": value / world / pk["bf16"],
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
@@ -572,7 +808,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS) + sorted(PROJ_WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS) + sorted(PROJ_WORKLOADS) + sorted(TRI_MUL_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -584,6 +820,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.workload in PROJ_WORKLOADS:
         return run_projection(args, PROJ_WORKLOADS[args.workload], rank, world, local)
+    if args.workload in TRI_MUL_WORKLOADS:
+        return run_tri_mul(args, TRI_MUL_WORKLOADS[args.workload], rank, world, local)
     w = WORKLOADS[args.workload]
 
     if args.impl == "reference":

@@ -33,7 +33,8 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 #: Every symbol include/evo_attn.h declares.
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
            "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc",
-           "evo_attn_timing_enable", "evo_attn_timing_collect", "evo_ln_linear", "evo_ln_pair_bias")
+           "evo_attn_timing_enable", "evo_attn_timing_collect", "evo_ln_linear", "evo_ln_pair_bias",
+           "evo_tri_mul")
 
 #: Size of the library's fixed scratch area used by evo_attn_bwd_noalloc (bytes).
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -54,7 +55,7 @@ class Strides(ctypes.Structure):
 
 
 #: Timing phases (evo_timing_t indices).
-PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj")
+PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj", "pair_bias", "tri_mul")
 
 
 class Timing(ctypes.Structure):
@@ -98,6 +99,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_ln_linear.restype = ctypes.c_int
     lib.evo_ln_pair_bias.argtypes = [i64, i64, i64, i64, vp, vp, vp, f32, vp, vp, vp, vp]
     lib.evo_ln_pair_bias.restype = ctypes.c_int
+    lib.evo_tri_mul.argtypes = [i64, i64, i64, vp, vp, ctypes.c_int, vp, vp]
+    lib.evo_tri_mul.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -292,6 +295,24 @@ def ln_pair_bias(z, ln_w, ln_b, eps, w, bias=None, out=None):
                               _ptr(out), _stream(z.device))
     _check("evo_ln_pair_bias", rc)
     return out
+
+
+def tri_mul(a, b, incoming: bool = False, z=None):
+    """Triangular multiplicative update contraction on channel-first bf16 [B, C, N, N] tensors.
+
+    Outgoing edges: z[b, c, i, j] = sum_k a[b, c, i, k] * b[b, c, j, k]; incoming:
+    z[b, c, i, j] = sum_k a[b, c, k, i] * b[b, c, k, j].  Returns z (bf16, same shape).
+    """
+    lib = load_library()
+    if a.dim() != 4 or a.shape != b.shape or a.shape[2] != a.shape[3]:
+        raise ValueError("a and b must both be [B, C, N, N]")
+    B, C, N, _ = a.shape
+    ac, bc = a.contiguous(), b.contiguous()
+    if z is None:
+        z = torch.empty_like(ac)
+    rc = lib.evo_tri_mul(B, C, N, _ptr(ac), _ptr(bc), 1 if incoming else 0, _ptr(z), _stream(a.device))
+    _check("evo_tri_mul", rc)
+    return z
 
 
 def timing_enable(on: bool = True) -> None:

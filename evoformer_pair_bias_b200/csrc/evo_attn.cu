@@ -25,6 +25,7 @@
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "proj_sm100.cuh"
+#include "trimul_sm100.cuh"
 
 #define EVO_VERSION 10000
 
@@ -259,7 +260,7 @@ evo_status_t launch_pair_bias(const evo::proj::PbParams& p, int64_t total, cudaS
     const int hp = (p.H + 3) & ~3;
     const size_t shm = (size_t)p.c_z * hp * sizeof(float) + (size_t)p.H * evo::proj::PB_ROWS * 2;
     {
-        evo::timing::Scope t(EVO_PHASE_PROJ, stream);
+        evo::timing::Scope t(EVO_PHASE_PAIR_BIAS, stream);
         kern<<<grid, evo::proj::PB_THREADS, shm, stream>>>(p);
     }
     g_launches += 1;
@@ -461,6 +462,39 @@ evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, cons
     if (chunks > 4) return launch_pair_bias<1, 8>(p, total, s);
     if (chunks > 2) return launch_pair_bias<1, 4>(p, total, s);
     return launch_pair_bias<1, 2>(p, total, s);      // at least 2 lanes per row: 16 rows per warp step
+}
+
+evo_status_t evo_tri_mul(int64_t B, int64_t C, int64_t N, const void* a, const void* bb, int incoming,
+                         void* z, void* stream) {
+    if (B < 0 || C < 0 || N < 0) return EVO_ERR_INVALID_ARG;
+    if (B == 0 || C == 0 || N == 0) return EVO_OK;
+    if (!a || !bb || !z) return EVO_ERR_INVALID_ARG;
+    const int64_t BC = B * C;
+    if (N % 8 != 0 || BC > (int64_t)0x7fffffff || N > (int64_t)0x7fffffff / 2) return EVO_ERR_UNSUPPORTED;
+    for (const void* q : {a, bb, (const void*)z})
+        if (!aligned(q, 16)) return EVO_ERR_UNSUPPORTED;
+    using namespace evo::trimul;
+    CUtensorMap maps[3];
+    std::memset(maps, 0, sizeof(maps));
+    const bool in = incoming != 0;
+    if (!evo::tma::stack_bf16(&maps[0], a, N, BC, 64, in ? 64 : BM) ||
+        !evo::tma::stack_bf16(&maps[1], bb, N, BC, 64, in ? 64 : BN) ||
+        !evo::tma::stack_bf16(&maps[2], z, N, BC, 64, 32))
+        return EVO_ERR_CUDA;
+    TriParams p{};
+    p.N = (int)N; p.BC = (int)BC; p.incoming = in ? 1 : 0;
+    p.tiles_i = (int)((N + BM - 1) / BM); p.tiles_j = (int)((N + BN - 1) / BN);
+    const int64_t tiles = BC * p.tiles_i * p.tiles_j;
+    static cudaError_t attr = set_smem(tri_mul_kernel, TLayout::bytes);
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    const int grid = (int)std::min<int64_t>(tiles, sm_count());
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    {
+        evo::timing::Scope t(EVO_PHASE_TRI_MUL, s);
+        tri_mul_kernel<<<grid, THREADS, TLayout::bytes, s>>>(maps[0], maps[1], maps[2], p);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
 evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,

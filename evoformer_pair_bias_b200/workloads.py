@@ -188,7 +188,7 @@ def ceil_div(a: int, b: int) -> int:
 __all__ = ["Workload", "WORKLOADS", "DEFAULT_BENCH", "MASK_VALUE", "make_inputs",
            "logical_view", "storage_empty", "sample_rows", "logits_bytes", "pair_rep_bytes",
            "mask_columns", "ceil_div", "ProjWorkload", "PROJ_WORKLOADS", "make_proj_inputs",
-           "make_pair_bias_params"]
+           "make_pair_bias_params", "TriMulWorkload", "TRI_MUL_WORKLOADS", "make_tri_mul_inputs"]
 
 
 # ---------------------------------------------------------------------------
@@ -259,3 +259,43 @@ def make_pair_bias_params(w: ProjWorkload, device="cpu") -> dict:
     bias = torch.randn(w.H, generator=g)
     return {"w": wt.to(torch.bfloat16).to(device), "ln_w": ln_w.to(device), "ln_b": ln_b.to(device),
             "bias": bias.to(device)}
+
+
+# ---------------------------------------------------------------------------
+# Triangular multiplicative update (its contraction): seeded inputs only.
+#
+# Recipe (generator seeded with ``seed``): a then b ~ N(0, 1) drawn as
+# [B, C, N, N] (channel-first, the layout the contraction reads), scaled by
+# N^(-1/4) so that z = sum_k a b stays O(1) whatever N, rounded to bf16.
+# Shapes: the pair representation of N residues with C = 128 hidden channels
+# (the update's width in AlphaFold2-style trunks).
+
+
+@dataclasses.dataclass(frozen=True)
+class TriMulWorkload:
+    name: str
+    B: int
+    N: int
+    C: int
+    seed: int
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.B * self.C * self.N ** 3
+
+
+TRI_MUL_WORKLOADS = {
+    "tri_mul_256": TriMulWorkload("tri_mul_256", 1, 256, 128, 20281),
+    "tri_mul_384": TriMulWorkload("tri_mul_384", 1, 384, 128, 20282),
+    "tri_mul_768": TriMulWorkload("tri_mul_768", 1, 768, 128, 20283),
+    "tri_mul_tiny": TriMulWorkload("tri_mul_tiny", 2, 40, 3, 20284),
+}
+
+
+def make_tri_mul_inputs(w: TriMulWorkload, device="cpu") -> dict:
+    """a, b: bf16 [B, C, N, N] (channel-first)."""
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    s = w.N ** -0.25
+    a = torch.randn((w.B, w.C, w.N, w.N), generator=g) * s
+    b = torch.randn((w.B, w.C, w.N, w.N), generator=g) * s
+    return {"a": a.to(torch.bfloat16).to(device), "b": b.to(torch.bfloat16).to(device)}

@@ -218,6 +218,25 @@ evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, cons
                               const float* ln_w, const float* ln_b, float eps,
                               const void* w, const float* bias, void* pair_bias, void* stream);
 
+/*
+ * The contraction of the triangular multiplicative update ("Evoformer: the
+ * memory wall ZeRO cannot move", section "The three operations"): every edge
+ * (i, j) gathers the third residues k, channel by channel,
+ *
+ *   outgoing (incoming == 0):  z[b,c,i,j] = sum_k a[b,c,i,k] * bb[b,c,j,k]
+ *   incoming (incoming != 0):  z[b,c,i,j] = sum_k a[b,c,k,i] * bb[b,c,k,j]
+ *
+ * one N x N x N matrix product per (b, c).  a, bb, z: bf16 [B, C, N, N]
+ * contiguous (channel-first: the matrix of each (b, c) contiguous); products
+ * accumulate in fp32 on the tensor cores and z is rounded to bf16 on the
+ * store.  Supported: N a multiple of 8, a / bb / z 16-byte aligned, B*C and
+ * N below 2^31 (else EVO_ERR_UNSUPPORTED); B, C or N == 0 is a no-op.
+ * Stream-ordered, no allocation, no synchronisation; the kernel's waits are
+ * bounded, and one that gives up is reported by evo_attn_device_status.
+ */
+evo_status_t evo_tri_mul(int64_t B, int64_t C, int64_t N, const void* a, const void* bb, int incoming,
+                         void* z, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* evo_status_string(evo_status_t status);
 
@@ -238,10 +257,11 @@ uint64_t evo_attn_launch_count(void);
 
 /*
  * Per-kernel device timing (off by default).  While switched on, each
- * evo_attn_fwd / evo_attn_bwd call records a pair of CUDA events on its own
- * `stream` around its main kernel, and evo_attn_bwd a second pair around all
- * of its kernels, so that a caller can see how a step's device time splits
- * between the kernels without a profiler.  The events come from a pool kept
+ * evo_attn_fwd / evo_attn_bwd / evo_ln_linear / evo_ln_pair_bias / evo_tri_mul call records
+ * a pair of CUDA events on its own `stream` around its main kernel, and
+ * evo_attn_bwd a second pair around all of its kernels, so that a caller can
+ * see how a step's device time splits between the kernels without a
+ * profiler.  The events come from a pool kept
  * by the library (created on first use, reused afterwards); recording them
  * adds no kernel and no synchronisation.  Recording is best-effort: if an
  * event cannot be created or recorded that call simply goes untimed.
@@ -253,12 +273,14 @@ uint64_t evo_attn_launch_count(void);
  * read (that phase is then left out of the sums).  Both functions are safe to
  * call from several host threads.
  */
-#define EVO_TIMING_PHASES 4
+#define EVO_TIMING_PHASES 6
 enum {
     EVO_PHASE_FWD_MAIN = 0,   /* the forward kernel                         */
     EVO_PHASE_BWD_MAIN = 1,   /* the backward's main (tensor-core) kernel    */
     EVO_PHASE_BWD_ALL = 2,    /* every kernel and memset of one evo_attn_bwd */
-    EVO_PHASE_PROJ = 3        /* evo_ln_linear / evo_ln_pair_bias kernels    */
+    EVO_PHASE_PROJ = 3,       /* the evo_ln_linear kernel                    */
+    EVO_PHASE_PAIR_BIAS = 4,  /* the evo_ln_pair_bias kernel                 */
+    EVO_PHASE_TRI_MUL = 5     /* the evo_tri_mul kernel                      */
 };
 typedef struct {
     uint64_t calls[EVO_TIMING_PHASES];

@@ -6,6 +6,7 @@ Tolerances (per output tensor, over the compared elements):
                                   ||gpu - oracle||_2 / ||oracle||_2 <= 5e-3
   fp32 path:                      ||gpu - oracle||_2 / ||oracle||_2 <= 1e-4
   fused LayerNorm + linear (bf16): element-wise projection_bound() and rel-L2 <= 5e-3
+  triangular update contraction (bf16): element-wise tri_mul_bound() and rel-L2 <= 5e-3
 """
 from __future__ import annotations
 
@@ -66,6 +67,18 @@ def projection_bound(x, ln_w, ln_b, eps, w, ref):
     """
     ln = oracle.ln_linear(x, ln_w, ln_b, eps, np.eye(x.shape[-1]))      # LN(x) itself
     return 2.0 ** -8 * (np.abs(ref) + np.abs(ln) @ np.abs(w))
+
+
+def tri_mul_bound(a, b, incoming, ref):
+    """Per-element error bound of the bf16 tensor-core contraction z = sum_k a b.
+
+    The inputs are exact bf16 values; the products accumulate in fp32 over N
+    terms (error <= N 2^-24 sum_k |a| |b| <= 2^-12 sum_k |a| |b| for N <= 4096)
+    and z is rounded to bf16 on the store (<= 2^-9 |z|, doubled for slack).
+    a, b: fp64 arrays in the oracle's [B, N, N, C] layout; ref: the oracle's z.
+    """
+    mag = oracle.tri_mul(np.abs(a), np.abs(b), incoming)
+    return 2.0 ** -8 * np.abs(ref) + 2.0 ** -12 * mag
 
 
 def metrics(got, ref):
