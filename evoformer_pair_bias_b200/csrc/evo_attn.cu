@@ -250,21 +250,34 @@ evo_status_t launch_ln_linear_cin(const CUtensorMap* maps, const evo::proj::LnPa
     return EVO_ERR_UNSUPPORTED;
 }
 
-template <int CPL, int LPR>
+template <int CPL, int LPR, int HQ>
 evo_status_t launch_pair_bias(const evo::proj::PbParams& p, int64_t total, cudaStream_t stream) {
-    auto kern = evo::proj::pair_bias_kernel<CPL, LPR>;
+    auto kern = evo::proj::pair_bias_kernel<CPL, LPR, HQ>;
     static cudaError_t attr = set_smem(kern, evo::proj::PB_SMEM);
     if (attr != cudaSuccess) return EVO_ERR_CUDA;
     const int64_t blocks = (total + evo::proj::PB_ROWS - 1) / evo::proj::PB_ROWS;
-    const int grid = (int)std::min<int64_t>(blocks, (int64_t)sm_count() * 8);
-    const int hp = (p.H + 3) & ~3;
-    const size_t shm = (size_t)p.c_z * hp * sizeof(float) + (size_t)p.H * evo::proj::PB_ROWS * 2;
+    const size_t shm = (size_t)p.c_z * 4 * HQ * sizeof(float) + (size_t)4 * HQ * evo::proj::PB_ROWS * 2;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, evo::proj::PB_THREADS, shm) != cudaSuccess)
+        return EVO_ERR_CUDA;
+    const int grid = (int)std::min<int64_t>(blocks, (int64_t)sm_count() * std::max(per_sm, 1));
     {
         evo::timing::Scope t(EVO_PHASE_PAIR_BIAS, stream);
         kern<<<grid, evo::proj::PB_THREADS, shm, stream>>>(p);
     }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+template <int CPL, int LPR>
+evo_status_t launch_pair_bias_h(const evo::proj::PbParams& p, int64_t total, cudaStream_t stream) {
+    switch ((p.H + 3) / 4) {
+        case 1: return launch_pair_bias<CPL, LPR, 1>(p, total, stream);
+        case 2: return launch_pair_bias<CPL, LPR, 2>(p, total, stream);
+        case 3: return launch_pair_bias<CPL, LPR, 3>(p, total, stream);
+        case 4: return launch_pair_bias<CPL, LPR, 4>(p, total, stream);
+    }
+    return EVO_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -455,13 +468,13 @@ evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, cons
     const int64_t total = B * N * N;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t chunks = c_z / 8;
-    if (chunks > 64) return launch_pair_bias<4, 32>(p, total, s);
-    if (chunks > 32) return launch_pair_bias<2, 32>(p, total, s);
-    if (chunks > 16) return launch_pair_bias<1, 32>(p, total, s);
-    if (chunks > 8) return launch_pair_bias<1, 16>(p, total, s);
-    if (chunks > 4) return launch_pair_bias<1, 8>(p, total, s);
-    if (chunks > 2) return launch_pair_bias<1, 4>(p, total, s);
-    return launch_pair_bias<1, 2>(p, total, s);      // at least 2 lanes per row: 16 rows per warp step
+    if (chunks > 64) return launch_pair_bias_h<4, 32>(p, total, s);
+    if (chunks > 32) return launch_pair_bias_h<2, 32>(p, total, s);
+    if (chunks > 16) return launch_pair_bias_h<1, 32>(p, total, s);
+    if (chunks > 8) return launch_pair_bias_h<1, 16>(p, total, s);
+    if (chunks > 4) return launch_pair_bias_h<1, 8>(p, total, s);
+    if (chunks > 2) return launch_pair_bias_h<1, 4>(p, total, s);
+    return launch_pair_bias_h<1, 2>(p, total, s);    // at least 2 lanes per row: 16 rows per warp step
 }
 
 evo_status_t evo_tri_mul(int64_t B, int64_t C, int64_t N, const void* a, const void* bb, int incoming,

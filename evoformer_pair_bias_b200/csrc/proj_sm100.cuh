@@ -336,18 +336,20 @@ constexpr int PB_MAX_H = 16;
 constexpr int PB_MAX_CZ = 1024;
 constexpr int PB_ROWS = 128;                   // pair rows per block step
 constexpr int PB_THREADS = 256;
-constexpr int PB_SMEM = PB_MAX_CZ * PB_MAX_H * 4 + PB_MAX_H * PB_ROWS * 2;
+constexpr int PB_SMEM = PB_MAX_CZ * PB_MAX_H * 4 + PB_MAX_H * PB_ROWS * 2;   // w (fp32, heads padded to 4) + outputs
 
-// CPL = 16-byte chunks per lane (chunk c = lane % LPR + LPR * t), LPR = lanes per row.
-template <int CPL, int LPR>
+// CPL = 16-byte chunks per lane (chunk c = lane % LPR + LPR * t), LPR = lanes
+// per row, HQ = heads / 4 rounded up (the head loops are unrolled exactly).
+template <int CPL, int LPR, int HQ>
 __global__ void __launch_bounds__(PB_THREADS) pair_bias_kernel(const PbParams p) {
+    constexpr int HP = 4 * HQ;
     extern __shared__ float pb_smem[];
-    const int H = p.H, HP = (H + 3) & ~3, HQ = HP / 4;
+    const int H = p.H;
     const int ch = p.c_z / 8;
     // w[k][h] at ((k % 8) * ch + k / 8) * HP + h: for a fixed k % 8 the lanes of a
     // row, which hold consecutive chunks k / 8, read consecutive 16-byte words
     float* wsh = pb_smem;
-    __nv_bfloat16* osh = reinterpret_cast<__nv_bfloat16*>(pb_smem + p.c_z * HP);   // [H][PB_ROWS]
+    __nv_bfloat16* osh = reinterpret_cast<__nv_bfloat16*>(pb_smem + p.c_z * HP);   // [HP][PB_ROWS]
     for (int o = threadIdx.x; o < p.c_z * HP; o += PB_THREADS) {
         const int k = o / HP, h = o - k * HP;
         wsh[((k & 7) * ch + (k >> 3)) * HP + h] = h < H ? __bfloat162float(p.w[k * H + h]) : 0.f;
@@ -371,9 +373,9 @@ __global__ void __launch_bounds__(PB_THREADS) pair_bias_kernel(const PbParams p)
             gw[t * 8 + e] = (c < ch && p.ln_w) ? __ldg(p.ln_w + k) : 1.f;
             gb[t * 8 + e] = (c < ch && p.ln_b) ? __ldg(p.ln_b + k) : 0.f;
         }
-    float bh[PB_MAX_H];
+    float bh[HP];
 #pragma unroll
-    for (int h = 0; h < PB_MAX_H; ++h) bh[h] = (h < H && p.bias) ? __ldg(p.bias + h) : 0.f;
+    for (int h = 0; h < HP; ++h) bh[h] = (h < H && p.bias) ? __ldg(p.bias + h) : 0.f;
     __syncthreads();
     for (int64_t r0 = (int64_t)blockIdx.x * PB_ROWS; r0 < total; r0 += (int64_t)gridDim.x * PB_ROWS) {
 #pragma unroll 1
@@ -410,9 +412,9 @@ __global__ void __launch_bounds__(PB_THREADS) pair_bias_kernel(const PbParams p)
 #pragma unroll
                 for (int o = LPR / 2; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
                 const float rstd = rsqrtf(sq * inv_c + p.eps);
-                float acc[PB_MAX_H];
+                float acc[HP];
 #pragma unroll
-                for (int h = 0; h < PB_MAX_H; ++h) acc[h] = 0.f;
+                for (int h = 0; h < HP; ++h) acc[h] = 0.f;
 #pragma unroll
                 for (int t = 0; t < CPL; ++t) {
                     const int c = cl + LPR * t;
@@ -422,27 +424,24 @@ __global__ void __launch_bounds__(PB_THREADS) pair_bias_kernel(const PbParams p)
                             const float nv = fmaf((f[8 * t + e] - mean) * rstd, gw[8 * t + e], gb[8 * t + e]);
                             const float4* w4 = reinterpret_cast<const float4*>(wsh + (e * ch + c) * HP);
 #pragma unroll
-                            for (int hq = 0; hq < PB_MAX_H / 4; ++hq)
-                                if (hq < HQ) {
-                                    const float4 wv = w4[hq];
-                                    acc[4 * hq] = fmaf(nv, wv.x, acc[4 * hq]);
-                                    acc[4 * hq + 1] = fmaf(nv, wv.y, acc[4 * hq + 1]);
-                                    acc[4 * hq + 2] = fmaf(nv, wv.z, acc[4 * hq + 2]);
-                                    acc[4 * hq + 3] = fmaf(nv, wv.w, acc[4 * hq + 3]);
-                                }
+                            for (int hq = 0; hq < HQ; ++hq) {
+                                const float4 wv = w4[hq];
+                                acc[4 * hq] = fmaf(nv, wv.x, acc[4 * hq]);
+                                acc[4 * hq + 1] = fmaf(nv, wv.y, acc[4 * hq + 1]);
+                                acc[4 * hq + 2] = fmaf(nv, wv.z, acc[4 * hq + 2]);
+                                acc[4 * hq + 3] = fmaf(nv, wv.w, acc[4 * hq + 3]);
+                            }
                         }
                     }
                 }
 #pragma unroll
-                for (int h = 0; h < PB_MAX_H; ++h)
-                    if (h < H) {
+                for (int h = 0; h < HP; ++h) {
 #pragma unroll
-                        for (int o = LPR / 2; o >= 1; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-                    }
+                    for (int o = LPR / 2; o >= 1; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+                }
                 if (cl == 0) {
 #pragma unroll
-                    for (int h = 0; h < PB_MAX_H; ++h)
-                        if (h < H) osh[h * PB_ROWS + rloc] = __float2bfloat16_rn(acc[h] + bh[h]);
+                    for (int h = 0; h < HP; ++h) osh[h * PB_ROWS + rloc] = __float2bfloat16_rn(acc[h] + bh[h]);
                 }
             }
         }

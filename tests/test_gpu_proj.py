@@ -136,3 +136,18 @@ def test_unsupported_projection_shapes_raise():
     with pytest.raises(A.EvoError) as e:
         A.ln_linear(x, None, None, EPS, wt)
     assert e.value.code == 2                               # c_in not a multiple of 64
+
+
+@pytest.mark.parametrize("c_z,H,N,B", [(8, 1, 24, 2), (40, 2, 17, 1), (136, 3, 33, 1), (264, 6, 20, 1),
+                                       (520, 13, 12, 1), (1024, 16, 9, 2)])
+def test_pair_bias_projection_shapes(c_z, H, N, B):
+    # every lane layout (2..32 lanes per row, 1..4 chunks per lane) and head-group count
+    g = torch.Generator("cpu").manual_seed(c_z * 31 + H)
+    z = torch.randn((B, N, N, c_z), generator=g).to(torch.bfloat16).cuda()
+    wb = (torch.randn((c_z, H), generator=g) / c_z ** 0.5).to(torch.bfloat16).cuda()
+    ln_w = (1 + 0.1 * torch.randn(c_z, generator=g)).cuda()
+    ln_b = (0.1 * torch.randn(c_z, generator=g)).cuda()
+    bias = torch.randn(H, generator=g).cuda()
+    pb = A.ln_pair_bias(z, ln_w, ln_b, EPS, wb, bias)
+    y = oracle.ln_linear(f64(z), f64(ln_w), f64(ln_b), EPS, f64(wb), f64(bias))
+    check(pb, np.transpose(y, (0, 3, 1, 2))[:, None], ("pair_bias", c_z, H))
