@@ -218,22 +218,30 @@ evo_status_t bwd_f32(const evo_shape_t& sh, evo::simt::Args a, cudaStream_t stre
 }
 
 // ---------------------------------------------------------------- fused pre-attention projection
-// maps[0]: w [c_in, n_out], boxes of 64 columns x c_in rows; maps[1]: y [rows, n_out] (pitch ldy),
-// boxes of 64 columns x 32 rows.  Persistent grid: n_slices x (CTAs per slice), at most one per SM.
+// maps[0]: w [c_in, n_out], boxes of 64 columns x 64 rows; maps[1]: y [rows, n_out] (pitch ldy),
+// boxes of 64 columns x 32 rows.  Persistent grid: n_groups x (CTAs per group), at most one per SM.
 template <int BNO, int CIN>
 evo_status_t launch_ln_linear(const CUtensorMap* maps, const evo::proj::LnParams& p, cudaStream_t stream) {
     using L = evo::proj::PLayout<BNO, CIN>;
     auto kern = evo::proj::ln_linear_kernel<BNO, CIN>;
     static cudaError_t attr = set_smem(kern, L::bytes);
     if (attr != cudaSuccess) return EVO_ERR_CUDA;
-    const int64_t nsl = p.n_out / BNO;
     const int64_t nrb = (p.rows + evo::proj::BM - 1) / evo::proj::BM;
-    const int64_t per_slice = std::min<int64_t>(nrb, std::max<int64_t>(1, sm_count() / nsl));
-    const int64_t grid = nsl * per_slice;
+    // the widest column group whose w chunks stay resident; else all columns in one group
+    const int nsl = p.n_out / BNO, kc = CIN / evo::proj::KBOX;
+    int gsl = nsl;
+    if (nsl * kc > L::NW) {
+        for (int g = nsl; g >= 1; --g)
+            if (nsl % g == 0 && g * kc <= L::NW) { gsl = g; break; }
+    }
+    evo::proj::LnParams q = p;
+    q.gsl = gsl;
+    const int64_t ngr = nsl / gsl;
+    const int64_t grid = ngr * std::min<int64_t>(nrb, std::max<int64_t>(1, sm_count() / ngr));
     if (grid > 0x7fffffff) return EVO_ERR_UNSUPPORTED;
     {
         evo::timing::Scope t(EVO_PHASE_PROJ, stream);
-        kern<<<(unsigned)grid, evo::proj::THREADS, L::bytes, stream>>>(maps[0], maps[1], p);
+        kern<<<(unsigned)grid, evo::proj::THREADS, L::bytes, stream>>>(maps[0], maps[1], q);
     }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
@@ -264,6 +272,27 @@ evo_status_t launch_pair_bias(const evo::proj::PbParams& p, int64_t total, cudaS
     {
         evo::timing::Scope t(EVO_PHASE_PAIR_BIAS, stream);
         kern<<<grid, evo::proj::PB_THREADS, shm, stream>>>(p);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+template <int HQ>
+evo_status_t launch_pair_bias_rows(const evo::proj::PbParams& p, int64_t total, cudaStream_t stream) {
+    auto kern = evo::proj::pair_bias_rows_kernel<HQ>;
+    static cudaError_t attr = set_smem(kern, evo::proj::PBR_SMEM);
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    const int64_t ch = p.c_z / 8;
+    const size_t shm = (size_t)evo::proj::PBR_THREADS * (ch | 1) * 16 + (size_t)p.c_z * 4 * HQ * 4 +
+                       (size_t)(1 + evo::proj::PBR_THREADS / 32) * 4 * HQ * 4;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, evo::proj::PBR_THREADS, shm) != cudaSuccess)
+        return EVO_ERR_CUDA;
+    const int64_t blocks = (total + evo::proj::PBR_THREADS - 1) / evo::proj::PBR_THREADS;
+    const int grid = (int)std::min<int64_t>(blocks, (int64_t)sm_count() * std::max(per_sm, 1));
+    {
+        evo::timing::Scope t(EVO_PHASE_PAIR_BIAS, stream);
+        kern<<<grid, evo::proj::PBR_THREADS, shm, stream>>>(p);
     }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
@@ -438,11 +467,12 @@ evo_status_t evo_ln_linear(int64_t rows, int64_t c_in, int64_t n_out, const void
     if (rows > (int64_t)0x7fffffff - evo::proj::BM || n_out > (int64_t)0x7fffffff) return EVO_ERR_UNSUPPORTED;
     for (const void* q : {x, w, (const void*)y})
         if (!aligned(q, 16)) return EVO_ERR_UNSUPPORTED;
-    for (const void* q : {(const void*)ln_w, (const void*)ln_b, (const void*)bias})
+    if (bias && !aligned(bias, 16)) return EVO_ERR_UNSUPPORTED;      // read as float4
+    for (const void* q : {(const void*)ln_w, (const void*)ln_b})
         if (q && !aligned(q, 4)) return EVO_ERR_INVALID_ARG;
     CUtensorMap maps[2];
     std::memset(maps, 0, sizeof(maps));
-    if (!evo::tma::matrix_bf16(&maps[0], w, c_in, n_out, n_out, (uint32_t)c_in) ||
+    if (!evo::tma::matrix_bf16(&maps[0], w, c_in, n_out, n_out, 64) ||
         !evo::tma::matrix_bf16(&maps[1], y, rows, n_out, ldy, 32))
         return EVO_ERR_CUDA;
     evo::proj::LnParams p{};
@@ -468,6 +498,14 @@ evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, cons
     const int64_t total = B * N * N;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t chunks = c_z / 8;
+    if (c_z <= evo::proj::PBR_MAX_CZ) {
+        switch ((H + 3) / 4) {
+            case 1: return launch_pair_bias_rows<1>(p, total, s);
+            case 2: return launch_pair_bias_rows<2>(p, total, s);
+            case 3: return launch_pair_bias_rows<3>(p, total, s);
+            default: return launch_pair_bias_rows<4>(p, total, s);
+        }
+    }
     if (chunks > 64) return launch_pair_bias_h<4, 32>(p, total, s);
     if (chunks > 32) return launch_pair_bias_h<2, 32>(p, total, s);
     if (chunks > 16) return launch_pair_bias_h<1, 32>(p, total, s);

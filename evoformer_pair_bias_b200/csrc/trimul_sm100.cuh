@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint32_t v[64];
                 tmem_ld32x2_sync(taddr + 64 * g, taddr + 64 * g + 32, v);
                 const uint32_t sb = stg + (uint32_t)((g & 1) * STG_TILE);
-                if (lane == 0) bulk_wait_read<1>();
+                if (lane == 0) bulk_wait_read<1>();      // the store that last read this buffer is done with it
                 __syncwarp();
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -211,8 +211,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0 && row0 < p.N && j0 + 64 * g < p.N) {   // partial boxes are clipped
-                    tma_store_3d(&tm_z, sb, j0 + 64 * g, row0, bc);
+                // partial boxes are clipped; a box wholly past N is not stored, but its
+                // group is still committed: "every group but the newest is done" must
+                // keep meaning "the store that last read the other buffer is done"
+                if (lane == 0) {
+                    if (row0 < p.N && j0 + 64 * g < p.N) tma_store_3d(&tm_z, sb, j0 + 64 * g, row0, bc);
                     bulk_commit();
                 }
             }

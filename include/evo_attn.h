@@ -194,7 +194,7 @@ evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype,
  * q, k, v and g of the attention, as [B, S, N, H, c] views with row stride
  * 4*H*c that evo_attn_fwd / evo_attn_bwd take through their strides.
  * Supported: c_in a multiple of 64 up to 256, n_out a multiple of 128, ldy a
- * multiple of 8, x / w / y 16-byte aligned (else EVO_ERR_UNSUPPORTED); rows
+ * multiple of 8, x / w / y / bias 16-byte aligned (else EVO_ERR_UNSUPPORTED); rows
  * == 0 is a no-op.  Only y[0:rows, 0:n_out] is written (columns n_out..ldy-1
  * keep their contents).  The normalised activations are rounded to bf16
  * before the product, y to bf16 on the store.  Stream-ordered, no

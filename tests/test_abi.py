@@ -95,6 +95,12 @@ def test_projection_host_checks_need_no_gpu(lib):
     assert lib.evo_ln_linear(8, 48, 1024, fake, nul, nul, 1e-5, fake, nul, fake, 1024, nul) == 2  # c_in % 64
     assert lib.evo_ln_linear(8, 320, 1024, fake, nul, nul, 1e-5, fake, nul, fake, 1024, nul) == 2  # c_in > 256
     assert lib.evo_ln_linear(8, 256, 192, fake, nul, nul, 1e-5, fake, nul, fake, 192, nul) == 2   # n_out % 128
+    odd = ctypes.c_void_p((1 << 20) + 4)                  # 4-byte but not 16-byte aligned
+    assert lib.evo_ln_linear(8, 256, 1024, fake, nul, nul, 1e-5, fake, odd, fake, 1024, nul) == 2  # bias
+    assert lib.evo_tri_mul(1, 2, 12, fake, fake, 0, fake, nul) == 2                                # N % 8
+    assert lib.evo_tri_mul(1, 2, 16, fake, odd, 0, fake, nul) == 2                                 # alignment
+    assert lib.evo_tri_mul(1, 0, 16, nul, nul, 0, nul, nul) == 0                                   # empty
+    assert lib.evo_tri_mul(-1, 2, 16, fake, fake, 0, fake, nul) == 1
     assert lib.evo_ln_pair_bias(1, 16, 128, 17, fake, nul, nul, 1e-5, fake, nul, fake, nul) == 2  # H > 16
     assert lib.evo_ln_pair_bias(1, 16, 12, 4, fake, nul, nul, 1e-5, fake, nul, fake, nul) == 2    # c_z % 8
     assert lib.evo_ln_pair_bias(1, 0, 128, 4, nul, nul, nul, 1e-5, nul, nul, nul, nul) == 0       # empty

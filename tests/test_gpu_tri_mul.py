@@ -6,8 +6,8 @@ cannot move", section "The three operations".  The kernel reads channel-first
 [B, C, N, N] bf16; the oracle gets the same rounded values in its [B, N, N, C]
 layout.  Tolerance (tri_mul_bound in the parity helpers, from the
 arithmetic): per element 2^-8 |z| + 2^-12 sum_k |a| |b|, and rel-L2 <= 5e-3.
-Covers both edge directions, several tiles with ragged edges in i, j and k,
-the full-size workloads the benchmark times, and the degenerate sizes.
+Covers both edge directions, one and several tiles per CTA, ragged edges in
+i, j and k, the full-size workload, and the degenerate sizes.
 """
 import numpy as np
 import pytest
@@ -52,6 +52,15 @@ def check(w, incoming):
 @pytest.mark.parametrize("N,C,B", [(40, 3, 2), (128, 2, 1), (200, 4, 1), (264, 2, 1), (512, 1, 1)])
 def test_contraction_matches_the_oracle(N, C, B, incoming):
     check(TriMulWorkload("case", B, N, C, 9000 + N + C), incoming)
+
+
+@pytest.mark.parametrize("incoming", [False, True])
+@pytest.mark.parametrize("N,C", [(128, 300), (128, 400), (136, 160), (192, 300), (256, 160)])
+def test_several_tiles_per_cta(N, C, incoming):
+    # enough channels for two or more tiles per SM, so that CTAs run several tiles through
+    # the double-buffered accumulators.  With N not a multiple of 256 some 64-column groups
+    # lie wholly past N and store nothing, between groups that do
+    check(TriMulWorkload("many", 1, N, C, 9100 + N + C), incoming)
 
 
 @pytest.mark.parametrize("incoming", [False, True])
