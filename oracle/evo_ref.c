@@ -42,7 +42,8 @@
  *
  * The file also holds the fused pre-attention projection (LayerNorm + linear,
  * evo_ref_ln_linear below) that produces q, k, v, g and the pair bias, and
- * the contraction of the triangular multiplicative update (evo_ref_tri_mul).
+ * the contraction of the triangular multiplicative update (evo_ref_tri_mul),
+ * and the outer product mean (evo_ref_outer_product_mean).
  *
  * Planted mistakes (mutation testing of the pins): building with
  * -DEVO_REF_MUTANT=n swaps in one deliberate error, see mutant_* below.
@@ -364,6 +365,53 @@ int evo_ref_tri_mul(int64_t B, int64_t N, int64_t C, const double* a, const doub
 #endif
                     for (int64_t c = 0; c < C; ++c) zr[c] += ar[c] * br[c];
                 }
+#endif
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Outer product mean, the bridge from the MSA to the pair representation
+ * ("Evoformer: the memory wall ZeRO cannot move", section "The three
+ * operations"): the outer product of MSA columns i and j averaged over the
+ * S sequences,
+ *
+ *   out[b,i,j,c1,c2] = (1/S) sum_s a[b,s,i,c1] * bb[b,s,j,c2]
+ *
+ * a: [B, S, N, Ca], bb: [B, S, N, Cb], out: [B, N, N, Ca, Cb], contiguous
+ * fp64.  Returns 0, or -1 for a bad size.
+ */
+int evo_ref_outer_product_mean(int64_t B, int64_t S, int64_t N, int64_t Ca, int64_t Cb, const double* a,
+                               const double* bb, double* out) {
+    if (B < 0 || S <= 0 || N < 0 || Ca <= 0 || Cb <= 0) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t i = 0; i < N; ++i) {
+            for (int64_t j = 0; j < N; ++j) {
+                double* o = out + (((b * N + i) * N + j) * Ca) * Cb;
+                for (int64_t e = 0; e < Ca * Cb; ++e) o[e] = 0.0;
+                for (int64_t s = 0; s < S; ++s) {
+                    const double* ar = a + ((b * S + s) * N + i) * Ca;
+                    const double* br = bb + ((b * S + s) * N + j) * Cb;
+                    for (int64_t c1 = 0; c1 < Ca; ++c1)
+                        for (int64_t c2 = 0; c2 < Cb; ++c2) o[c1 * Cb + c2] += ar[c1] * br[c2];
+                }
+#if EVO_REF_MUTANT == 12
+                /* mutant: the sum over sequences, not its mean */
+#else
+                for (int64_t e = 0; e < Ca * Cb; ++e) o[e] /= (double)S;
+#endif
+#if EVO_REF_MUTANT == 13
+                /* mutant: the two channel axes swapped (Ca == Cb only) */
+                if (Ca == Cb)
+                    for (int64_t c1 = 0; c1 < Ca; ++c1)
+                        for (int64_t c2 = c1 + 1; c2 < Cb; ++c2) {
+                            const double t = o[c1 * Cb + c2];
+                            o[c1 * Cb + c2] = o[c2 * Cb + c1];
+                            o[c2 * Cb + c1] = t;
+                        }
 #endif
             }
         }
