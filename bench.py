@@ -30,6 +30,10 @@ contraction of the triangular multiplicative update ("Evoformer: the memory
 wall ZeRO cannot move", section "The three operations"): one step is the
 outgoing-edge update z[b,c,i,j] = sum_k a[b,c,i,k] b[b,c,j,k] over every channel,
 then the incoming-edge one; metric TFLOP/s (2 * B * C * N^3 per direction).
+
+``--workload opm_256 | opm_384`` benchmarks the outer product mean (same
+section): one step is out[b,i,c1,j,c2] = (1/S) sum_s a[b,s,i,c1] b[b,s,j,c2];
+metric TFLOP/s (2 * B * S * (N C)^2).
 """
 from __future__ import annotations
 
@@ -42,6 +46,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -50,11 +55,13 @@ sys.path.insert(0, ROOT)
 from evoformer_pair_bias_b200 import attention as A  # noqa: E402
 from evoformer_pair_bias_b200.workloads import (WORKLOADS, DEFAULT_BENCH, PROJ_WORKLOADS, logical_view,  # noqa: E402
                                                 make_inputs, make_pair_bias_params, make_proj_inputs,
-                                                TRI_MUL_WORKLOADS, make_tri_mul_inputs)
+                                                TRI_MUL_WORKLOADS, make_tri_mul_inputs, OPM_WORKLOADS,
+                                                make_opm_inputs)
 
 METRIC = "Evoformer pair-bias attention fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
 PROJ_METRIC = "fused LayerNorm + linear pre-attention projection TFLOP/s"
 TRI_METRIC = "triangular multiplicative update contraction TFLOP/s"
+OPM_METRIC = "outer product mean TFLOP/s"
 PROJ_EPS = 1e-5
 NOMINAL_BF16_TFLOPS = 2250.0
 
@@ -803,12 +810,195 @@ def run_tri_mul(args, tw, rank, world, local):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# Outer product mean
+
+
+def opm_oracle_sample(ow, target_s: float = 12.0):
+    """Time the fp64 oracle on the first r columns i of the workload (all j), sized for about target_s."""
+    import oracle
+    oracle.build()
+    d = make_opm_inputs(ow)
+    a_all, b = d["a"].double().numpy(), d["b"].double().numpy()
+
+    def run(r):
+        a = np.ascontiguousarray(a_all[:, :, :r])
+        t0 = time.perf_counter()
+        oracle.outer_product_mean(a, b)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    r = max(1, min(ow.N, int(target_s / max(t1, 1e-6) / 2)))
+    t, reps = 0.0, 0
+    while reps == 0 or t < 0.7 * target_s:
+        t += run(r)
+        reps += 1
+    fl = ow.flops * r / ow.N * reps
+    return dict(value=fl / t / 1e12, unit="TFLOP/s", cores=oracle_threads(), kind="oracle",
+                sample=f"{r} of {ow.N} columns i (all j) x{reps}, fp64, {t:.2f} s", seconds=t, rows=r)
+
+
+def run_opm(args, ow, rank, world, local):
+    fl = ow.flops
+    by = 2 * ow.B * ow.S * ow.N * ow.C * 2 + ow.B * (ow.N * ow.C) ** 2 * 2
+    cfg = {"workload": ow.name, "B": ow.B, "N_seq": ow.S, "N_res": ow.N, "C": ow.C,
+           "output": "bf16 [B, N, C, N, C]"}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps, warm = args.steps, args.warmup
+        info = opm_oracle_sample(ow, target_s=max(0.5, 60.0 / max(1, steps + warm)))
+        r = info["rows"]
+        import oracle
+        d = make_opm_inputs(ow)
+        a = np.ascontiguousarray(d["a"].double().numpy()[:, :, :r])
+        b = d["b"].double().numpy()
+        times = []
+        for i in range(warm + steps):
+            t0 = time.perf_counter()
+            oracle.outer_product_mean(a, b)
+            if i >= warm:
+                times.append(time.perf_counter() - t0)
+        t = sum(times)
+        val = fl * r / ow.N * steps / t / 1e12
+        line = {"metric": OPM_METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps,
+                "warmup": warm, "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {**cfg, "sample_columns": r, "l2": "n/a (CPU)"},
+                "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": f"{r} of {ow.N} columns i per step, fp64"},
+                "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import datetime
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    A.load_library()
+    hin = make_opm_inputs(ow)
+    d = {k: v.to(dev) for k, v in hin.items()}
+    out = torch.empty((ow.B, ow.N, ow.C, ow.N, ow.C), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    A.timing_enable(True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        A.outer_product_mean(d["a"], d["b"], out=out)
+    torch.cuda.synchronize()
+    A.timing_collect()
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported an error during warm-up")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with ClockSampler(gpu_uuid(dev)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        n0 = A.launch_count()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record()
+            A.outer_product_mean(d["a"], d["b"], out=out)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        launches = A.launch_count() - n0
+    kt = A.timing_collect()
+    A.timing_enable(False)
+    tot = max_over_ranks([sum(e0.elapsed_time(e1) for e0, e1 in ev)], world, dev)[0]
+    if A.device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported an error during the timed region")
+    value = job_throughput(fl, K, world, tot)
+    pk = peaks()
+    n_l, ms_l = kt["opm"]
+    us = 1e3 * ms_l / max(n_l, 1)
+    sec = us * 1e-6
+    sustained = tot * 1e-3 > 1.0
+    tflops_peak = pk["bf16_sustained"] if sustained else pk["bf16"]
+    t_tensor, t_hbm = fl / (tflops_peak * 1e12), by / (pk["hbm"] * 1e9)
+    common = {"kernel": "trimul::tri_mul_kernel (MN-major, scale 1/S)", "launches": n_l, "us_per_launch": us,
+              "flops_per_launch": fl, "algorithmic_bytes_per_launch": by, "traffic": None,
+              "tensor_floor_us": t_tensor * 1e6, "hbm_floor_us": t_hbm * 1e6}
+    if t_tensor >= t_hbm:
+        a_ = fl / sec / 1e12
+        roof = {"bound": "tensor", "achieved": a_, "peak": tflops_peak, "unit": "TFLOP/s", "frac": a_ / tflops_peak,
+                "peak_source": f"{pk['source']} bf16 {'sustained' if sustained else 'burst'}", **common}
+    else:
+        a_ = by / sec / 1e9
+        roof = {"bound": "hbm", "achieved": a_, "peak": pk["hbm"], "unit": "GB/s", "frac": a_ / pk["hbm"],
+                "peak_source": f"{pk['source']} HBM copy", "tensor_frac": fl / sec / 1e12 / tflops_peak, **common}
+
+    e2e = None
+    if not args.no_e2e:
+        ha, hb = hin["a"].pin_memory(), hin["b"].pin_memory()
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        da, db = torch.empty_like(ha, device=dev), torch.empty_like(hb, device=dev)
+
+        def e2e_step():
+            da.copy_(ha, non_blocking=True)
+            db.copy_(hb, non_blocking=True)
+            A.outer_product_mean(da, db, out=out)
+            ho.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        et = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+        e2e = {"value": job_throughput(fl, K, world, et), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 2 * ha.numel() * ha.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": et / K}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            cpu = opm_oracle_sample(ow)
+            cpu.pop("seconds", None)
+            cpu.pop("rows", None)
+        except Exception as exc:  # the baseline is reported, never required
+            cpu = {"error": repr(exc)}
+
+    if rank == 0:
+        line = {
+            "metric": OPM_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": tot / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**cfg, "l2": "flushed (256 MB write) before every step",
+                       "parallelism": f"replicas x{world}, batches independent, no collective"},
+            "roofline": roof,
+            "kernels": {"opm": {"launches": n_l, "us_per_launch": us}},
+            "frac_measured_peak": value / world / pk["bf16"],
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS) + sorted(PROJ_WORKLOADS) + sorted(TRI_MUL_WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS) + sorted(PROJ_WORKLOADS) + sorted(TRI_MUL_WORKLOADS) + sorted(OPM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -822,6 +1012,8 @@ def main():
         return run_projection(args, PROJ_WORKLOADS[args.workload], rank, world, local)
     if args.workload in TRI_MUL_WORKLOADS:
         return run_tri_mul(args, TRI_MUL_WORKLOADS[args.workload], rank, world, local)
+    if args.workload in OPM_WORKLOADS:
+        return run_opm(args, OPM_WORKLOADS[args.workload], rank, world, local)
     w = WORKLOADS[args.workload]
 
     if args.impl == "reference":

@@ -34,7 +34,7 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
            "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc",
            "evo_attn_timing_enable", "evo_attn_timing_collect", "evo_ln_linear", "evo_ln_pair_bias",
-           "evo_tri_mul")
+           "evo_tri_mul", "evo_outer_product_mean")
 
 #: Size of the library's fixed scratch area used by evo_attn_bwd_noalloc (bytes).
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -55,7 +55,7 @@ class Strides(ctypes.Structure):
 
 
 #: Timing phases (evo_timing_t indices).
-PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj", "pair_bias", "tri_mul")
+PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj", "pair_bias", "tri_mul", "opm")
 
 
 class Timing(ctypes.Structure):
@@ -101,6 +101,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_ln_pair_bias.restype = ctypes.c_int
     lib.evo_tri_mul.argtypes = [i64, i64, i64, vp, vp, ctypes.c_int, vp, vp]
     lib.evo_tri_mul.restype = ctypes.c_int
+    lib.evo_outer_product_mean.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, vp]
+    lib.evo_outer_product_mean.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -313,6 +315,30 @@ def tri_mul(a, b, incoming: bool = False, z=None):
     rc = lib.evo_tri_mul(B, C, N, _ptr(ac), _ptr(bc), 1 if incoming else 0, _ptr(z), _stream(a.device))
     _check("evo_tri_mul", rc)
     return z
+
+
+def outer_product_mean(a, b, out=None):
+    """Outer product mean: out[b, i, c1, j, c2] = (1/S) sum_s a[b, s, i, c1] b[b, s, j, c2].
+
+    a: bf16 [B, S, N, Ca], b: bf16 [B, S, N, Cb].  Returns bf16 [B, N, Ca, N, Cb];
+    opm_pair_view(out) is the same data as the pair layout [B, N, N, Ca, Cb].
+    """
+    lib = load_library()
+    if a.dim() != 4 or b.dim() != 4 or a.shape[:3] != b.shape[:3]:
+        raise ValueError("a and b must be [B, S, N, C] with the same B, S, N")
+    B, S, N, Ca = a.shape
+    Cb = b.shape[3]
+    ac, bc = a.contiguous(), b.contiguous()
+    if out is None:
+        out = torch.empty((B, N, Ca, N, Cb), dtype=torch.bfloat16, device=a.device)
+    rc = lib.evo_outer_product_mean(B, S, N, Ca, Cb, _ptr(ac), _ptr(bc), _ptr(out), _stream(a.device))
+    _check("evo_outer_product_mean", rc)
+    return out
+
+
+def opm_pair_view(out):
+    """[B, N, Ca, N, Cb] outer-product-mean output as the pair layout [B, N, N, Ca, Cb] (a view)."""
+    return out.permute(0, 1, 3, 2, 4)
 
 
 def timing_enable(on: bool = True) -> None:

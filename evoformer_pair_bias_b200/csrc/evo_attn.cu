@@ -309,6 +309,33 @@ evo_status_t launch_pair_bias_h(const evo::proj::PbParams& p, int64_t total, cud
     return EVO_ERR_UNSUPPORTED;
 }
 
+// z[m] (M x Nc) = scale * a[m]^T b[m] (incoming: a, b are K x M, K x Nc) or a[m] b[m]^T
+// (outgoing: a, b are M x K, Nc x K) for the `batch` matrices m, on the tri_mul kernel.
+evo_status_t launch_contraction(const void* a, const void* bb, void* z, int64_t M, int64_t Nc, int64_t K,
+                                int64_t batch, bool incoming, float scale, int phase, cudaStream_t stream) {
+    using namespace evo::trimul;
+    CUtensorMap maps[3];
+    std::memset(maps, 0, sizeof(maps));
+    const bool ok = incoming ? (evo::tma::batch_bf16(&maps[0], a, M, K, batch, 64, 64) &&
+                                evo::tma::batch_bf16(&maps[1], bb, Nc, K, batch, 64, 64))
+                             : (evo::tma::batch_bf16(&maps[0], a, K, M, batch, 64, BM) &&
+                                evo::tma::batch_bf16(&maps[1], bb, K, Nc, batch, 64, BN));
+    if (!ok || !evo::tma::batch_bf16(&maps[2], z, Nc, M, batch, 64, 32)) return EVO_ERR_CUDA;
+    TriParams p{};
+    p.M = (int)M; p.Nc = (int)Nc; p.K = (int)K; p.BC = (int)batch; p.incoming = incoming ? 1 : 0; p.scale = scale;
+    p.tiles_i = (int)((M + BM - 1) / BM); p.tiles_j = (int)((Nc + BN - 1) / BN);
+    const int64_t tiles = batch * p.tiles_i * p.tiles_j;
+    static cudaError_t attr = set_smem(tri_mul_kernel, TLayout::bytes);
+    if (attr != cudaSuccess) return EVO_ERR_CUDA;
+    const int grid = (int)std::min<int64_t>(tiles, sm_count());
+    {
+        evo::timing::Scope t(phase, stream);
+        tri_mul_kernel<<<grid, THREADS, TLayout::bytes, stream>>>(maps[0], maps[1], maps[2], p);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -524,28 +551,24 @@ evo_status_t evo_tri_mul(int64_t B, int64_t C, int64_t N, const void* a, const v
     if (N % 8 != 0 || BC > (int64_t)0x7fffffff || N > (int64_t)0x7fffffff / 2) return EVO_ERR_UNSUPPORTED;
     for (const void* q : {a, bb, (const void*)z})
         if (!aligned(q, 16)) return EVO_ERR_UNSUPPORTED;
-    using namespace evo::trimul;
-    CUtensorMap maps[3];
-    std::memset(maps, 0, sizeof(maps));
     const bool in = incoming != 0;
-    if (!evo::tma::stack_bf16(&maps[0], a, N, BC, 64, in ? 64 : BM) ||
-        !evo::tma::stack_bf16(&maps[1], bb, N, BC, 64, in ? 64 : BN) ||
-        !evo::tma::stack_bf16(&maps[2], z, N, BC, 64, 32))
-        return EVO_ERR_CUDA;
-    TriParams p{};
-    p.N = (int)N; p.BC = (int)BC; p.incoming = in ? 1 : 0;
-    p.tiles_i = (int)((N + BM - 1) / BM); p.tiles_j = (int)((N + BN - 1) / BN);
-    const int64_t tiles = BC * p.tiles_i * p.tiles_j;
-    static cudaError_t attr = set_smem(tri_mul_kernel, TLayout::bytes);
-    if (attr != cudaSuccess) return EVO_ERR_CUDA;
-    const int grid = (int)std::min<int64_t>(tiles, sm_count());
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    {
-        evo::timing::Scope t(EVO_PHASE_TRI_MUL, s);
-        tri_mul_kernel<<<grid, THREADS, TLayout::bytes, s>>>(maps[0], maps[1], maps[2], p);
-    }
-    g_launches += 1;
-    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+    return launch_contraction(a, bb, z, N, N, N, BC, in, 1.f, EVO_PHASE_TRI_MUL, static_cast<cudaStream_t>(stream));
+}
+
+evo_status_t evo_outer_product_mean(int64_t B, int64_t S, int64_t N, int64_t Ca, int64_t Cb, const void* a,
+                                    const void* bb, void* out, void* stream) {
+    if (B < 0 || S < 0 || N < 0 || Ca <= 0 || Cb <= 0) return EVO_ERR_INVALID_ARG;
+    if (B == 0 || N == 0) return EVO_OK;
+    if (S == 0 || !a || !bb || !out) return EVO_ERR_INVALID_ARG;
+    const int64_t M = N * Ca, Nc = N * Cb;
+    if (M % 8 != 0 || Nc % 8 != 0 || M > (int64_t)0x7fffffff / 2 || Nc > (int64_t)0x7fffffff / 2 ||
+        S > (int64_t)0x7fffffff || B > (int64_t)0x7fffffff)
+        return EVO_ERR_UNSUPPORTED;
+    for (const void* q : {a, bb, (const void*)out})
+        if (!aligned(q, 16)) return EVO_ERR_UNSUPPORTED;
+    // out[b, (i, c1), (j, c2)] = (1/S) sum_s a[b, s, (i, c1)] bb[b, s, (j, c2)]: the MN-major contraction
+    return launch_contraction(a, bb, out, M, Nc, S, B, true, (float)(1.0 / (double)S), EVO_PHASE_OPM,
+                              static_cast<cudaStream_t>(stream));
 }
 
 evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,

@@ -115,11 +115,12 @@ inline bool matrix_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t c
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// A stack of BC contiguous N x N bf16 matrices [BC][N][N] (rows of N elements),
+// A stack of `batch` contiguous rows x cols bf16 matrices [batch][rows][cols],
 // boxes of box0 (<= 64, one 128-byte swizzle span) x box1 rows of one matrix.
-inline bool stack_bf16(CUtensorMap* m, const void* ptr, int64_t N, int64_t BC, uint32_t box0, uint32_t box1) {
-    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)BC};
-    const uint64_t str[2] = {(uint64_t)N * 2, (uint64_t)N * N * 2};
+inline bool batch_bf16(CUtensorMap* m, const void* ptr, int64_t cols, int64_t rows, int64_t batch, uint32_t box0,
+                       uint32_t box1) {
+    const uint64_t dims[3] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)batch};
+    const uint64_t str[2] = {(uint64_t)cols * 2, (uint64_t)rows * cols * 2};
     const uint32_t box[3] = {box0, box1, 1};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }

@@ -7,7 +7,10 @@
 //   incoming edges:  z[b, c, i, j] = sum_k a[b, c, k, i] * bb[b, c, k, j]
 //
 // i.e. one N x N x N matrix product per (batch, channel): a dense contraction
-// for the tensor cores.  The operands are channel-first [B, C, N, N] bf16
+// for the tensor cores.  The kernel takes rectangular products (z is M x Nc,
+// the sum runs over K) and a scale on z, which the outer product mean uses:
+// out[(i, c1), (j, c2)] = (1/S) sum_s a[s, (i, c1)] b[s, (j, c2)] is the
+// MN-major form with M = N Ca, Nc = N Cb, K = S.  The operands are channel-first [B, C, N, N] bf16
 // (the per-channel matrices contiguous); outgoing reads both operands
 // K-major (k contiguous), incoming reads the same layout MN-major (i or j
 // contiguous), so neither direction needs a transposed copy.  fp32
@@ -20,9 +23,10 @@
 //              accumulator t % 2 of its t-th tile;
 //   warps 2-5  epilogue: TMEM -> bf16 -> shared staging (128B swizzle) ->
 //              TMA store, 32 rows x 64 columns per store.
-// Tiles (b, c, 128-row block of i, 256-column block of j) go round-robin to
-// the CTAs.  3D tensor maps (inner, N, B*C) zero-fill rows and k past N, so
-// a ragged N never reads the next channel.  Every wait is bounded.
+// Tiles (matrix, 128-row block of i, 256-column block of j) go round-robin
+// to the CTAs.  3D tensor maps (inner, rows, matrices) zero-fill rows and k
+// past the ends, so a ragged size never reads the next matrix.  Every wait is
+// bounded.
 #pragma once
 
 #include "sm100.cuh"
@@ -56,9 +60,10 @@ struct TLayout {
 };
 
 struct TriParams {
-    int N;
-    int BC;             // B * C (independent matrices)
-    int incoming;       // 0: outgoing edges, 1: incoming edges
+    int M, Nc, K;       // z is M x Nc per matrix, the contraction runs over K
+    int BC;             // independent matrices (B * C for the triangular update)
+    int incoming;       // 0: a[i][k], b[j][k] (K-major); 1: a[k][i], b[k][j] (MN-major)
+    float scale;        // z is multiplied by it before the bf16 rounding
     int tiles_i, tiles_j;
 };
 
@@ -75,7 +80,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int per_mat = p.tiles_i * p.tiles_j;
     const int64_t n_tiles = (int64_t)p.BC * per_mat;
-    const int nk = (p.N + BK - 1) / BK;
+    const int nk = (p.K + BK - 1) / BK;
     auto bar_full = [&](int s) { return base + L::bar_off + 8u * s; };
     auto bar_empty = [&](int s) { return base + L::bar_off + 8u * (STAGES + s); };
     auto bar_accf = [&](int b) { return base + L::bar_off + 8u * (2 * STAGES + b); };
@@ -197,6 +202,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int g = 0; g < BN / 64; ++g) {
                 uint32_t v[64];
                 tmem_ld32x2_sync(taddr + 64 * g, taddr + 64 * g + 32, v);
+                if (p.scale != 1.f) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * p.scale);
+                }
                 const uint32_t sb = stg + (uint32_t)((g & 1) * STG_TILE);
                 if (lane == 0) bulk_wait_read<1>();      // the store that last read this buffer is done with it
                 __syncwarp();
@@ -211,11 +220,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                // partial boxes are clipped; a box wholly past N is not stored, but its
+                // partial boxes are clipped; a box wholly outside z is not stored, but its
                 // group is still committed: "every group but the newest is done" must
                 // keep meaning "the store that last read the other buffer is done"
                 if (lane == 0) {
-                    if (row0 < p.N && j0 + 64 * g < p.N) tma_store_3d(&tm_z, sb, j0 + 64 * g, row0, bc);
+                    if (row0 < p.M && j0 + 64 * g < p.Nc) tma_store_3d(&tm_z, sb, j0 + 64 * g, row0, bc);
                     bulk_commit();
                 }
             }

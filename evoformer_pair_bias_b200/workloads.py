@@ -188,7 +188,8 @@ def ceil_div(a: int, b: int) -> int:
 __all__ = ["Workload", "WORKLOADS", "DEFAULT_BENCH", "MASK_VALUE", "make_inputs",
            "logical_view", "storage_empty", "sample_rows", "logits_bytes", "pair_rep_bytes",
            "mask_columns", "ceil_div", "ProjWorkload", "PROJ_WORKLOADS", "make_proj_inputs",
-           "make_pair_bias_params", "TriMulWorkload", "TRI_MUL_WORKLOADS", "make_tri_mul_inputs"]
+           "make_pair_bias_params", "TriMulWorkload", "TRI_MUL_WORKLOADS", "make_tri_mul_inputs",
+           "OpmWorkload", "OPM_WORKLOADS", "make_opm_inputs"]
 
 
 # ---------------------------------------------------------------------------
@@ -298,4 +299,42 @@ def make_tri_mul_inputs(w: TriMulWorkload, device="cpu") -> dict:
     s = w.N ** -0.25
     a = torch.randn((w.B, w.C, w.N, w.N), generator=g) * s
     b = torch.randn((w.B, w.C, w.N, w.N), generator=g) * s
+    return {"a": a.to(torch.bfloat16).to(device), "b": b.to(torch.bfloat16).to(device)}
+
+
+# ---------------------------------------------------------------------------
+# Outer product mean: seeded inputs only.
+#
+# Recipe (generator seeded with ``seed``): a then b ~ N(0, 1) drawn as
+# [B, S, N, C] (the MSA representation's layout), rounded to bf16.  Shapes:
+# an MSA of S sequences over N residues projected to C = 32 channels, the
+# width of the outer product mean in AlphaFold2-style trunks.
+
+
+@dataclasses.dataclass(frozen=True)
+class OpmWorkload:
+    name: str
+    B: int
+    S: int
+    N: int
+    C: int
+    seed: int
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.B * self.S * (self.N * self.C) ** 2
+
+
+OPM_WORKLOADS = {
+    "opm_256": OpmWorkload("opm_256", 1, 128, 256, 32, 20291),
+    "opm_384": OpmWorkload("opm_384", 1, 512, 384, 32, 20292),
+    "opm_tiny": OpmWorkload("opm_tiny", 2, 5, 12, 8, 20293),
+}
+
+
+def make_opm_inputs(w: OpmWorkload, device="cpu") -> dict:
+    """a, b: bf16 [B, S, N, C]."""
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    a = torch.randn((w.B, w.S, w.N, w.C), generator=g)
+    b = torch.randn((w.B, w.S, w.N, w.C), generator=g)
     return {"a": a.to(torch.bfloat16).to(device), "b": b.to(torch.bfloat16).to(device)}

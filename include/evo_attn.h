@@ -237,6 +237,28 @@ evo_status_t evo_ln_pair_bias(int64_t B, int64_t N, int64_t c_z, int64_t H, cons
 evo_status_t evo_tri_mul(int64_t B, int64_t C, int64_t N, const void* a, const void* bb, int incoming,
                          void* z, void* stream);
 
+/*
+ * Outer product mean, the bridge from the MSA to the pair representation
+ * ("Evoformer: the memory wall ZeRO cannot move", section "The three
+ * operations"): the outer product of MSA columns i and j averaged over the S
+ * sequences,
+ *
+ *   out[b, i, c1, j, c2] = (1/S) sum_s a[b, s, i, c1] * bb[b, s, j, c2]
+ *
+ * a: bf16 [B, S, N, Ca], bb: bf16 [B, S, N, Cb], both contiguous (the MSA
+ * representation's layout); out: bf16 [B, N, Ca, N, Cb] contiguous, i.e. for
+ * each b the (N Ca) x (N Cb) matrix a^T bb / S -- the pair layout
+ * [B, N, N, Ca, Cb] is its view with axes 2 and 3 swapped.  Products
+ * accumulate in fp32 on the tensor cores; the 1/S scale is applied in fp32
+ * before the bf16 rounding.  Supported: N*Ca and N*Cb multiples of 8,
+ * pointers 16-byte aligned, sizes below 2^31 (else EVO_ERR_UNSUPPORTED);
+ * B or N == 0 is a no-op; S == 0 is EVO_ERR_INVALID_ARG (no mean).
+ * Stream-ordered, no allocation, no synchronisation; the kernel's waits are
+ * bounded, and one that gives up is reported by evo_attn_device_status.
+ */
+evo_status_t evo_outer_product_mean(int64_t B, int64_t S, int64_t N, int64_t Ca, int64_t Cb, const void* a,
+                                    const void* bb, void* out, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* evo_status_string(evo_status_t status);
 
@@ -257,7 +279,8 @@ uint64_t evo_attn_launch_count(void);
 
 /*
  * Per-kernel device timing (off by default).  While switched on, each
- * evo_attn_fwd / evo_attn_bwd / evo_ln_linear / evo_ln_pair_bias / evo_tri_mul call records
+ * evo_attn_fwd / evo_attn_bwd / evo_ln_linear / evo_ln_pair_bias / evo_tri_mul /
+ * evo_outer_product_mean call records
  * a pair of CUDA events on its own `stream` around its main kernel, and
  * evo_attn_bwd a second pair around all of its kernels, so that a caller can
  * see how a step's device time splits between the kernels without a
@@ -273,14 +296,15 @@ uint64_t evo_attn_launch_count(void);
  * read (that phase is then left out of the sums).  Both functions are safe to
  * call from several host threads.
  */
-#define EVO_TIMING_PHASES 6
+#define EVO_TIMING_PHASES 7
 enum {
     EVO_PHASE_FWD_MAIN = 0,   /* the forward kernel                         */
     EVO_PHASE_BWD_MAIN = 1,   /* the backward's main (tensor-core) kernel    */
     EVO_PHASE_BWD_ALL = 2,    /* every kernel and memset of one evo_attn_bwd */
     EVO_PHASE_PROJ = 3,       /* the evo_ln_linear kernel                    */
     EVO_PHASE_PAIR_BIAS = 4,  /* the evo_ln_pair_bias kernel                 */
-    EVO_PHASE_TRI_MUL = 5     /* the evo_tri_mul kernel                      */
+    EVO_PHASE_TRI_MUL = 5,    /* the evo_tri_mul kernel                      */
+    EVO_PHASE_OPM = 6         /* the evo_outer_product_mean kernel           */
 };
 typedef struct {
     uint64_t calls[EVO_TIMING_PHASES];

@@ -95,7 +95,7 @@ def _lib(mutant: int = 0) -> ctypes.CDLL:
         lib.evo_ref_ln_linear.restype = ctypes.c_int
         lib.evo_ref_tri_mul.argtypes = [ctypes.c_int64] * 3 + [p] * 2 + [ctypes.c_int, p]
         lib.evo_ref_tri_mul.restype = ctypes.c_int
-        lib.evo_ref_outer_product_mean.argtypes = [ctypes.c_int64] * 5 + [p] * 3
+        lib.evo_ref_outer_product_mean.argtypes = [ctypes.c_int64] * 6 + [p] * 3
         lib.evo_ref_outer_product_mean.restype = ctypes.c_int
         _LIBS[mutant] = lib
     return _LIBS[mutant]
@@ -224,18 +224,19 @@ def tri_mul(a, b, incoming: bool = False, *, mutant: int = 0):
 def outer_product_mean(a, b, *, mutant: int = 0):
     """The outer product mean in fp64: out[b, i, j, c1, c2] = (1/S) sum_s a[b, s, i, c1] b[b, s, j, c2].
 
-    a: [B, S, N, Ca], b: [B, S, N, Cb] (the MSA representation's layout); returns
-    [B, N, N, Ca, Cb] ("Evoformer: the memory wall ZeRO cannot move", section
+    a: [B, S, Na, Ca], b: [B, S, Nb, Cb] (the MSA representation's layout; Na = Nb
+    = N for the full operation, Na < N for a subset of columns i); returns
+    [B, Na, Nb, Ca, Cb] ("Evoformer: the memory wall ZeRO cannot move", section
     "The three operations": the outer product of MSA columns i and j averaged
     over the sequences).
     """
     a, b = _f64(a), _f64(b)
-    if a.ndim != 4 or b.ndim != 4 or a.shape[:3] != b.shape[:3]:
-        raise ValueError(f"a {a.shape} and b {b.shape} must be [B, S, N, C] with the same B, S, N")
-    B, S, N, Ca = a.shape
-    Cb = b.shape[3]
-    out = np.empty((B, N, N, Ca, Cb), np.float64)
-    rc = _lib(mutant).evo_ref_outer_product_mean(B, S, N, Ca, Cb, _ptr(a), _ptr(b), _ptr(out))
+    if a.ndim != 4 or b.ndim != 4 or a.shape[:2] != b.shape[:2]:
+        raise ValueError(f"a {a.shape} and b {b.shape} must be [B, S, N, C] with the same B, S")
+    B, S, Na, Ca = a.shape
+    Nb, Cb = b.shape[2], b.shape[3]
+    out = np.empty((B, Na, Nb, Ca, Cb), np.float64)
+    rc = _lib(mutant).evo_ref_outer_product_mean(B, S, Na, Nb, Ca, Cb, _ptr(a), _ptr(b), _ptr(out))
     if rc != 0:
         raise ValueError("evo_ref_outer_product_mean rejected its arguments")
     return out

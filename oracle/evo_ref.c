@@ -380,21 +380,23 @@ int evo_ref_tri_mul(int64_t B, int64_t N, int64_t C, const double* a, const doub
  *
  *   out[b,i,j,c1,c2] = (1/S) sum_s a[b,s,i,c1] * bb[b,s,j,c2]
  *
- * a: [B, S, N, Ca], bb: [B, S, N, Cb], out: [B, N, N, Ca, Cb], contiguous
- * fp64.  Returns 0, or -1 for a bad size.
+ * a: [B, S, Na, Ca], bb: [B, S, Nb, Cb], out: [B, Na, Nb, Ca, Cb],
+ * contiguous fp64.  Na = Nb = N for the full operation; Na < N evaluates the
+ * definition at a subset of columns i (a smaller, equally valid problem).
+ * Returns 0, or -1 for a bad size.
  */
-int evo_ref_outer_product_mean(int64_t B, int64_t S, int64_t N, int64_t Ca, int64_t Cb, const double* a,
-                               const double* bb, double* out) {
-    if (B < 0 || S <= 0 || N < 0 || Ca <= 0 || Cb <= 0) return -1;
+int evo_ref_outer_product_mean(int64_t B, int64_t S, int64_t Na, int64_t Nb, int64_t Ca, int64_t Cb,
+                               const double* a, const double* bb, double* out) {
+    if (B < 0 || S <= 0 || Na < 0 || Nb < 0 || Ca <= 0 || Cb <= 0) return -1;
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t b = 0; b < B; ++b) {
-        for (int64_t i = 0; i < N; ++i) {
-            for (int64_t j = 0; j < N; ++j) {
-                double* o = out + (((b * N + i) * N + j) * Ca) * Cb;
+        for (int64_t i = 0; i < Na; ++i) {
+            for (int64_t j = 0; j < Nb; ++j) {
+                double* o = out + (((b * Na + i) * Nb + j) * Ca) * Cb;
                 for (int64_t e = 0; e < Ca * Cb; ++e) o[e] = 0.0;
                 for (int64_t s = 0; s < S; ++s) {
-                    const double* ar = a + ((b * S + s) * N + i) * Ca;
-                    const double* br = bb + ((b * S + s) * N + j) * Cb;
+                    const double* ar = a + ((b * S + s) * Na + i) * Ca;
+                    const double* br = bb + ((b * S + s) * Nb + j) * Cb;
                     for (int64_t c1 = 0; c1 < Ca; ++c1)
                         for (int64_t c2 = 0; c2 < Cb; ++c2) o[c1 * Cb + c2] += ar[c1] * br[c2];
                 }

@@ -7,6 +7,7 @@ Tolerances (per output tensor, over the compared elements):
   fp32 path:                      ||gpu - oracle||_2 / ||oracle||_2 <= 1e-4
   fused LayerNorm + linear (bf16): element-wise projection_bound() and rel-L2 <= 5e-3
   triangular update contraction (bf16): element-wise tri_mul_bound() and rel-L2 <= 5e-3
+  outer product mean (bf16): element-wise opm_bound() and rel-L2 <= 5e-3
 """
 from __future__ import annotations
 
@@ -79,6 +80,19 @@ def tri_mul_bound(a, b, incoming, ref):
     """
     mag = oracle.tri_mul(np.abs(a), np.abs(b), incoming)
     return 2.0 ** -8 * np.abs(ref) + 2.0 ** -12 * mag
+
+
+def opm_bound(a, b, ref):
+    """Per-element error bound of the bf16 tensor-core outer product mean.
+
+    Exact bf16 inputs; products accumulate in fp32 over S terms (error <= S 2^-24
+    sum_s |a| |b|, i.e. <= S 2^-24 mean_s |a| |b| <= 2^-12 mean_s |a| |b| after the
+    1/S scale, for S <= 4096); the scale is one more fp32 rounding; out is rounded
+    to bf16 (<= 2^-9 |out|, doubled).  Bound:
+    2^-8 |out| + 2^-12 * mean_s |a| |b|.  a: [B, S, Na, Ca], b: [B, S, N, Cb] fp64;
+    ref: the oracle's [B, Na, N, Ca, Cb].
+    """
+    return 2.0 ** -8 * np.abs(ref) + 2.0 ** -12 * oracle.outer_product_mean(np.abs(a), np.abs(b))
 
 
 def metrics(got, ref):

@@ -73,6 +73,14 @@ def test_constant_sequences_average_to_themselves():
     assert np.allclose(oracle.outer_product_mean(a, b), oracle.outer_product_mean(a1, b1), rtol=0, atol=1e-13)
 
 
+def test_column_subset_is_the_matching_block():
+    # evaluating a subset of columns i gives exactly those rows of the full result
+    a, b = rnd(2, 7, 10, 3, 4, 9)
+    full = oracle.outer_product_mean(a, b)
+    idx = [1, 4, 9]
+    assert np.array_equal(oracle.outer_product_mean(np.ascontiguousarray(a[:, :, idx]), b), full[:, idx])
+
+
 @pytest.mark.parametrize("mutant", oracle.OPM_MUTANTS)
 def test_planted_mistakes_fail_the_pins(mutant):
     assert oracle.mutant_id(mutant) == mutant
