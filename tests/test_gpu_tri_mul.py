@@ -6,8 +6,9 @@ cannot move", section "The three operations".  The kernel reads channel-first
 [B, C, N, N] bf16; the oracle gets the same rounded values in its [B, N, N, C]
 layout.  Tolerance (tri_mul_bound in the parity helpers, from the
 arithmetic): per element 2^-8 |z| + 2^-12 sum_k |a| |b|, and rel-L2 <= 5e-3.
-Covers both edge directions, one and several tiles per CTA, ragged edges in
-i, j and k, the full-size workload, and the degenerate sizes.
+Covers both edge directions, one and several (up to eight or more) tiles per
+CTA, ragged edges in i, j and k, the full-size workload, and the degenerate
+sizes.
 """
 import numpy as np
 import pytest
@@ -55,11 +56,13 @@ def test_contraction_matches_the_oracle(N, C, B, incoming):
 
 
 @pytest.mark.parametrize("incoming", [False, True])
-@pytest.mark.parametrize("N,C", [(128, 300), (128, 400), (136, 160), (192, 300), (256, 160)])
+@pytest.mark.parametrize("N,C", [(128, 300), (128, 400), (136, 160), (192, 300), (256, 160),
+                                 (128, 1200), (136, 700)])
 def test_several_tiles_per_cta(N, C, incoming):
     # enough channels for two or more tiles per SM, so that CTAs run several tiles through
     # the double-buffered accumulators.  With N not a multiple of 256 some 64-column groups
-    # lie wholly past N and store nothing, between groups that do
+    # lie wholly past N and store nothing, between groups that do.  The last two cases give
+    # every CTA eight or more tiles
     check(TriMulWorkload("many", 1, N, C, 9100 + N + C), incoming)
 
 
