@@ -326,6 +326,57 @@ def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float)
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
+def run_e2e(K: int, h2d, compute, d2h, world: int, dev, barrier) -> float:
+    """End-to-end device milliseconds for K steps, copies overlapped across steps.
+
+    Step j uses buffer set j % 2.  Its inputs are copied host -> device on one
+    stream, its compute runs on a second, and its results are copied
+    device -> host on a third, so one step's copies overlap its neighbours'
+    compute (PCIe is full duplex).  Events order each step's three parts and
+    keep a buffer set from being refilled before the step that used it two
+    steps earlier is done with it.  Every step's copies are inside the timed
+    region.  h2d(b), compute(b) and d2h(b) enqueue on the current stream.
+    Returns the max over ranks.
+    """
+    st = [torch.cuda.Stream(device=dev) for _ in range(3)]
+    ev = {(k, b): torch.cuda.Event() for k in ("in", "cmp", "out") for b in (0, 1)}
+
+    def step(j):
+        b = j % 2
+        with torch.cuda.stream(st[0]):
+            if j >= 2:
+                st[0].wait_event(ev[("cmp", b)])       # the compute that read these inputs is done
+            h2d(b)
+            ev[("in", b)].record(st[0])
+        with torch.cuda.stream(st[1]):
+            st[1].wait_event(ev[("in", b)])
+            if j >= 2:
+                st[1].wait_event(ev[("out", b)])       # the copy-out of these results is done
+            compute(b)
+            ev[("cmp", b)].record(st[1])
+        with torch.cuda.stream(st[2]):
+            st[2].wait_event(ev[("cmp", b)])
+            d2h(b)
+            ev[("out", b)].record(st[2])
+
+    for j in range(2):
+        step(j)
+    torch.cuda.synchronize()
+    barrier()
+    cur = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for x in st:
+        x.wait_event(e0)
+    for j in range(K):
+        step(j)
+    for x in st:
+        cur.wait_stream(x)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    return max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return 0
@@ -545,33 +596,37 @@ def run_projection(args, pw, rank, world, local):
     e2e = None
     if not args.no_e2e:
         hx = hin["x"].pin_memory()
-        hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        hpb = torch.empty(pb.shape, dtype=pb.dtype).pin_memory() if pb is not None else None
-        dx = torch.empty_like(hx, device=dev)
-
-        def e2e_step():
-            dx.copy_(hx, non_blocking=True)
-            step(dx)
-            hy.copy_(y, non_blocking=True)
-            if hpb is not None:
-                hpb.copy_(pb, non_blocking=True)
-
+        slots = []
         for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(K):
-            e2e_step()
-        e1.record()
-        torch.cuda.synchronize()
-        et = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+            sl = {"x": torch.empty_like(hx, device=dev), "y": torch.empty_like(y),
+                  "pb": torch.empty_like(pb) if pb is not None else None,
+                  "hy": torch.empty(y.shape, dtype=y.dtype).pin_memory(),
+                  "hpb": torch.empty(pb.shape, dtype=pb.dtype).pin_memory() if pb is not None else None}
+            slots.append(sl)
+
+        def e2e_h2d(b):
+            slots[b]["x"].copy_(hx, non_blocking=True)
+
+        def e2e_compute(b):
+            sl = slots[b]
+            A.ln_linear(sl["x"], d["ln_w"], d["ln_b"], PROJ_EPS, d["w"], d["bias"], y=sl["y"])
+            if pbp is not None:
+                A.ln_pair_bias(sl["x"], pbp["ln_w"], pbp["ln_b"], PROJ_EPS, pbp["w"], pbp["bias"], out=sl["pb"])
+
+        def e2e_d2h(b):
+            sl = slots[b]
+            sl["hy"].copy_(sl["y"], non_blocking=True)
+            if sl["hpb"] is not None:
+                sl["hpb"].copy_(sl["pb"], non_blocking=True)
+
+        et = run_e2e(K, e2e_h2d, e2e_compute, e2e_d2h, world, dev, barrier)
+        hy, hpb = slots[0]["hy"], slots[0]["hpb"]
         e2e = {"value": job_throughput(fl_step, K, world, et), "unit": "TFLOP/s",
                "h2d_bytes_per_step": hx.numel() * hx.element_size(),
                "d2h_bytes_per_step": hy.numel() * hy.element_size() + (0 if hpb is None else
                                                                        hpb.numel() * hpb.element_size()),
-               "ms_per_step": et / K}
+               "ms_per_step": et / K,
+               "pipelining": "step j+1's input in and step j-1's results out overlap step j's compute"}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -753,31 +808,30 @@ def run_tri_mul(args, tw, rank, world, local):
     e2e = None
     if not args.no_e2e:
         ha, hb = hin["a"].pin_memory(), hin["b"].pin_memory()
-        hzo = torch.empty(z_out.shape, dtype=z_out.dtype).pin_memory()
-        hzi = torch.empty(z_in.shape, dtype=z_in.dtype).pin_memory()
-        da, db = torch.empty_like(ha, device=dev), torch.empty_like(hb, device=dev)
+        slots = [{"a": torch.empty_like(ha, device=dev), "b": torch.empty_like(hb, device=dev),
+                  "zo": torch.empty_like(z_out), "zi": torch.empty_like(z_in),
+                  "hzo": torch.empty(z_out.shape, dtype=z_out.dtype).pin_memory(),
+                  "hzi": torch.empty(z_in.shape, dtype=z_in.dtype).pin_memory()} for _ in range(2)]
 
-        def e2e_step():
-            da.copy_(ha, non_blocking=True)
-            db.copy_(hb, non_blocking=True)
-            step(da, db)
-            hzo.copy_(z_out, non_blocking=True)
-            hzi.copy_(z_in, non_blocking=True)
+        def e2e_h2d(b):
+            slots[b]["a"].copy_(ha, non_blocking=True)
+            slots[b]["b"].copy_(hb, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(K):
-            e2e_step()
-        e1.record()
-        torch.cuda.synchronize()
-        et = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+        def e2e_compute(b):
+            sl = slots[b]
+            A.tri_mul(sl["a"], sl["b"], False, z=sl["zo"])
+            A.tri_mul(sl["a"], sl["b"], True, z=sl["zi"])
+
+        def e2e_d2h(b):
+            sl = slots[b]
+            sl["hzo"].copy_(sl["zo"], non_blocking=True)
+            sl["hzi"].copy_(sl["zi"], non_blocking=True)
+
+        et = run_e2e(K, e2e_h2d, e2e_compute, e2e_d2h, world, dev, barrier)
         e2e = {"value": job_throughput(fl_step, K, world, et), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 2 * ha.numel() * ha.element_size(),
-               "d2h_bytes_per_step": 2 * hzo.numel() * hzo.element_size(), "ms_per_step": et / K}
+               "d2h_bytes_per_step": 2 * z_out.numel() * z_out.element_size(), "ms_per_step": et / K,
+               "pipelining": "step j+1's inputs in and step j-1's results out overlap step j's compute"}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -938,29 +992,25 @@ def run_opm(args, ow, rank, world, local):
     e2e = None
     if not args.no_e2e:
         ha, hb = hin["a"].pin_memory(), hin["b"].pin_memory()
-        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        da, db = torch.empty_like(ha, device=dev), torch.empty_like(hb, device=dev)
+        slots = [{"a": torch.empty_like(ha, device=dev), "b": torch.empty_like(hb, device=dev),
+                  "o": torch.empty_like(out), "ho": torch.empty(out.shape, dtype=out.dtype).pin_memory()}
+                 for _ in range(2)]
 
-        def e2e_step():
-            da.copy_(ha, non_blocking=True)
-            db.copy_(hb, non_blocking=True)
-            A.outer_product_mean(da, db, out=out)
-            ho.copy_(out, non_blocking=True)
+        def e2e_h2d(b):
+            slots[b]["a"].copy_(ha, non_blocking=True)
+            slots[b]["b"].copy_(hb, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(K):
-            e2e_step()
-        e1.record()
-        torch.cuda.synchronize()
-        et = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+        def e2e_compute(b):
+            A.outer_product_mean(slots[b]["a"], slots[b]["b"], out=slots[b]["o"])
+
+        def e2e_d2h(b):
+            slots[b]["ho"].copy_(slots[b]["o"], non_blocking=True)
+
+        et = run_e2e(K, e2e_h2d, e2e_compute, e2e_d2h, world, dev, barrier)
         e2e = {"value": job_throughput(fl, K, world, et), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 2 * ha.numel() * ha.element_size(),
-               "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": et / K}
+               "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": et / K,
+               "pipelining": "step j+1's inputs in and step j-1's results out overlap step j's compute"}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -1096,42 +1146,48 @@ def main():
                 return v.permute(0, 2, 1, 3, 4)
             return v
         hin = {k: (None if v is None else storage(k, v).contiguous().pin_memory()) for k, v in inp.items()}
-        hout = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
-                "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
-        for n, g in grads.items():
-            hout[n] = torch.empty(g.shape, dtype=g.dtype).pin_memory()
-        dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in hin.items()}
         h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
-        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+        slots = []
+        for _ in range(2):           # device inputs, outputs and pinned host results per buffer set
+            sl = {"in": {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in hin.items()},
+                  "out": A.empty_like_rows(d["q"]),
+                  "lse": torch.empty((w.B, w.S, w.H, w.N), dtype=torch.float32, device=dev),
+                  "dout": A.empty_like_rows(d["q"]),
+                  "grads": {n: A.empty_like_rows(d["q"]) for n in ("dq", "dk", "dv", "dg")}}
+            sl["grads"]["d_pair_bias"] = torch.empty((w.B, 1, w.H, w.N, w.N), dtype=torch.float32, device=dev)
+            sl["host"] = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                          "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
+            for n, g in sl["grads"].items():
+                sl["host"][n] = torch.empty(g.shape, dtype=g.dtype).pin_memory()
+            slots.append(sl)
+        d2h = sum(v.numel() * v.element_size() for v in slots[0]["host"].values())
 
-        def e2e_step():
+        def e2e_h2d(b):
             for k, v in hin.items():
                 if v is not None:
-                    dev_in[k].copy_(v, non_blocking=True)
-            q, k_, v_, g_, do = (logical_view(w, dev_in[n]) for n in ("q", "k", "v", "g", "dout"))
-            o, l_ = A.evo_attn_fwd(q, k_, v_, g_, dev_in["mask_bias"], dev_in["pair_bias"], out=out, lse=lse)
-            do = do if do.stride() == o.stride() else dout.copy_(do)
-            gr = A.evo_attn_bwd(q, k_, v_, g_, dev_in["mask_bias"], dev_in["pair_bias"], o, l_, do,
-                                grads=grads, workspace=ws)
-            hout["out"].copy_(o, non_blocking=True)
-            hout["lse"].copy_(l_, non_blocking=True)
-            for n in grads:
-                hout[n].copy_(gr[n], non_blocking=True)
+                    slots[b]["in"][k].copy_(v, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(K):
-            e2e_step()
-        e1.record()
-        torch.cuda.synchronize()
-        et = e0.elapsed_time(e1)
-        et = max_over_ranks([et], world, dev)[0]
+        def e2e_compute(b):
+            sl = slots[b]
+            di = sl["in"]
+            q, k_, v_, g_, do = (logical_view(w, di[n]) for n in ("q", "k", "v", "g", "dout"))
+            o, l_ = A.evo_attn_fwd(q, k_, v_, g_, di["mask_bias"], di["pair_bias"], out=sl["out"], lse=sl["lse"])
+            do = do if do.stride() == o.stride() else sl["dout"].copy_(do)
+            A.evo_attn_bwd(q, k_, v_, g_, di["mask_bias"], di["pair_bias"], o, l_, do, grads=sl["grads"],
+                           workspace=ws)
+
+        def e2e_d2h(b):
+            sl = slots[b]
+            sl["host"]["out"].copy_(sl["out"], non_blocking=True)
+            sl["host"]["lse"].copy_(sl["lse"], non_blocking=True)
+            for n, g in sl["grads"].items():
+                sl["host"][n].copy_(g, non_blocking=True)
+
+        et = run_e2e(K, e2e_h2d, e2e_compute, e2e_d2h, world, dev, barrier)
         e2e = {"value": job_throughput(ff + bf, K, world, et), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": et / K}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": et / K,
+               "pipelining": "step j+1's inputs in and step j-1's results out overlap step j's compute "
+                             "(three streams, two buffer sets)"}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
