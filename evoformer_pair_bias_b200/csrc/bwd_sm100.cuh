@@ -562,10 +562,19 @@ __device__ __forceinline__ void pre_rows(const PreParams& p, int blk, int nblk) 
             }
             continue;
         }
-        const int h = (int)(t % p.H);
-        const int i = (int)((t / p.H) % p.N);
-        const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
-        const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
+        int h, i, s, b;
+        if (rows < 0x7fffffff) {             // 32-bit index arithmetic: a fraction of the 64-bit cost
+            const uint32_t u = (uint32_t)t, q1 = u / (uint32_t)p.H, q2 = q1 / (uint32_t)p.N;
+            h = (int)(u - q1 * (uint32_t)p.H);
+            i = (int)(q1 - q2 * (uint32_t)p.N);
+            b = (int)(q2 / (uint32_t)p.S);
+            s = (int)(q2 - (uint32_t)b * (uint32_t)p.S);
+        } else {
+            h = (int)(t % p.H);
+            i = (int)((t / p.H) % p.N);
+            s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
+            b = (int)(t / ((int64_t)p.H * p.N * p.S));
+        }
         const uint4 ow = reinterpret_cast<const uint4*>(p.out + p.os.off(b, s, i, h))[part];
         const uint4 dw = reinterpret_cast<const uint4*>(p.dout + p.os.off(b, s, i, h))[part];
         const uint4 gw = reinterpret_cast<const uint4*>(p.g + p.in.off(b, s, i, h))[part];
@@ -577,7 +586,8 @@ __device__ __forceinline__ void pre_rows(const PreParams& p, int blk, int nblk) 
         for (int e = 0; e < 4; ++e) {
             const float o0 = bf16lo(ov[e]), o1 = bf16hi(ov[e]);
             const float d0 = bf16lo(dv[e]), d1 = bf16hi(dv[e]);
-            const float s0 = 1.0f / (1.0f + __expf(-bf16lo(gv[e]))), s1 = 1.0f / (1.0f + __expf(-bf16hi(gv[e])));
+            const float s0 = __fdividef(1.0f, 1.0f + __expf(-bf16lo(gv[e]))),
+                        s1 = __fdividef(1.0f, 1.0f + __expf(-bf16hi(gv[e])));
             D = fmaf(d0, o0, D);
             D = fmaf(d1, o1, D);
             dgv[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
@@ -673,10 +683,19 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const PostParams p) {
         if (g < nq) {
             const int64_t t = g / PRE_LANES;
             const int part = (int)(g % PRE_LANES);
-            const int h = (int)(t % p.H);
-            const int i = (int)((t / p.H) % p.N);
-            const int s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
-            const int b = (int)(t / ((int64_t)p.H * p.N * p.S));
+            int h, i, s, b;
+            if (rows < 0x7fffffff) {         // 32-bit index arithmetic: a fraction of the 64-bit cost
+                const uint32_t u = (uint32_t)t, q1 = u / (uint32_t)p.H, q2 = q1 / (uint32_t)p.N;
+                h = (int)(u - q1 * (uint32_t)p.H);
+                i = (int)(q1 - q2 * (uint32_t)p.N);
+                b = (int)(q2 / (uint32_t)p.S);
+                s = (int)(q2 - (uint32_t)b * (uint32_t)p.S);
+            } else {
+                h = (int)(t % p.H);
+                i = (int)((t / p.H) % p.N);
+                s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
+                b = (int)(t / ((int64_t)p.H * p.N * p.S));
+            }
             const float4* a = reinterpret_cast<const float4*>(p.dq_acc + t * HD) + 2 * part;
             const float4 x = a[0], y = a[1];
             reinterpret_cast<uint4*>(p.dq + p.gs.off(b, s, i, h))[part] =
