@@ -74,10 +74,12 @@ def test_ln_linear_matches_the_oracle(name):
 
 
 @pytest.mark.parametrize("rows,c_in,n_out", [(1, 64, 128), (130, 128, 384), (257, 192, 256), (127, 256, 640),
-                                            (296 * 128 + 40, 64, 128)])
+                                            (296 * 128 + 40, 64, 128), (296 * 128 + 50, 256, 384),
+                                            (74 * 128 * 3 + 70, 128, 512)])
 def test_ln_linear_shapes_and_ragged_rows(rows, c_in, n_out):
-    # the last case gives a CTA three row blocks with a ragged last one, where some
-    # epilogue warps have no rows to store right after storing a full block
+    # the last three cases give CTAs three row blocks with a ragged last one (some epilogue
+    # warps have no rows to store right after storing a full block): w resident in one
+    # column group, w streamed from L2 (c_in = 256), and two column groups (c_in = 128)
     w = ProjWorkload("shape", 1, 1, rows, c_in, 1, 32, 7000 + rows + c_in)
     d = make_proj_inputs(w, n_out=n_out, device="cuda")
     y = A.ln_linear(d["x"], d["ln_w"], d["ln_b"], EPS, d["w"], d["bias"])
