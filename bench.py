@@ -1228,7 +1228,7 @@ def main():
             "frac_measured_peak": value / world / pk["bf16"],
             "roofline": roof,
             "kernels": {p: {"launches": kt[p][0], "us_per_launch": 1e3 * kt[p][1] / max(kt[p][0], 1)}
-                        for p in A.PHASES},
+                        for p in A.PHASES if kt[p][0]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
