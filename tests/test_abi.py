@@ -101,6 +101,11 @@ def test_projection_host_checks_need_no_gpu(lib):
     assert lib.evo_tri_mul(1, 2, 16, fake, odd, 0, fake, nul) == 2                                 # alignment
     assert lib.evo_tri_mul(1, 0, 16, nul, nul, 0, nul, nul) == 0                                   # empty
     assert lib.evo_tri_mul(-1, 2, 16, fake, fake, 0, fake, nul) == 1
+    assert lib.evo_outer_product_mean(0, 4, 8, 8, 8, nul, nul, nul, nul) == 0           # B = 0: no-op
+    assert lib.evo_outer_product_mean(1, 0, 8, 8, 8, fake, fake, fake, nul) == 1        # S = 0: no mean
+    assert lib.evo_outer_product_mean(1, 4, 3, 5, 5, fake, fake, fake, nul) == 2        # N*C % 8
+    assert lib.evo_outer_product_mean(1, 4, 8, 8, 8, fake, odd, fake, nul) == 2        # alignment
+    assert lib.evo_outer_product_mean(1, 4, 8, 0, 8, fake, fake, fake, nul) == 1        # no channels
     assert lib.evo_ln_pair_bias(1, 16, 128, 17, fake, nul, nul, 1e-5, fake, nul, fake, nul) == 2  # H > 16
     assert lib.evo_ln_pair_bias(1, 16, 12, 4, fake, nul, nul, 1e-5, fake, nul, fake, nul) == 2    # c_z % 8
     assert lib.evo_ln_pair_bias(1, 0, 128, 4, nul, nul, nul, 1e-5, nul, nul, nul, nul) == 0       # empty
