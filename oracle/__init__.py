@@ -9,7 +9,8 @@ The arithmetic lives in ``evo_ref.c`` (plain C, fp64, OpenMP over independent
 outputs); this module compiles it with gcc on first use and wraps it with
 ctypes.  Every function takes numpy arrays of any float dtype and widens them
 to fp64 before the call, so a caller that wants the oracle to see bf16 inputs
-rounds them to bf16 first and passes the rounded values.
+rounds them to bf16 first and passes the rounded values.  The one exception
+is ordered_sum_f32, whose definition is an fp32 sum in a fixed order.
 
 What is computed, per (b, s, h) and query i (see the header of evo_ref.c):
 
@@ -51,12 +52,15 @@ MUTANTS = {
     11: "triangular update reading the second edge as k-j instead of j-k",
     12: "outer product summed over the sequences instead of averaged",
     13: "outer product mean with its two channel axes swapped",
+    14: "partials of d_pair_bias added in reverse rank order",
+    15: "last partial of d_pair_bias left out of the sum",
 }
 #: Which function each planted mistake breaks.
 ATTENTION_MUTANTS = (1, 2, 3, 4, 5, 6, 7)
 LN_LINEAR_MUTANTS = (8, 9)
 TRI_MUL_MUTANTS = (10, 11)
 OPM_MUTANTS = (12, 13)
+PARTIALS_MUTANTS = (14, 15)
 
 
 class _Dims(ctypes.Structure):
@@ -97,6 +101,9 @@ def _lib(mutant: int = 0) -> ctypes.CDLL:
         lib.evo_ref_tri_mul.restype = ctypes.c_int
         lib.evo_ref_outer_product_mean.argtypes = [ctypes.c_int64] * 6 + [p] * 3
         lib.evo_ref_outer_product_mean.restype = ctypes.c_int
+        pf = ctypes.POINTER(ctypes.c_float)
+        lib.evo_ref_ordered_sum_f32.argtypes = [ctypes.c_int64, ctypes.c_int64, pf, pf]
+        lib.evo_ref_ordered_sum_f32.restype = ctypes.c_int
         _LIBS[mutant] = lib
     return _LIBS[mutant]
 
@@ -239,6 +246,27 @@ def outer_product_mean(a, b, *, mutant: int = 0):
     rc = _lib(mutant).evo_ref_outer_product_mean(B, S, Na, Nb, Ca, Cb, _ptr(a), _ptr(b), _ptr(out))
     if rc != 0:
         raise ValueError("evo_ref_outer_product_mean rejected its arguments")
+    return out
+
+
+def ordered_sum_f32(parts, *, mutant: int = 0):
+    """Rank-ordered fp32 sum: out = (...((parts[0] + parts[1]) + parts[2]) ...) + parts[-1].
+
+    Unlike the other functions this one works in fp32, each addition rounded
+    to nearest: it is the exact expected value of the fixed-order exchange of
+    d_pair_bias when the rows s of one problem are split over GPUs (the sum
+    over s of the backward's dS, grouped by GPU).  parts: [count, ...] array
+    (converted to fp32); returns an fp32 array of parts.shape[1:].
+    """
+    p = np.ascontiguousarray(parts, dtype=np.float32)
+    if p.ndim < 1 or p.shape[0] < 1:
+        raise ValueError("ordered_sum_f32 needs at least one partial")
+    out = np.empty(p.shape[1:], np.float32)
+    pf = ctypes.POINTER(ctypes.c_float)
+    rc = _lib(mutant).evo_ref_ordered_sum_f32(p.shape[0], out.size, p.ctypes.data_as(pf),
+                                              out.ctypes.data_as(pf))
+    if rc != 0:
+        raise ValueError("evo_ref_ordered_sum_f32 rejected its arguments")
     return out
 
 

@@ -421,5 +421,37 @@ int evo_ref_outer_product_mean(int64_t B, int64_t S, int64_t Na, int64_t Nb, int
     return 0;
 }
 
+/*
+ * Rank-ordered sum of fp32 partials, every addition rounded to fp32:
+ *
+ *   out[i] = (...((parts[0][i] + parts[1][i]) + parts[2][i]) ...) + parts[count-1][i]
+ *
+ * When the rows s of one problem are split over GPUs, d_pair_bias -- the sum
+ * over s of dS (backward, above) -- is the sum of each GPU's partial over its
+ * own rows.  The library adds those partials left to right in fp32, so this
+ * function is held to the same precision (not fp64): its result is the
+ * exchange's exact expected value, compared bit for bit.
+ * parts: [count, n] contiguous fp32; out: [n].  Returns 0, or -1 for a bad size.
+ */
+int evo_ref_ordered_sum_f32(int64_t count, int64_t n, const float* parts, float* out) {
+    if (count < 1 || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+#if EVO_REF_MUTANT == 14
+        /* mutant: the partials added in reverse order */
+        float acc = parts[(count - 1) * n + i];
+        for (int64_t r = count - 2; r >= 0; --r) acc = acc + parts[r * n + i];
+#elif EVO_REF_MUTANT == 15
+        /* mutant: the last partial left out */
+        float acc = parts[i];
+        for (int64_t r = 1; r < count - 1; ++r) acc = acc + parts[r * n + i];
+#else
+        float acc = parts[i];
+        for (int64_t r = 1; r < count; ++r) acc = acc + parts[r * n + i];
+#endif
+        out[i] = acc;
+    }
+    return 0;
+}
+
 /* Which planted mistake this build carries (0 = none). */
 int evo_ref_mutant(void) { return EVO_REF_MUTANT; }
