@@ -34,7 +34,10 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
            "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc",
            "evo_attn_timing_enable", "evo_attn_timing_collect", "evo_ln_linear", "evo_ln_pair_bias",
-           "evo_tri_mul", "evo_outer_product_mean")
+           "evo_tri_mul", "evo_outer_product_mean", "evo_sum_partials")
+
+#: Most partials one evo_sum_partials call adds (EVO_MAX_PARTIALS).
+MAX_PARTIALS = 64
 
 #: Size of the library's fixed scratch area used by evo_attn_bwd_noalloc (bytes).
 NOALLOC_WORKSPACE_BYTES = 32 << 20
@@ -103,6 +106,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_tri_mul.restype = ctypes.c_int
     lib.evo_outer_product_mean.argtypes = [i64, i64, i64, i64, i64, vp, vp, vp, vp]
     lib.evo_outer_product_mean.restype = ctypes.c_int
+    lib.evo_sum_partials.argtypes = [i64, ctypes.POINTER(ctypes.c_void_p), i64, vp, vp]
+    lib.evo_sum_partials.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -333,6 +338,37 @@ def outer_product_mean(a, b, out=None):
         out = torch.empty((B, N, Ca, N, Cb), dtype=torch.bfloat16, device=a.device)
     rc = lib.evo_outer_product_mean(B, S, N, Ca, Cb, _ptr(ac), _ptr(bc), _ptr(out), _stream(a.device))
     _check("evo_outer_product_mean", rc)
+    return out
+
+
+def sum_partials(parts, out=None):
+    """Fixed-order fp32 sum: out = (...((parts[0] + parts[1]) + parts[2]) ...) + parts[-1].
+
+    ``parts`` is a sequence of contiguous fp32 CUDA tensors with one number of
+    elements, or one tensor whose first axis indexes the partials (an
+    all-gathered buffer).  Callers that pass the same partials in the same
+    order get the same bits.  Returns ``out`` (shaped like one partial,
+    allocated when None; it may be one of the partials).
+    """
+    lib = load_library()
+    if isinstance(parts, torch.Tensor):
+        parts = list(parts.unbind(0))
+    parts = list(parts)
+    if not parts:
+        raise ValueError("sum_partials needs at least one partial")
+    n = parts[0].numel()
+    for t in parts:
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != n or t.device != parts[0].device:
+            raise ValueError("partials must be contiguous fp32 tensors of one size on one device")
+    if out is None:
+        out = torch.empty_like(parts[0])
+    if out.dtype != torch.float32 or not out.is_contiguous() or out.numel() != n:
+        raise ValueError("out must be a contiguous fp32 tensor with as many elements as a partial")
+    if n == 0:
+        return out                                   # the empty sum: nothing to add
+    arr = (ctypes.c_void_p * len(parts))(*[t.data_ptr() for t in parts])
+    rc = lib.evo_sum_partials(len(parts), arr, n, _ptr(out), _stream(out.device))
+    _check("evo_sum_partials", rc)
     return out
 
 

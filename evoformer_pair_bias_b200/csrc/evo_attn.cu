@@ -26,6 +26,7 @@
 #include "bwd_sm100.cuh"
 #include "proj_sm100.cuh"
 #include "trimul_sm100.cuh"
+#include "partials.cuh"
 
 #define EVO_VERSION 10000
 
@@ -569,6 +570,31 @@ evo_status_t evo_outer_product_mean(int64_t B, int64_t S, int64_t N, int64_t Ca,
     // out[b, (i, c1), (j, c2)] = (1/S) sum_s a[b, s, (i, c1)] bb[b, s, (j, c2)]: the MN-major contraction
     return launch_contraction(a, bb, out, M, Nc, S, B, true, (float)(1.0 / (double)S), EVO_PHASE_OPM,
                               static_cast<cudaStream_t>(stream));
+}
+
+evo_status_t evo_sum_partials(int64_t count, const float* const* parts, int64_t n, float* out, void* stream) {
+    static_assert(EVO_MAX_PARTIALS == evo::partials::MAX_PARTS, "partials limit");
+    if (count < 1 || n < 0 || !parts || !out) return EVO_ERR_INVALID_ARG;
+    if (count > EVO_MAX_PARTIALS) return EVO_ERR_UNSUPPORTED;
+    evo::partials::Params p{};
+    bool vec = aligned(out, 16);
+    for (int64_t r = 0; r < count; ++r) {
+        if (!parts[r]) return EVO_ERR_INVALID_ARG;
+        if (!aligned(parts[r], 4)) return EVO_ERR_UNSUPPORTED;
+        vec = vec && aligned(parts[r], 16);
+        p.part[r] = parts[r];
+    }
+    if (!aligned(out, 4)) return EVO_ERR_UNSUPPORTED;
+    if (n == 0) return EVO_OK;
+    p.out = out;
+    p.n = n;
+    p.count = (int)count;
+    p.vec = vec ? 1 : 0;
+    const int64_t items = vec ? n / 4 + n % 4 : n;
+    const int blocks = (int)std::min<int64_t>((items + 255) / 256, 148 * 8);
+    evo::partials::sum_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
 evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,

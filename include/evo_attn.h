@@ -259,6 +259,35 @@ evo_status_t evo_tri_mul(int64_t B, int64_t C, int64_t N, const void* a, const v
 evo_status_t evo_outer_product_mean(int64_t B, int64_t S, int64_t N, int64_t Ca, int64_t Cb, const void* a,
                                     const void* bb, void* out, void* stream);
 
+/*
+ * Fixed-order sum of fp32 partial results: the exchange step of a backward
+ * pass whose rows s are split over several GPUs, the way a sequence-parallel
+ * group partitions the pair tensor (MegaFold summary, section "EvoSP-3D").
+ * Rows s are independent problems that share the additive pair bias, which
+ * is broadcast over them (same page, section "EvoFlash-3D"), so every input
+ * gradient but d_pair_bias stays on the GPU that holds its row, and
+ * d_pair_bias -- the sum over all s of dL/dx -- is the sum of the per-GPU
+ * partials that evo_attn_bwd returns for each GPU's rows:
+ *
+ *   out[i] = (...((parts[0][i] + parts[1][i]) + parts[2][i]) ...) + parts[count-1][i]
+ *
+ * in fp32, each addition rounded to nearest, left to right: every caller that
+ * passes the same partials in the same (rank) order gets the same bits.
+ *   count   number of partials, 1 <= count <= EVO_MAX_PARTIALS
+ *           (EVO_ERR_INVALID_ARG below 1, EVO_ERR_UNSUPPORTED above).
+ *   parts   HOST array of `count` device pointers, each to n fp32 values; it
+ *           is read during the call only.  The pointers may be slices of
+ *           one all-gathered buffer, or any memory this device can load from.
+ *   n       elements per partial; 0 is a no-op, negative EVO_ERR_INVALID_ARG.
+ *   out     device pointer to n fp32 values.  It may be one of parts[r]
+ *           (element-wise in place); any other overlap is undefined.
+ * NULL pointers are EVO_ERR_INVALID_ARG; pointers not 4-byte aligned are
+ * EVO_ERR_UNSUPPORTED.  All 16-byte aligned pointers take 16-byte loads.
+ * Stream-ordered, no allocation, no synchronisation, no waits.
+ */
+#define EVO_MAX_PARTIALS 64
+evo_status_t evo_sum_partials(int64_t count, const float* const* parts, int64_t n, float* out, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* evo_status_string(evo_status_t status);
 

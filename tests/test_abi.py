@@ -111,6 +111,23 @@ def test_projection_host_checks_need_no_gpu(lib):
     assert lib.evo_ln_pair_bias(1, 0, 128, 4, nul, nul, nul, 1e-5, nul, nul, nul, nul) == 0       # empty
 
 
+def test_sum_partials_host_checks_need_no_gpu(lib):
+    fake, odd, nul = 1 << 20, (1 << 20) + 2, None          # never dereferenced: the checks fail first
+    arr = lambda *ps: (ctypes.c_void_p * len(ps))(*ps)    # noqa: E731
+    out = ctypes.c_void_p(fake)
+    assert lib.evo_sum_partials(2, arr(fake, fake), 0, out, nul) == 0              # n = 0: no-op
+    assert lib.evo_sum_partials(0, arr(fake), 8, out, nul) == 1                    # no partials
+    assert lib.evo_sum_partials(2, None, 8, out, nul) == 1                         # null array
+    assert lib.evo_sum_partials(2, arr(fake, 0), 8, out, nul) == 1                 # null partial
+    assert lib.evo_sum_partials(1, arr(fake), -1, out, nul) == 1                   # negative size
+    assert lib.evo_sum_partials(1, arr(fake), 8, None, nul) == 1                   # null out
+    assert lib.evo_sum_partials(2, arr(fake, odd), 8, out, nul) == 2               # not 4-byte aligned
+    assert lib.evo_sum_partials(1, arr(fake), 8, ctypes.c_void_p(odd), nul) == 2
+    assert lib.evo_sum_partials(A.MAX_PARTIALS + 1, arr(*[fake] * (A.MAX_PARTIALS + 1)), 8, out, nul) == 2
+    assert lib.evo_sum_partials(A.MAX_PARTIALS, arr(*[fake] * A.MAX_PARTIALS), 0, out, nul) == 0
+    assert "EVO_MAX_PARTIALS %d" % A.MAX_PARTIALS in open(HEADER).read().replace("  ", " ")
+
+
 def test_product_path_never_touches_the_oracle():
     """The package must not import, load or mention the CPU oracle."""
     pkg = os.path.join(ROOT, "evoformer_pair_bias_b200")
