@@ -43,16 +43,48 @@ def _world(group) -> int:
     return dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
 
 
-def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
-    """All-gather one partial per rank: a [world, *partial.shape] tensor, rank r's at index r.
+def start_gather(partial: torch.Tensor, group=None):
+    """Start the all-gather of one partial per rank; returns (parts, work).
 
-    Every rank takes part, in the same order as the others' calls.
+    ``parts`` is a [world, *partial.shape] view of the gathered buffer, rank
+    r's partial at index r, valid once ``work.wait()`` has returned (with
+    NCCL: once the caller's current stream has been made to wait).  Until
+    then ``partial`` is being read and must not change.  Every rank takes
+    part, in the same order as the others' calls.
     """
     world = _world(group)
     flat = partial.contiguous().reshape(-1)
     buf = torch.empty(world * flat.numel(), dtype=partial.dtype, device=partial.device)
-    dist.all_gather_into_tensor(buf, flat, group=group)
-    return buf.view(world, *partial.shape)
+    work = dist.all_gather_into_tensor(buf, flat, group=group, async_op=True)
+    return buf.view(world, *partial.shape), work
+
+
+def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather one partial per rank: a [world, *partial.shape] tensor, rank r's at index r."""
+    parts, work = start_gather(partial, group)
+    work.wait()
+    return parts
+
+
+class PendingPairBiasGrad:
+    """The d_pair_bias exchange of one row-split backward, started but not finished.
+
+    wait() waits for the all-gather and adds the gathered partials, in rank
+    order, into the tensor that held this rank's partial; it returns that
+    tensor.  Between attn_bwd(..., async_op=True) and wait() the caller can
+    enqueue work that needs only dq, dk, dv, dg (their projections'
+    backward, say), which then overlaps the transfer.
+    """
+
+    def __init__(self, parts=None, work=None, out=None):
+        self._parts, self._work, self._out = parts, work, out
+
+    def wait(self) -> torch.Tensor:
+        if self._work is not None:
+            self._work.wait()
+            A.sum_partials(self._parts, out=self._out)
+            self._work = self._parts = None
+        return self._out
 
 
 def attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None):
@@ -64,16 +96,23 @@ def attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None):
     return A.evo_attn_fwd(q, k, v, g, mask_bias, pair_bias, out, lse)
 
 
-def attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, group=None, grads=None, workspace=None):
+def attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, group=None, grads=None, workspace=None,
+             async_op: bool = False):
     """Backward of this rank's rows, with d_pair_bias summed over every rank's rows.
 
     Arguments as for evo_attn_bwd, restricted to this rank's rows (pair_bias
     in full).  Returns its dict of gradients, in which d_pair_bias is the sum
     over all ranks, added in rank order.  Every rank of ``group`` must call it
-    (a collective).  With one rank, no collective runs.
+    (a collective).  With one rank, no collective runs.  With
+    ``async_op=True`` it returns (grads, pending) instead: grads["d_pair_bias"]
+    holds this rank's partial until pending.wait() turns it into the sum.
     """
     grads = A.evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads, workspace)
+    pending = PendingPairBiasGrad(out=grads["d_pair_bias"])
     if _world(group) > 1:
-        parts = gather_partials(grads["d_pair_bias"], group)
-        A.sum_partials(parts, out=grads["d_pair_bias"])
+        parts, work = start_gather(grads["d_pair_bias"], group)
+        pending = PendingPairBiasGrad(parts, work, grads["d_pair_bias"])
+    if async_op:
+        return grads, pending
+    pending.wait()
     return grads

@@ -123,3 +123,8 @@ def test_one_rank_needs_no_exchange():
     torch.cuda.synchronize()
     assert torch.equal(grads["d_pair_bias"], plain["d_pair_bias"])
     assert n1 - n0 == n2 - n1                              # no collective and no sum: the plain backward
+    grads2, pending = row_shards.attn_bwd(d["q"], d["k"], d["v"], d["g"], None, d["pair_bias"], out, lse,
+                                          d["dout"], async_op=True)
+    assert pending.wait() is grads2["d_pair_bias"]
+    torch.cuda.synchronize()
+    assert torch.equal(grads2["d_pair_bias"], plain["d_pair_bias"])

@@ -79,6 +79,9 @@ def _shard_main(rank, world, port, out_dir, S):
             part = np.zeros((1, 1, 2, 16, 16))
         part = torch.from_numpy(part.astype(np.float32))
         gathered = row_shards.gather_partials(part)
+        started, work = row_shards.start_gather(part)       # the asynchronous form, same collective
+        work.wait()
+        assert torch.equal(started, gathered)
         np.save(os.path.join(out_dir, f"part{rank}.npy"), part.numpy())
         np.save(os.path.join(out_dir, f"gathered{rank}.npy"), gathered.numpy())
         np.save(os.path.join(out_dir, f"sum{rank}.npy"), oracle.ordered_sum_f32(gathered.numpy()))
