@@ -6,8 +6,8 @@ stream.  Every step of the computation runs in the library's CUDA kernels;
 there is no fallback of any kind -- if the library is missing or rejects a
 call, an exception says why.
 
-    out, lse = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias)
-    grads = evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout)
+    out, lse, out_lo = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias, out_lo=True)
+    grads = evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, out_lo=out_lo)
 
 Per-row tensors (q, k, v, g, out, dout and the gradients) are logical
 ``[B, S, N, H, C]`` views with a contiguous C axis; any other strides are
@@ -34,7 +34,11 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 EXPORTS = ("evo_attn_fwd", "evo_attn_bwd", "evo_attn_bwd_workspace_bytes", "evo_status_string",
            "evo_attn_device_status", "evo_attn_version", "evo_attn_launch_count", "evo_attn_bwd_noalloc",
            "evo_attn_timing_enable", "evo_attn_timing_collect", "evo_ln_linear", "evo_ln_pair_bias",
-           "evo_tri_mul", "evo_outer_product_mean", "evo_sum_partials")
+           "evo_tri_mul", "evo_outer_product_mean", "evo_sum_partials", "evo_attn_set_wait_limit_ns",
+           "evo_exp2_fma")
+
+#: Default limit of the kernels' bounded waits (EVO_WAIT_LIMIT_NS), nanoseconds.
+DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
 
 #: Most partials one evo_sum_partials call adds (EVO_MAX_PARTIALS).
 MAX_PARTIALS = 64
@@ -58,7 +62,7 @@ class Strides(ctypes.Structure):
 
 
 #: Timing phases (evo_timing_t indices).
-PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj", "pair_bias", "tri_mul", "opm")
+PHASES = ("fwd_main", "bwd_main", "bwd_all", "proj", "pair_bias", "tri_mul", "opm", "bwd_dbias")
 
 
 class Timing(ctypes.Structure):
@@ -77,9 +81,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         raise RuntimeError(f"{path} is missing: build it with `python -m evoformer_pair_bias_b200.build`")
     lib = ctypes.CDLL(path)
     vp, sp, stp = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.POINTER(Strides)
-    lib.evo_attn_fwd.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, stp, vp, vp]
+    lib.evo_attn_fwd.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, stp, vp, vp]
     lib.evo_attn_fwd.restype = ctypes.c_int
-    lib.evo_attn_bwd.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, stp, vp,
+    lib.evo_attn_bwd.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, vp, stp, vp,
                                  vp, vp, vp, vp, stp, vp, vp, ctypes.c_size_t, vp]
     lib.evo_attn_bwd.restype = ctypes.c_int
     lib.evo_attn_bwd_workspace_bytes.argtypes = [sp, ctypes.c_int]
@@ -90,7 +94,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_attn_device_status.restype = ctypes.c_int
     lib.evo_attn_version.restype = ctypes.c_int
     lib.evo_attn_launch_count.restype = ctypes.c_uint64
-    lib.evo_attn_bwd_noalloc.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, stp, vp,
+    lib.evo_attn_bwd_noalloc.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, stp, vp, vp, vp, vp, vp, stp, vp,
                                          vp, vp, vp, vp, stp, vp, vp]
     lib.evo_attn_bwd_noalloc.restype = ctypes.c_int
     lib.evo_attn_timing_enable.argtypes = [ctypes.c_int]
@@ -108,6 +112,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.evo_outer_product_mean.restype = ctypes.c_int
     lib.evo_sum_partials.argtypes = [i64, ctypes.POINTER(ctypes.c_void_p), i64, vp, vp]
     lib.evo_sum_partials.restype = ctypes.c_int
+    lib.evo_attn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.evo_attn_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.evo_exp2_fma.argtypes = [vp, vp, i64, vp]
+    lib.evo_exp2_fma.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -145,6 +153,33 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _check_biases(q, mask_bias, pair_bias):
+    """mask_bias [B,S,1,1,N] and pair_bias [B,1,H,N,N]: contiguous, of q's dtype, on q's device.
+
+    The library reads both as dense arrays of those shapes, so a strided view
+    (a slice of a larger mask over rows s, say) or another dtype would be read
+    as the wrong values; such arguments are refused here instead.
+    """
+    B, S, N, H, _ = q.shape
+    for name, t, shape in (("mask_bias", mask_bias, (B, S, 1, 1, N)), ("pair_bias", pair_bias, (B, 1, H, N, N))):
+        if t is None:
+            continue
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous (pass .contiguous() of a strided view)")
+        if t.dtype != q.dtype or t.device != q.device:
+            raise ValueError(f"{name} must be of q's dtype and device")
+
+
+def _check_lse(q, lse):
+    """lse [B,S,H,N]: contiguous fp32 on q's device."""
+    B, S, N, H, _ = q.shape
+    if tuple(lse.shape) != (B, S, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous() \
+            or lse.device != q.device:
+        raise ValueError(f"lse must be a contiguous fp32 tensor of shape {(B, S, H, N)} on q's device")
+
+
 def empty_like_rows(t: torch.Tensor, dtype=None) -> torch.Tensor:
     """Uninitialised tensor with t's shape and strides (keeps the transposed-pair layout)."""
     return torch.empty_strided(t.shape, t.stride(), dtype=dtype or t.dtype, device=t.device)
@@ -155,37 +190,58 @@ def workspace_bytes(q: torch.Tensor) -> int:
     return int(lib.evo_attn_bwd_workspace_bytes(ctypes.byref(_shape(q)), DTYPES[q.dtype]))
 
 
-def evo_attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None):
-    """Forward pass; returns (out, lse).  out/lse may be passed in preallocated."""
+def evo_attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None, out_lo=None):
+    """Forward pass; returns (out, lse), or (out, lse, out_lo) when ``out_lo`` is given.
+
+    out/lse may be passed in preallocated.  ``out_lo`` (bf16 only): True to
+    allocate, or a tensor shaped and strided like out, that receives the
+    rounding residual of out (pass it on to evo_attn_bwd for an accurate D_i,
+    which is what keeps d_pair_bias's error small at large N_seq).
+    """
     lib = load_library()
     _same_strides(q, k, v, g)
     sh = _shape(q)
     B, S, N, H, C = q.shape
     if out is None:
         out = empty_like_rows(q)
+    _check_biases(q, mask_bias, pair_bias)
     if lse is None:
         lse = torch.empty((B, S, H, N), dtype=torch.float32, device=q.device)
-    for t in (mask_bias, pair_bias):
-        if t is not None and (not t.is_contiguous() or t.dtype != q.dtype):
-            raise ValueError("mask_bias / pair_bias must be contiguous and of q's dtype")
+    _check_lse(q, lse)
+    want_lo = out_lo is not None and out_lo is not False
+    if out_lo is True:
+        out_lo = empty_like_rows(out)
+    if want_lo and (out_lo.stride() != out.stride() or out_lo.dtype != out.dtype or out_lo.shape != out.shape):
+        raise ValueError("out_lo must have out's shape, strides and dtype")
     rc = lib.evo_attn_fwd(ctypes.byref(sh), DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                           ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out),
-                          ctypes.byref(_strides(out)), _ptr(lse), _stream(q.device))
+                          _ptr(out_lo) if want_lo else None, ctypes.byref(_strides(out)), _ptr(lse),
+                          _stream(q.device))
     _check("evo_attn_fwd", rc)
-    return out, lse
+    return (out, lse, out_lo) if want_lo else (out, lse)
 
 
-def evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, workspace=None):
+def _check_out_lo(out, out_lo):
+    if out_lo is not None and (out_lo.stride() != out.stride() or out_lo.dtype != out.dtype
+                               or out_lo.shape != out.shape or out_lo.device != out.device):
+        raise ValueError("out_lo must have out's shape, strides, dtype and device")
+
+
+def evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, workspace=None, out_lo=None):
     """Backward pass; returns dict(dq, dk, dv, dg, d_pair_bias).
 
     d_pair_bias is fp32 ``[B, 1, H, N, N]``.  ``grads`` may hold preallocated
-    outputs, ``workspace`` a preallocated uint8 buffer of ``workspace_bytes(q)``.
+    outputs, ``workspace`` a preallocated uint8 buffer of ``workspace_bytes(q)``,
+    ``out_lo`` the forward's rounding residual of out (or None).
     """
     lib = load_library()
     _same_strides(q, k, v, g)
     _same_strides(out, dout)
     sh = _shape(q)
     B, S, N, H, C = q.shape
+    _check_biases(q, mask_bias, pair_bias)
+    _check_lse(q, lse)
+    _check_out_lo(out, out_lo)
     grads = dict(grads or {})
     for n in ("dq", "dk", "dv", "dg"):
         if grads.get(n) is None:
@@ -197,8 +253,8 @@ def evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, w
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     rc = lib.evo_attn_bwd(ctypes.byref(sh), DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                          ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out), _ptr(dout),
-                          ctypes.byref(_strides(out)), _ptr(lse), _ptr(grads["dq"]), _ptr(grads["dk"]),
+                          ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out), _ptr(out_lo),
+                          _ptr(dout), ctypes.byref(_strides(out)), _ptr(lse), _ptr(grads["dq"]), _ptr(grads["dk"]),
                           _ptr(grads["dv"]), _ptr(grads["dg"]), ctypes.byref(_strides(grads["dq"])),
                           _ptr(grads["d_pair_bias"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
                           _stream(q.device))
@@ -206,7 +262,7 @@ def evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, w
     return grads
 
 
-def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None):
+def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads=None, out_lo=None):
     """Backward pass through evo_attn_bwd_noalloc: no workspace is passed or allocated.
 
     For callers that must not allocate device memory: the library uses its own
@@ -219,6 +275,9 @@ def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads
     _same_strides(out, dout)
     sh = _shape(q)
     B, S, N, H, C = q.shape
+    _check_biases(q, mask_bias, pair_bias)
+    _check_lse(q, lse)
+    _check_out_lo(out, out_lo)
     grads = dict(grads or {})
     for n in ("dq", "dk", "dv", "dg"):
         if grads.get(n) is None:
@@ -228,7 +287,7 @@ def evo_attn_bwd_noalloc(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads
     _same_strides(grads["dq"], grads["dk"], grads["dv"], grads["dg"])
     rc = lib.evo_attn_bwd_noalloc(ctypes.byref(sh), DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                   ctypes.byref(_strides(q)), _ptr(mask_bias), _ptr(pair_bias), _ptr(out),
-                                  _ptr(dout), ctypes.byref(_strides(out)), _ptr(lse), _ptr(grads["dq"]),
+                                  _ptr(out_lo), _ptr(dout), ctypes.byref(_strides(out)), _ptr(lse), _ptr(grads["dq"]),
                                   _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
                                   ctypes.byref(_strides(grads["dq"])), _ptr(grads["d_pair_bias"]),
                                   _stream(q.device))
@@ -389,6 +448,21 @@ def timing_collect() -> dict:
     return {name: (int(t.calls[i]), float(t.ms[i])) for i, name in enumerate(PHASES)}
 
 
+def set_wait_limit_ns(ns: int) -> int:
+    """Limit of the forward kernels' bounded waits from now on (nanoseconds); returns the previous one."""
+    return int(load_library().evo_attn_set_wait_limit_ns(int(ns)))
+
+
+def exp2_fma(x, y=None):
+    """2^x for a contiguous fp32 CUDA tensor, by the kernels' FMA-pipe exponential."""
+    if x.dtype != torch.float32 or not x.is_contiguous() or not x.is_cuda:
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    if y is None:
+        y = torch.empty_like(x)
+    _check("evo_exp2_fma", load_library().evo_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(x.device)))
+    return y
+
+
 def device_status(clear: bool = True) -> int:
     """Synchronises and returns the library's device status (0 = EVO_OK, 5 = a wait timed out)."""
     return int(load_library().evo_attn_device_status(1 if clear else 0))
@@ -399,15 +473,18 @@ class EvoformerAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, g, mask_bias, pair_bias):
-        out, lse = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias)
-        ctx.save_for_backward(q, k, v, g, mask_bias, pair_bias, out, lse)
+        if q.dtype == torch.bfloat16:
+            out, lse, out_lo = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias, out_lo=True)
+        else:
+            (out, lse), out_lo = evo_attn_fwd(q, k, v, g, mask_bias, pair_bias), None
+        ctx.save_for_backward(q, k, v, g, mask_bias, pair_bias, out, lse, out_lo)
         return out
 
     @staticmethod
     def backward(ctx, dout):
-        q, k, v, g, mask_bias, pair_bias, out, lse = ctx.saved_tensors
+        q, k, v, g, mask_bias, pair_bias, out, lse, out_lo = ctx.saved_tensors
         dout = dout if dout.stride() == out.stride() else empty_like_rows(out).copy_(dout)
-        gr = evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout)
+        gr = evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, out_lo=out_lo)
         dpb = None
         if pair_bias is not None and ctx.needs_input_grad[5]:
             dpb = gr["d_pair_bias"].to(pair_bias.dtype)

@@ -76,28 +76,29 @@ class PendingPairBiasGrad:
     backward, say), which then overlaps the transfer.
     """
 
-    def __init__(self, parts=None, work=None, out=None):
+    def __init__(self, parts=None, work=None, out=None, summer=None):
         self._parts, self._work, self._out = parts, work, out
+        self._sum = summer or A.sum_partials
 
     def wait(self) -> torch.Tensor:
         if self._work is not None:
             self._work.wait()
-            A.sum_partials(self._parts, out=self._out)
+            self._sum(self._parts, out=self._out)
             self._work = self._parts = None
         return self._out
 
 
-def attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None):
+def attn_fwd(q, k, v, g, mask_bias=None, pair_bias=None, out=None, lse=None, out_lo=None):
     """Forward of this rank's rows: evo_attn_fwd on them, no communication.
 
     q, k, v, g (and mask_bias, if any) hold this rank's rows only; pair_bias
-    is the full bias every rank shares.
+    is the full bias every rank shares.  out_lo as for evo_attn_fwd.
     """
-    return A.evo_attn_fwd(q, k, v, g, mask_bias, pair_bias, out, lse)
+    return A.evo_attn_fwd(q, k, v, g, mask_bias, pair_bias, out, lse, out_lo)
 
 
 def attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, group=None, grads=None, workspace=None,
-             async_op: bool = False):
+             async_op: bool = False, backward=None, summer=None, out_lo=None):
     """Backward of this rank's rows, with d_pair_bias summed over every rank's rows.
 
     Arguments as for evo_attn_bwd, restricted to this rank's rows (pair_bias
@@ -106,12 +107,25 @@ def attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, group=None, grads
     (a collective).  With one rank, no collective runs.  With
     ``async_op=True`` it returns (grads, pending) instead: grads["d_pair_bias"]
     holds this rank's partial until pending.wait() turns it into the sum.
+
+    ``backward`` and ``summer`` replace the library's evo_attn_bwd and
+    sum_partials (same signatures); they exist so that the exchange can be
+    exercised on CPU ranks with another implementation of the two.
     """
-    grads = A.evo_attn_bwd(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads, workspace)
+    world = _world(group)
+    if world > A.MAX_PARTIALS:
+        # refused before any kernel or collective runs, on every rank alike
+        raise ValueError(f"a row split over {world} ranks exceeds the {A.MAX_PARTIALS} partials "
+                         "evo_sum_partials adds in one call")
+    if out_lo is None:
+        grads = (backward or A.evo_attn_bwd)(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads, workspace)
+    else:
+        grads = (backward or A.evo_attn_bwd)(q, k, v, g, mask_bias, pair_bias, out, lse, dout, grads, workspace,
+                                             out_lo=out_lo)
     pending = PendingPairBiasGrad(out=grads["d_pair_bias"])
-    if _world(group) > 1:
+    if world > 1:
         parts, work = start_gather(grads["d_pair_bias"], group)
-        pending = PendingPairBiasGrad(parts, work, grads["d_pair_bias"])
+        pending = PendingPairBiasGrad(parts, work, grads["d_pair_bias"], summer)
     if async_op:
         return grads, pending
     pending.wait()

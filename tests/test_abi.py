@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "evo_attn.h")
 def header_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(evo_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(evo_[a-z0-9_]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -59,20 +59,21 @@ def test_host_argument_errors_need_no_gpu(lib):
     st = A.Strides(0, 0, 0, 0)
     sh = A.Shape(1, 2, 8, 1, 32)
     nul = None
-    rc = lib.evo_attn_fwd(None, 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, ctypes.byref(st), nul, nul)
+    rc = lib.evo_attn_fwd(None, 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, nul, ctypes.byref(st), nul,
+                          nul)
     assert rc == 1
-    rc = lib.evo_attn_fwd(ctypes.byref(sh), 7, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+    rc = lib.evo_attn_fwd(ctypes.byref(sh), 7, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, nul,
                           ctypes.byref(st), nul, nul)
     assert rc == 1                                # unknown dtype
-    rc = lib.evo_attn_fwd(ctypes.byref(sh), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+    rc = lib.evo_attn_fwd(ctypes.byref(sh), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, nul,
                           ctypes.byref(st), nul, nul)
     assert rc == 1                                # null tensors
     empty = A.Shape(1, 0, 8, 1, 32)
-    rc = lib.evo_attn_fwd(ctypes.byref(empty), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+    rc = lib.evo_attn_fwd(ctypes.byref(empty), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, nul,
                           ctypes.byref(st), nul, nul)
     assert rc == 0                                # empty call: nothing to do
     neg = A.Shape(1, -1, 8, 1, 32)
-    rc = lib.evo_attn_fwd(ctypes.byref(neg), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul,
+    rc = lib.evo_attn_fwd(ctypes.byref(neg), 0, nul, nul, nul, nul, ctypes.byref(st), nul, nul, nul, nul,
                           ctypes.byref(st), nul, nul)
     assert rc == 1
 
@@ -137,3 +138,31 @@ def test_product_path_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "evo_ref" not in text and "libevo_ref" not in text, f
+
+
+def test_binding_refuses_strided_or_mistyped_biases_before_any_call(lib):
+    """A strided mask slice (rows s0:s1 of a B = 2 mask), an fp32 pair bias with bf16 q and a
+    non-contiguous lse are refused by the binding in the forward and in both backward entry
+    points, before the library sees a pointer it would read as a dense array of the wrong values."""
+    import torch
+    B, S, N, H, C = 2, 6, 16, 2, 32
+    q = torch.zeros(B, S, N, H, C, dtype=torch.bfloat16)
+    full_mask = torch.zeros(B, 2 * S, 1, 1, N, dtype=torch.bfloat16)
+    strided_mask = full_mask[:, 2:2 + S]               # rows of a larger mask: a strided view when B > 1
+    assert not strided_mask.is_contiguous()
+    pb = torch.zeros(B, 1, H, N, N, dtype=torch.bfloat16)
+    lse = torch.zeros(B, S, H, N, dtype=torch.float32)
+    calls = (A.evo_attn_bwd, A.evo_attn_bwd_noalloc)
+    for bwd in calls:
+        with pytest.raises(ValueError, match="mask_bias must be contiguous"):
+            bwd(q, q, q, q, strided_mask, pb, q, lse, q)
+        with pytest.raises(ValueError, match="pair_bias must be of q's dtype"):
+            bwd(q, q, q, q, None, pb.float(), q, lse, q)
+        with pytest.raises(ValueError, match="pair_bias must have shape"):
+            bwd(q, q, q, q, None, pb[:, :, :1], q, lse, q)
+        with pytest.raises(ValueError, match="lse must be"):
+            bwd(q, q, q, q, None, pb, q, lse.transpose(2, 3).contiguous().transpose(2, 3), q)
+    with pytest.raises(ValueError, match="mask_bias must be contiguous"):
+        A.evo_attn_fwd(q, q, q, q, strided_mask, pb)
+    with pytest.raises(ValueError, match="lse must be"):
+        A.evo_attn_fwd(q, q, q, q, None, pb, lse=lse[:, :1])

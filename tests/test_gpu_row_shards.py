@@ -128,3 +128,40 @@ def test_one_rank_needs_no_exchange():
     assert pending.wait() is grads2["d_pair_bias"]
     torch.cuda.synchronize()
     assert torch.equal(grads2["d_pair_bias"], plain["d_pair_bias"])
+
+
+class _DoneWork:
+    """Stands in for a finished all-gather handle: wait() has nothing left to wait for."""
+
+    def __init__(self):
+        self.waited = 0
+
+    def wait(self):
+        self.waited += 1
+
+
+def test_pending_wait_sums_gathered_parts_in_place():
+    """PendingPairBiasGrad.wait() with a work handle: the branch a world > 1 backward takes.
+
+    The gathered buffer holds the per-block partials of a row split (run block
+    after block on this GPU); wait() must add them in rank order into the
+    tensor that held this rank's partial and return that very tensor, bit-equal
+    to the oracle's rank-ordered fp32 sum.
+    """
+    w = Workload("pending", 1, 7, 136, 2, 32, "bf16", "msa_row", 1.0, "frac:0.1", 17)
+    d = to_gpu(workload_inputs(w))
+    world = 3
+    parts = []
+    for rank in range(world):
+        s0, s1 = row_shards.row_range(w.S, world, rank)
+        blk = {k: (v if v is None or k == "pair_bias" else v[:, s0:s1].contiguous()) for k, v in d.items()}
+        parts.append(gpu_fwd_bwd(blk)["d_pair_bias"])
+    gathered = torch.stack(parts)                      # what the all-gather leaves in its buffer
+    mine = parts[1].clone()                            # this rank's partial, to be overwritten by the sum
+    work = _DoneWork()
+    pending = row_shards.PendingPairBiasGrad(gathered, work, mine)
+    got = pending.wait()
+    torch.cuda.synchronize()
+    assert got is mine and work.waited == 1
+    assert np.array_equal(got.cpu().numpy(), oracle.ordered_sum_f32(gathered.cpu().numpy()))
+    assert pending.wait() is mine and work.waited == 1  # a second wait() does nothing more
