@@ -17,7 +17,6 @@
 //                  nl = -1e30, so padded queries get P = 0;
 //                  pair_bias[b,h,i,j] -> biasT[b,h,j,i] (bf16), so that the
 //                  main kernel reads bias rows along its TMEM lanes (keys);
-//                  the d_pair_bias partial slabs cleared.
 //   bwd_main       CTA = (key tile j, row group g, b*H + h); loops over the
 //                  group's rows s (outer) and query tiles i (inner):
 //                    S^T  = K_j Q_i^T      dP^T = V_j (dOa_hi + dOa_lo)_i^T  (TMEM)
@@ -25,19 +24,20 @@
 //                    dS^T = P^T (dP^T - D_i)
 //                    dV_j += P^T dOa_hi_i  dK_j += dS^T Q_i         (TMEM)
 //                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
-//                    d_pair_bias partial[g][i,j] += dS (atomic add; one thread
-//                    is the only writer of each address, rows s in order)
 //                  The dS^T smem tile and the P^T TMEM tile are double-buffered
 //                  by step parity, so the dS warps write step t while the MMAs of
 //                  step t-1 still read the other buffer.
+//   dbias          d_pair_bias, summed over the rows s on chip (dbias_sm100.cuh):
+//                  one partial slab per row group, plain stores.
 //   bwd_post       one launch: dq = bf16(accumulator); d_pair_bias = sum over
-//                  g of the partials in index order (when there are several).
+//                  the row groups' slabs in group order (when there are several).
 // The result of d_pair_bias is therefore bitwise reproducible; dq's last bits
 // depend on the order of the atomic adds.
 #pragma once
 
 #include "sm100.cuh"
 #include "tma_maps.cuh"
+#include "dbias_sm100.cuh"
 
 namespace evo {
 namespace bwd {
@@ -53,24 +53,33 @@ constexpr int RT_BYTES = 4096;                    // 16 x 128 bf16 rank-term blo
 constexpr int CONST_BYTES = 4096;                 // 128 x 16 bf16 constant block, no swizzle
 // per row s (double-buffered): K, V, mask block (row 0 = mask row of s; MN-major A operand)
 constexpr int KV_K = 0, KV_V = TILE_BYTES, KV_MASK = 2 * TILE_BYTES, KVB = 2 * TILE_BYTES + RT_BYTES;
-// per step (double-buffered): Q, dOa high / low parts, transposed bias tile,
-// nl block (rows 0,1 = high/low of -lse*sqrt(C)) and -D block (rows 0,1 = high/low of -D)
-constexpr int ST_Q = 0, ST_DOH = TILE_BYTES, ST_DOL = 2 * TILE_BYTES, ST_BT = 3 * TILE_BYTES;
-constexpr int ST_NL = ST_BT + 2 * BT_BOX, ST_ND = ST_NL + RT_BYTES, STB = ST_ND + RT_BYTES;
+// Per step (query tile of a row s), two rings with different lifetimes, so that
+// the next steps' loads are not held back by the last products of this one:
+//   ring X (2 stages): transposed bias tile, dOa low part, nl block (rows 0,1 =
+//     high/low of -lse*sqrt(C)) and -D block (rows 0,1 = high/low of -D); read
+//     by the S^T / dP^T products and the dS warps' bias adds, released early
+//   ring Y (3 stages): Q and dOa high part; read also by dK and dV, released late
+constexpr int X_BT = 0, X_DOL = 2 * BT_BOX, X_NL = X_DOL + TILE_BYTES, X_ND = X_NL + RT_BYTES,
+              XB = X_ND + RT_BYTES;
+constexpr int Y_Q = 0, Y_DOH = TILE_BYTES, YB = 2 * TILE_BYTES;
+constexpr int X_STAGES = 2, Y_STAGES = 3;
 constexpr int OFF_KV = 0;
-constexpr int OFF_ST = 2 * KVB;
-constexpr int OFF_DS = OFF_ST + 2 * STB;           // dS^T tile, 2 boxes of 128 rows x 128 B
+constexpr int OFF_X = 2 * KVB;
+constexpr int OFF_Y = OFF_X + X_STAGES * XB;
+constexpr int OFF_DS = OFF_Y + Y_STAGES * YB;      // dS^T tile, 2 boxes of 128 rows x 128 B
 constexpr int DS_BYTES = 2 * BT_BOX;
 constexpr int OFF_ONES = OFF_DS + DS_BYTES;        // A operand: columns 0 and 1 equal to 1
-constexpr int OFF_RROW = OFF_ONES + CONST_BYTES;   // B operand: row 0 equal to r = bf16(sqrt(C))
+constexpr int OFF_RROW = OFF_ONES + CONST_BYTES;   // B operand: columns k = 0, 8 equal to r1, r2 (sum sqrt(C))
 constexpr int OFF_BAR = OFF_RROW + CONST_BYTES;
-// kv_full[2] kv_empty[2] q_full[2] q_empty[2] sdp_full sdp_free ds_full pt_free[2] ds_free
-// dq_full dq_free dkv_full dkv_free mma_done
-constexpr int NBARS = 19;
+// kv_full[2] kv_empty[2] x_full[2] x_empty[2] y_full[3] y_empty[3] sdp_full sdp_free ds_full[2]
+// pt_free[2] ds_free dq_full dq_free dkv_full dkv_free mma_done[3]
+constexpr int NBARS = 28;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-// Warps 0..7: two dS warpgroups (queries 0..63 / 64..127 of the tile); warp 8 TMA,
-// warp 9 MMA, warps 10, 11 idle.  The last warpgroup hands registers to the dS
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+// Warps 0..7: two dS warpgroups (queries 0..63 / 64..127 of the tile); warp 8 TMA;
+// three MMA issuers, so that no single issuing thread serialises a step's 33
+// instructions: warp 9 S^T and dP^T of the next step, warp 10 dV and dK, warp 11 dQ.  The last warpgroup hands registers to the dS
 // warpgroups: 2*128*208 + 128*88 = 384*168, the launch's register pool.
 constexpr int THREADS = 384;
 constexpr int LAUNCH_REGS = 168;
@@ -79,8 +88,8 @@ static_assert((2 * DS_REGS + CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "regi
 // TMEM columns: S^T, dP^T, two P^T buffers (bf16 pairs), dV, dK, dQ accumulators
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 384, TM_DK = 416, TM_DQ = 448, TM_COLS = 512;
 
-// Row groups for the deterministic d_pair_bias reduction: about one CTA
-// (key tile x head x batch x group) per SM of a 148-SM B200, in one wave.
+// Row groups of the main kernel: about one CTA (key tile x head x batch x
+// group) per SM of a 148-SM B200, in one wave.
 inline int num_groups(int64_t B, int64_t S, int64_t N, int64_t H) {
     const int64_t njt = (N + BK - 1) / BK;
     const int64_t base = njt * B * H;
@@ -98,8 +107,8 @@ struct MainParams {
     int gsz;             // rows s per group
     float sc2;           // log2(e) / sqrt(C)
     float rs;            // 1 / sqrt(C)
-    float r_bf16;        // bf16(sqrt(C))
-    float* part;         // [G,B,H,N,N] partials, or d_pair_bias when G == 1
+    float r_bf16;        // r1 = bf16(sqrt(C))
+    float r2_bf16;       // r2 = bf16(sqrt(C) - r1): the mask enters as (r1 + r2) * mask
     float* dq_acc;       // [B,S,N,H,C] fp32, contiguous
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -121,7 +130,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = 8, kMma = 9;
+    constexpr int kProducer = 8, kMma = 9, kMmaKV = 10, kMmaQ = 11;
     const int j0 = blockIdx.x * BK;
     const int grp = blockIdx.y;
     const int b = blockIdx.z / p.H, h = blockIdx.z % p.H;
@@ -133,35 +142,43 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t bar0 = base + OFF_BAR;
     auto kv_full = [&](int x) { return bar0 + 8u * (0 + x); };
     auto kv_empty = [&](int x) { return bar0 + 8u * (2 + x); };
-    auto q_full = [&](int x) { return bar0 + 8u * (4 + x); };
-    auto q_empty = [&](int x) { return bar0 + 8u * (6 + x); };
-    const uint32_t sdp_full = bar0 + 8u * 8, sdp_free = bar0 + 8u * 9;
-    const uint32_t ds_full = bar0 + 8u * 10;
-    auto pt_free = [&](int x) { return bar0 + 8u * (11 + x); };
-    const uint32_t ds_free = bar0 + 8u * 13;
-    const uint32_t dq_full = bar0 + 8u * 14, dq_free = bar0 + 8u * 15;
-    const uint32_t dkv_full = bar0 + 8u * 16, dkv_free = bar0 + 8u * 17;
-    const uint32_t mma_done = bar0 + 8u * 18;
+    auto x_full = [&](int x) { return bar0 + 8u * (4 + x); };
+    auto x_empty = [&](int x) { return bar0 + 8u * (6 + x); };
+    auto y_full = [&](int x) { return bar0 + 8u * (8 + x); };
+    auto y_empty = [&](int x) { return bar0 + 8u * (11 + x); };
+    const uint32_t sdp_full = bar0 + 8u * 14, sdp_free = bar0 + 8u * 15;
+    // ds_full[t & 1]: dS^T of step t in shared memory and P^T in TMEM (one barrier per step
+    // parity, because two issuers consume it and the dS warps may run a step ahead of one)
+    auto ds_full = [&](int x) { return bar0 + 8u * (16 + x); };
+    auto pt_free = [&](int x) { return bar0 + 8u * (18 + x); };
+    const uint32_t ds_free = bar0 + 8u * 20;
+    const uint32_t dq_full = bar0 + 8u * 21, dq_free = bar0 + 8u * 22;
+    const uint32_t dkv_full = bar0 + 8u * 23, dkv_free = bar0 + 8u * 24;
+    auto mma_done = [&](int x) { return bar0 + 8u * (25 + x); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(kv_full(x), 1);
-            mbar_init(kv_empty(x), 1);
-            mbar_init(q_full(x), 1);
-            mbar_init(q_empty(x), 1 + 8);
+            mbar_init(kv_empty(x), 2);            // K and V read by the S^T / dP^T issuer and the dQ issuer
+            mbar_init(x_full(x), 1);
+            mbar_init(x_empty(x), 1 + 8);         // the S^T / dP^T issuer and the dS warps (bias)
             mbar_init(pt_free(x), 1);
+            mbar_init(ds_full(x), 8);
+        }
+        for (int x = 0; x < Y_STAGES; ++x) {
+            mbar_init(y_full(x), 1);
+            mbar_init(y_empty(x), 2);             // the S^T / dP^T and the dV / dK issuers
         }
         mbar_init(sdp_full, 1);
         mbar_init(sdp_free, 8);
-        mbar_init(ds_full, 8);
-        mbar_init(ds_free, 1);
+        mbar_init(ds_free, 2);                    // dK and dQ read the dS^T tile
         mbar_init(dq_full, 1);
         mbar_init(dq_free, 8);
         mbar_init(dkv_full, 1);
         mbar_init(dkv_free, 8);
-        mbar_init(mma_done, 1);
+        for (int x = 0; x < 3; ++x) mbar_init(mma_done(x), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -188,17 +205,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         zero(OFF_RROW, CONST_BYTES);
         for (int x = 0; x < 2; ++x) {
             zero(OFF_KV + x * KVB + KV_MASK, RT_BYTES);
-            zero(OFF_ST + x * STB + ST_NL, RT_BYTES);
-            zero(OFF_ST + x * STB + ST_ND, RT_BYTES);
+            zero(OFF_X + x * XB + X_NL, RT_BYTES);
+            zero(OFF_X + x * XB + X_ND, RT_BYTES);
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (t < 128) {
             const uint16_t one = 0x3F80u;
             const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
+            const uint16_t rb2 = (uint16_t)(__float_as_uint(p.r2_bf16) >> 16);
             uint8_t* o = gbase + OFF_ONES + (t % 8) * 16 + (t / 8) * 256;
             reinterpret_cast<uint16_t*>(o)[0] = one;   // k = 0
             reinterpret_cast<uint16_t*>(o)[1] = one;   // k = 1
             *reinterpret_cast<uint16_t*>(gbase + OFF_RROW + (t % 8) * 16 + (t / 8) * 256) = rb;
+            *reinterpret_cast<uint16_t*>(gbase + OFF_RROW + (t % 8) * 16 + (t / 8) * 256 + 128) = rb2;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -211,51 +230,63 @@ __global__ void __launch_bounds__(THREADS, 1)
         regs_decrease<CONTROL_REGS>();
         // ---------------------------------------------------------------- producer
         if (lane == 0 && T > 0) {
-            int kv_issued[2] = {0, 0}, q_issued[2] = {0, 0};
+            int kv_issued[2] = {0, 0}, x_issued[X_STAGES] = {}, y_issued[Y_STAGES] = {};
             bool ok = true;
             for (int si = 0; si < ns && ok; ++si) {
                 const int s = s_begin + si, x = si & 1;
                 const uint32_t kb = base + OFF_KV + x * KVB;
                 if (si >= 2) ok = mbar_wait(kv_empty(x), ((si >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01);
                 if (!ok) break;
-                mbar_arrive_expect_tx(kv_full(x), 2 * TILE_BYTES + (HAS_MASK ? 256 : 0));
+                mbar_arrive_expect_tx(kv_full(x), 2 * TILE_BYTES + (HAS_MASK ? 512 : 0));
                 tma_load_5d(kb + KV_K, &tm_k, kv_full(x), 0, j0, h, s, b);
                 tma_load_5d(kb + KV_V, &tm_v, kv_full(x), 0, j0, h, s, b);
-                if (HAS_MASK) {   // mask row of s into row 0 of the two 64-key atoms of the A block
+                if (HAS_MASK) {   // mask row of s into rows 0 and 8 of the two 64-key halves of the A block
                     tma_load_3d(kb + KV_MASK, &tm_mask, kv_full(x), j0, s, b);
+                    tma_load_3d(kb + KV_MASK + 1024, &tm_mask, kv_full(x), j0, s, b);
                     tma_load_3d(kb + KV_MASK + 2048, &tm_mask, kv_full(x), j0 + 64, s, b);
+                    tma_load_3d(kb + KV_MASK + 3072, &tm_mask, kv_full(x), j0 + 64, s, b);
                 }
                 ++kv_issued[x];
                 for (int it = 0; it < ni; ++it) {
-                    const int t = si * ni + it, st = t & 1, i0 = it * BQ;
-                    const uint32_t sb = base + OFF_ST + st * STB;
-                    if (t >= 2) ok = mbar_wait(q_empty(st), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
+                    const int t = si * ni + it, i0 = it * BQ;
+                    const int xs = t % X_STAGES, ys = t % Y_STAGES;
+                    const uint32_t xb = base + OFF_X + xs * XB, yb = base + OFF_Y + ys * YB;
+                    if (t >= X_STAGES)
+                        ok = mbar_wait(x_empty(xs), ((t / X_STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(q_full(st), 3 * TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 4 * 256);
-                    tma_load_5d(sb + ST_Q, &tm_q, q_full(st), 0, i0, h, s, b);
-                    tma_load_5d(sb + ST_DOH, &tm_doa, q_full(st), 0, i0, h, s, b);
-                    tma_load_5d(sb + ST_DOL, &tm_dol, q_full(st), 0, i0, h, s, b);
+                    mbar_arrive_expect_tx(x_full(xs), TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 4 * 256);
                     if (HAS_BIAS) {
-                        tma_load_4d(sb + ST_BT, &tm_bt, q_full(st), i0, j0, h, b);
-                        tma_load_4d(sb + ST_BT + BT_BOX, &tm_bt, q_full(st), i0 + 64, j0, h, b);
+                        tma_load_4d(xb + X_BT, &tm_bt, x_full(xs), i0, j0, h, b);
+                        tma_load_4d(xb + X_BT + BT_BOX, &tm_bt, x_full(xs), i0 + 64, j0, h, b);
                     }
+                    tma_load_5d(xb + X_DOL, &tm_dol, x_full(xs), 0, i0, h, s, b);
                     // rows 0..1 (high, low) of the two 64-query atoms of the nl and -D blocks
-                    tma_load_5d(sb + ST_NL, &tm_nl, q_full(st), i0, 0, h, s, b);
-                    tma_load_5d(sb + ST_NL + 2048, &tm_nl, q_full(st), i0 + 64, 0, h, s, b);
-                    tma_load_5d(sb + ST_ND, &tm_d, q_full(st), i0, 0, h, s, b);
-                    tma_load_5d(sb + ST_ND + 2048, &tm_d, q_full(st), i0 + 64, 0, h, s, b);
-                    ++q_issued[st];
+                    tma_load_5d(xb + X_NL, &tm_nl, x_full(xs), i0, 0, h, s, b);
+                    tma_load_5d(xb + X_NL + 2048, &tm_nl, x_full(xs), i0 + 64, 0, h, s, b);
+                    tma_load_5d(xb + X_ND, &tm_d, x_full(xs), i0, 0, h, s, b);
+                    tma_load_5d(xb + X_ND + 2048, &tm_d, x_full(xs), i0 + 64, 0, h, s, b);
+                    ++x_issued[xs];
+                    if (t >= Y_STAGES)
+                        ok = mbar_wait(y_empty(ys), ((t / Y_STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x05);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(y_full(ys), 2 * TILE_BYTES);
+                    tma_load_5d(yb + Y_Q, &tm_q, y_full(ys), 0, i0, h, s, b);
+                    tma_load_5d(yb + Y_DOH, &tm_doa, y_full(ys), 0, i0, h, s, b);
+                    ++y_issued[ys];
                 }
             }
             volatile int no_abort = 0;
-            for (int x = 0; x < 2; ++x) {
+            for (int x = 0; x < 2; ++x)
                 if (kv_issued[x]) mbar_wait(kv_full(x), (kv_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x03);
-                if (q_issued[x]) mbar_wait(q_full(x), (q_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
-            }
+            for (int x = 0; x < X_STAGES; ++x)
+                if (x_issued[x]) mbar_wait(x_full(x), (x_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
+            for (int x = 0; x < Y_STAGES; ++x)
+                if (y_issued[x]) mbar_wait(y_full(x), (y_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x06);
         }
-    } else if (warp == kMma) {
+    } else if (warp == kMma || warp == kMmaKV || warp == kMmaQ) {
         regs_decrease<CONTROL_REGS>();
-        // ---------------------------------------------------------------- MMA issuer
+        // ---------------------------------------------------------------- MMA issuers
+        const int role = warp - kMma;            // 0: S^T, dP^T   1: dV, dK   2: dQ
         if (lane == 0 && T > 0) {
             constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // S^T, dP^T
             constexpr uint32_t ID_RT = idesc_bf16(BK, BQ, false, true);    // ones x rank-term block
@@ -263,80 +294,87 @@ __global__ void __launch_bounds__(THREADS, 1)
             constexpr uint32_t ID_KV = idesc_bf16(BK, HD, false, true);    // dV, dK (B MN-major)
             constexpr uint32_t ID_Q = idesc_bf16(BQ, HD, true, true);      // dQ (A and B MN-major)
             bool ok = true;
-            auto issue_sdp = [&](int t) -> bool {
-                const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
-                if (it == 0 && !mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x11)) return false;
-                if (!mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x12)) return false;
-                if (t > 0 && !mbar_wait(sdp_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x13)) return false;
-                tc_fence_after();
-                const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
-                // S^T = K Q^T - lse*sqrt(C) (+ r * mask_j)
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    mma_ss(tmem + TM_ST, smem_desc(kb + KV_K + kk * 32, 16, 512, kSw64),
-                           smem_desc(sb + ST_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-                mma_ss(tmem + TM_ST, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
-                       smem_desc(sb + ST_NL, 2048, 1024, kSw128), ID_RT, 1u);
-                if (HAS_MASK)
-                    mma_ss(tmem + TM_ST, smem_desc(kb + KV_MASK, 2048, 1024, kSw128),
-                           smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
-                // dP^T = V (dOa_hi + dOa_lo)^T - D
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
-                           smem_desc(sb + ST_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
-                           smem_desc(sb + ST_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
-                mma_ss(tmem + TM_DPT, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
-                       smem_desc(sb + ST_ND, 2048, 1024, kSw128), ID_RT, 1u);
-                mma_commit(sdp_full);
-                return true;
-            };
-            ok = issue_sdp(0);
+            const uint32_t ds = base + OFF_DS;
             for (int t = 0; ok && t < T; ++t) {
                 const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
-                if (t + 1 < T) ok = issue_sdp(t + 1);
-                if (!ok) break;
-                ok = mbar_wait(ds_full, t & 1, abort_flag, kTimeoutBase | 0x14);
-                if (ok && it == 0 && si > 0) ok = mbar_wait(dkv_free, (si - 1) & 1, abort_flag, kTimeoutBase | 0x15);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t kb = base + OFF_KV + x * KVB, sb = base + OFF_ST + st * STB;
-                const int pb = t & 1;                    // P^T buffer of this step
-                const uint32_t ds = base + OFF_DS;
+                const int xs = t % X_STAGES, ys = t % Y_STAGES;
+                const uint32_t kb = base + OFF_KV + x * KVB, xb = base + OFF_X + xs * XB, yb = base + OFF_Y + ys * YB;
+                if (role == 0) {
+                    // S^T = K Q^T - lse*sqrt(C) (+ (r1 + r2) * mask_j);  dP^T = V (dOa_hi + dOa_lo)^T - D.
+                    // Step t's products are issued as soon as the dS warps hold step t-1's in registers.
+                    if (it == 0) ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x11);
+                    if (ok) ok = mbar_wait(x_full(xs), (t / X_STAGES) & 1, abort_flag, kTimeoutBase | 0x12);
+                    if (ok) ok = mbar_wait(y_full(ys), (t / Y_STAGES) & 1, abort_flag, kTimeoutBase | 0x1D);
+                    if (ok && t > 0) ok = mbar_wait(sdp_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x13);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk)     // dV_j += P^T dOa_hi
-                    mma_ts(tmem + TM_DV, tmem + TM_PT + pb * 64 + kk * 8,
-                           smem_desc(sb + ST_DOH + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(pt_free(pb));
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        mma_ss(tmem + TM_ST, smem_desc(kb + KV_K + kk * 32, 16, 512, kSw64),
+                               smem_desc(yb + Y_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                    mma_ss(tmem + TM_ST, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                           smem_desc(xb + X_NL, 2048, 1024, kSw128), ID_RT, 1u);
+                    if (HAS_MASK)
+                        mma_ss(tmem + TM_ST, smem_desc(kb + KV_MASK, 2048, 1024, kSw128),
+                               smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
 #pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk) {   // dK_j += dS^T Q
-                    const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
-                    mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128),
-                           smem_desc(sb + ST_Q + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
-                           (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                if (t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x16);
-                if (!ok) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
+                               smem_desc(yb + Y_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)     // dQ_i = dS K_j
-                    mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
-                           smem_desc(kb + KV_K + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
-                mma_commit(ds_free);
-                mma_commit(dq_full);
-                mma_commit(q_empty(st));
-                if (it == ni - 1) {
-                    mma_commit(dkv_full);
-                    mma_commit(kv_empty(x));
+                    for (int kk = 0; kk < HD / 16; ++kk)
+                        mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
+                               smem_desc(xb + X_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
+                    mma_ss(tmem + TM_DPT, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                           smem_desc(xb + X_ND, 2048, 1024, kSw128), ID_RT, 1u);
+                    mma_commit(sdp_full);
+                    mma_commit(x_empty(xs));
+                    mma_commit(y_empty(ys));
+                    if (it == ni - 1) mma_commit(kv_empty(x));
+                } else if (role == 1) {
+                    // dV_j += P^T dOa_hi;  dK_j += dS^T Q
+                    ok = mbar_wait(y_full(ys), (t / Y_STAGES) & 1, abort_flag, kTimeoutBase | 0x14);
+                    if (ok) ok = mbar_wait(ds_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x15);
+                    if (ok && it == 0 && si > 0) ok = mbar_wait(dkv_free, (si - 1) & 1, abort_flag, kTimeoutBase | 0x16);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int pb = t & 1;                // P^T buffer of this step
+#pragma unroll
+                    for (int kk = 0; kk < BQ / 16; ++kk)
+                        mma_ts(tmem + TM_DV, tmem + TM_PT + pb * 64 + kk * 8,
+                               smem_desc(yb + Y_DOH + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(pt_free(pb));
+#pragma unroll
+                    for (int kk = 0; kk < BQ / 16; ++kk) {
+                        const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
+                        mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128),
+                               smem_desc(yb + Y_Q + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(ds_free);
+                    mma_commit(y_empty(ys));
+                    if (it == ni - 1) mma_commit(dkv_full);
+                } else {
+                    // dQ_i = dS K_j
+                    if (it == 0) ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x17);
+                    if (ok) ok = mbar_wait(ds_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x18);
+                    if (ok && t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x19);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
+                               smem_desc(kb + KV_K + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
+                    mma_commit(ds_free);
+                    mma_commit(dq_full);
+                    if (it == ni - 1) mma_commit(kv_empty(x));
                 }
             }
-            mma_commit(mma_done);
+            // Drain: every MMA issued by this thread has finished before TMEM is released.
+            mma_commit(mma_done(role));
             volatile int no_abort = 0;
-            mbar_wait(mma_done, 0, &no_abort, kTimeoutBase | 0x17);
+            mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x1A + role));
         }
     } else if (warp < 8) {
         regs_increase<DS_REGS>();
@@ -350,8 +388,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
         const uint64_t SC2 = f2(p.sc2, p.sc2);
         const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
-        // this group's slab of the partial sums (the output itself when there is one group)
-        float* part = p.part + ((int64_t)grp * p.B * p.H + (int64_t)b * p.H + h) * p.N * p.N;
         bool ok = true;
 
         auto drain_dq = [&](int t) -> bool {     // dQ rows of step t: lanes = queries
@@ -401,12 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         };
 
         for (int t = 0; t < T; ++t) {
-            const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
-            const int i0 = it * BQ;
-            if (it == 0) {
-                // the mask block of this row is read by the MMA only; no thread waits on kv_full
-                (void)x;
-            }
+            const int si = t / ni, it = t - si * ni, st = t & 1;
             ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
             if (!ok) break;
             tc_fence_after();
@@ -421,21 +452,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int c = 0; c < 64; ++c) sv[c] = __float_as_uint(-INFINITY);
             }
 
-            ok = mbar_wait(q_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x25);
+            const int xs = t % X_STAGES;
+            ok = mbar_wait(x_full(xs), (t / X_STAGES) & 1, abort_flag, kTimeoutBase | 0x25);
             const int pb = t & 1;                // P^T buffer of this step
             if (ok && t >= 2) ok = mbar_wait(pt_free(pb), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t sb = base + OFF_ST + st * STB;
-            const uint8_t* bt_ptr = gbase + (sb - base) + ST_BT + wg * BT_BOX + r * 128;
+            const uint8_t* bt_ptr = gbase + OFF_X + xs * XB + X_BT + wg * BT_BOX + r * 128;
             const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * 32;
-            // d_pair_bias partial (zeroed before the launch).  Each address of this
-            // group's slab is updated by exactly one thread, in row order s, with
-            // fire-and-forget atomic adds; same-thread atomics to one address are
-            // performed in program order, so the sum is bitwise reproducible.
-            const int ivalid = jvalid ? p.N - i0 - wg * 64 : 0;   // queries of this half inside N
-            float* col = part + (int64_t)(i0 + wg * 64) * p.N + j;
-            const int64_t rstride = p.N;
             // P = exp2(S^T * sc2 + bias * log2e) (S^T already holds -lse and the mask),
             // dS = P * dP^T (dP^T already holds -D); two columns per op
             uint32_t dk2[32];
@@ -462,22 +486,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt_addr + q * 4),
                              "r"(pk4[0]), "r"(pk4[1]), "r"(pk4[2]), "r"(pk4[3]));
-                // (no "memory" clobber: nothing in this kernel reads the slab)
-                if (ivalid >= 64) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (q * 8 + e) * rstride),
-                                     "f"(dsq[e]));
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (q * 8 + e < ivalid)
-                            asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(col + (q * 8 + e) * rstride),
-                                         "f"(dsq[e]));
-                }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(q_empty(st));           // bias tile of this stage consumed
+            if (lane == 0) mbar_arrive(x_empty(xs));           // bias tile of this stage consumed
             if (t > 0) ok = mbar_wait(ds_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x27);
             if (!ok) break;
             const uint32_t ds_row = base + OFF_DS + wg * BT_BOX + r * 128;
@@ -492,7 +503,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(ds_full);
+            if (lane == 0) mbar_arrive(ds_full(st));
 
             // The previous step's dQ and (at a row change) the previous row's dK/dV
             // are drained here, after this step's exponentials, so the MMAs that
@@ -523,6 +534,7 @@ struct PreParams {
     int B, S, N, H, n_pad;
     float sqrt_c;
     const __nv_bfloat16* out; const __nv_bfloat16* dout; Strides os;
+    const __nv_bfloat16* out_lo;   // the forward's rounding residual of out (strides os), or null
     const __nv_bfloat16* g; Strides in;
     const float* lse;
     __nv_bfloat16* dg; Strides gs;
@@ -575,16 +587,19 @@ __device__ __forceinline__ void pre_rows(const PreParams& p, int blk, int nblk) 
             s = (int)((t / ((int64_t)p.H * p.N)) % p.S);
             b = (int)(t / ((int64_t)p.H * p.N * p.S));
         }
-        const uint4 ow = reinterpret_cast<const uint4*>(p.out + p.os.off(b, s, i, h))[part];
+        const int64_t oo = p.os.off(b, s, i, h);
+        const uint4 ow = reinterpret_cast<const uint4*>(p.out + oo)[part];
+        const uint4 lw = p.out_lo ? reinterpret_cast<const uint4*>(p.out_lo + oo)[part] : make_uint4(0u, 0u, 0u, 0u);
         const uint4 dw = reinterpret_cast<const uint4*>(p.dout + p.os.off(b, s, i, h))[part];
         const uint4 gw = reinterpret_cast<const uint4*>(p.g + p.in.off(b, s, i, h))[part];
         const uint32_t ov[4] = {ow.x, ow.y, ow.z, ow.w}, dv[4] = {dw.x, dw.y, dw.z, dw.w},
-                       gv[4] = {gw.x, gw.y, gw.z, gw.w};
+                       gv[4] = {gw.x, gw.y, gw.z, gw.w}, lov[4] = {lw.x, lw.y, lw.z, lw.w};
         uint32_t dgv[4], hv[4], lv[4];
         float D = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float o0 = bf16lo(ov[e]), o1 = bf16hi(ov[e]);
+            // out as the forward computed it in fp32: the stored bf16 plus its rounding residual
+            const float o0 = bf16lo(ov[e]) + bf16lo(lov[e]), o1 = bf16hi(ov[e]) + bf16hi(lov[e]);
             const float d0 = bf16lo(dv[e]), d1 = bf16hi(dv[e]);
             const float s0 = __fdividef(1.0f, 1.0f + __expf(-bf16lo(gv[e]))),
                         s1 = __fdividef(1.0f, 1.0f + __expf(-bf16hi(gv[e])));
@@ -633,33 +648,22 @@ __device__ __forceinline__ void transpose_tile(const __nv_bfloat16* __restrict__
 }
 
 // The backward's preparation in one launch, by block range: the per-row pass
-// (pre_rows), the pair-bias transpose (one tile per block) and the clearing of
-// the d_pair_bias partial slabs.
+// (pre_rows) and the pair-bias transpose (one tile per block).
 struct PrepParams {
     PreParams pre;
     int nb_pre;
     const __nv_bfloat16* bias;
     __nv_bfloat16* biast;
     int nb_tr;                // transpose tiles (0 without a pair bias)
-    float4* zero;             // partial slabs to clear
-    int64_t n_zero4;
 };
 
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams pp) {
-    int blk = blockIdx.x;
+    const int blk = blockIdx.x;
     if (blk < pp.nb_pre) {
         pre_rows(pp.pre, blk, pp.nb_pre);
         return;
     }
-    blk -= pp.nb_pre;
-    if (blk < pp.nb_tr) {
-        transpose_tile(pp.bias, pp.biast, pp.pre.N, blk);
-        return;
-    }
-    blk -= pp.nb_tr;
-    const int nb_zero = (int)gridDim.x - pp.nb_pre - pp.nb_tr;
-    for (int64_t t = (int64_t)blk * blockDim.x + threadIdx.x; t < pp.n_zero4; t += (int64_t)nb_zero * blockDim.x)
-        pp.zero[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+    transpose_tile(pp.bias, pp.biast, pp.pre.N, blk - pp.nb_pre);
 }
 
 struct PostParams {
@@ -717,7 +721,7 @@ struct Call {
     evo_shape_t shape;
     const void *q, *k, *v, *g;
     evo_strides_t in;
-    const void *mask, *bias, *out, *dout;
+    const void *mask, *bias, *out, *out_lo, *dout;
     evo_strides_t os;
     const float* lse;
     void *dq, *dk, *dv, *dg;
@@ -725,7 +729,9 @@ struct Call {
     float* dbias;
     char* ws;
     size_t d_off, nl_off, doa_off, dol_off, dqacc_off, biast_off, part_off;
-    int groups;
+    int groups;        // row groups of the main kernel (parallelism only)
+    int db_groups;     // row groups of the d_pair_bias kernel: partial slabs at part_off when > 1
+    uint64_t wait_ns;  // limit of the d_pair_bias kernel's waits
 };
 
 inline bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -754,6 +760,25 @@ inline cudaError_t launch_main(const CUtensorMap* m, const MainParams& mp, dim3 
     return cudaGetLastError();
 }
 
+template <bool HM, bool HB>
+inline cudaError_t launch_dbias(const CUtensorMap* m, const dbias::Params& dp, int grid, cudaStream_t stream) {
+    auto kern = dbias::dbias_kernel<HM, HB>;
+    static cudaError_t attr =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dbias::SMEM_BYTES);
+    if (attr != cudaSuccess) return attr;
+    static int regs = [&] {
+        cudaFuncAttributes fa{};
+        return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
+    }();
+    if (regs != dbias::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    {
+        timing::Scope t(EVO_PHASE_BWD_DBIAS, stream);
+        kern<<<grid, dbias::THREADS, dbias::SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
+                                                                  m[8], dp);
+    }
+    return cudaGetLastError();
+}
+
 inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     const evo_shape_t& sh = c.shape;
     *launched = 0;
@@ -764,6 +789,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     for (const void* ptr : {c.q, c.k, c.v, c.g, c.out, c.dout, (const void*)c.dq, (const void*)c.dk,
                             (const void*)c.dv, (const void*)c.dg})
         if (!aligned16(ptr)) return EVO_ERR_UNSUPPORTED;
+    if (c.out_lo && !aligned16(c.out_lo)) return EVO_ERR_UNSUPPORTED;
     if ((c.mask && !aligned16(c.mask)) || (c.bias && !aligned16(c.bias)) || !aligned16(c.dbias))
         return EVO_ERR_UNSUPPORTED;
 
@@ -775,19 +801,19 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     __nv_bfloat16* dol = reinterpret_cast<__nv_bfloat16*>(c.ws + c.dol_off);
     float* dq_acc = reinterpret_cast<float*>(c.ws + c.dqacc_off);
     __nv_bfloat16* biasT = reinterpret_cast<__nv_bfloat16*>(c.ws + c.biast_off);
-    float* part = c.groups > 1 ? reinterpret_cast<float*>(c.ws + c.part_off) : c.dbias;
+    float* part = c.db_groups > 1 ? reinterpret_cast<float*>(c.ws + c.part_off) : c.dbias;
 
     const int64_t rows = (int64_t)B * S * N * H;
     PreParams pp{};
     pp.B = B; pp.S = S; pp.N = N; pp.H = H; pp.n_pad = n_pad;
     pp.sqrt_c = sqrtf((float)HD);
     pp.out = static_cast<const __nv_bfloat16*>(c.out); pp.dout = static_cast<const __nv_bfloat16*>(c.dout);
+    pp.out_lo = static_cast<const __nv_bfloat16*>(c.out_lo);
     pp.os = Strides{c.os.b, c.os.s, c.os.n, c.os.h};
     pp.g = static_cast<const __nv_bfloat16*>(c.g); pp.in = Strides{c.in.b, c.in.s, c.in.n, c.in.h};
     pp.lse = c.lse; pp.dg = static_cast<__nv_bfloat16*>(c.dg); pp.gs = Strides{c.gs.b, c.gs.s, c.gs.n, c.gs.h};
     pp.doa_hi = doa; pp.doa_lo = dol; pp.nl = nl; pp.nd = nd; pp.dq_acc = dq_acc;
-    // one launch: per-row pass, pair-bias transpose, and clearing of the partial
-    // slabs (or of the output itself), which accumulate by atomic adds from zero
+    // one launch: per-row pass and pair-bias transpose
     PrepParams prep{};
     prep.pre = pp;
     prep.nb_pre = grid_for((rows + (int64_t)B * S * H * (n_pad - N)) * PRE_LANES, 256);
@@ -795,10 +821,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     prep.biast = biasT;
     const int nt = (N + 31) / 32;
     prep.nb_tr = c.bias ? nt * nt * B * H : 0;
-    prep.zero = reinterpret_cast<float4*>(part);
-    prep.n_zero4 = (int64_t)c.groups * B * H * N * N / 4;   // N % 8 == 0: whole float4s
-    const int nb_zero = grid_for(prep.n_zero4, 256);
-    bwd_prep_kernel<<<prep.nb_pre + prep.nb_tr + nb_zero, 256, 0, stream>>>(prep);
+    bwd_prep_kernel<<<prep.nb_pre + prep.nb_tr, 256, 0, stream>>>(prep);
     ++*launched;
 
     // tensor maps: q, k, v, dOa high, dOa low, transposed bias, mask, nl rows, -D rows
@@ -824,7 +847,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     mp.sc2 = EVO_LOG2E / sqrtf((float)HD);
     mp.rs = 1.0f / sqrtf((float)HD);
     mp.r_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)HD)));
-    mp.part = part;
+    mp.r2_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)HD) - mp.r_bf16));
     mp.dq_acc = dq_acc;
     mp.dk = static_cast<__nv_bfloat16*>(c.dk);
     mp.dv = static_cast<__nv_bfloat16*>(c.dv);
@@ -839,11 +862,39 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     if (e != cudaSuccess) return EVO_ERR_CUDA;
     ++*launched;
 
+    // d_pair_bias: row sums on chip, one slab per row group (or the output itself)
+    dbias::Params dp{};
+    dp.B = B; dp.S = S; dp.N = N; dp.H = H;
+    dp.n_t = (N + dbias::BQ - 1) / dbias::BQ;
+    const int GD = c.db_groups;
+    dp.gsz = (S + GD - 1) / GD;
+    dp.groups = (S + dp.gsz - 1) / dp.gsz;
+    if (dp.groups != GD) return EVO_ERR_UNSUPPORTED;      // the workspace was sized for GD slabs
+    const int64_t items = (int64_t)B * H * dp.n_t * dp.n_t * GD;
+    if (items > 0x7fffffff) return EVO_ERR_UNSUPPORTED;
+    dp.n_items = (int)items;
+    dp.sc2 = mp.sc2;
+    dp.r_bf16 = mp.r_bf16;
+    dp.r2_bf16 = mp.r2_bf16;
+    dp.out = part;
+    dp.wait_ns = c.wait_ns;
+    int sms = 0, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    const int dgrid = (int)std::min<int64_t>(items, sms);
+    if (c.mask && c.bias) e = launch_dbias<true, true>(m, dp, dgrid, stream);
+    else if (c.mask) e = launch_dbias<true, false>(m, dp, dgrid, stream);
+    else if (c.bias) e = launch_dbias<false, true>(m, dp, dgrid, stream);
+    else e = launch_dbias<false, false>(m, dp, dgrid, stream);
+    if (e == cudaErrorInvalidConfiguration) return EVO_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return EVO_ERR_CUDA;
+    ++*launched;
+
     PostParams qp{};
     qp.B = B; qp.S = S; qp.N = N; qp.H = H;
     qp.dq_acc = dq_acc; qp.dq = static_cast<__nv_bfloat16*>(c.dq); qp.gs = mp.gs;
-    qp.part = part; qp.groups = G; qp.dbias = c.dbias;
-    bwd_post_kernel<<<grid_for(rows * PRE_LANES + (G > 1 ? (int64_t)B * H * N * N / 4 : 0), 256), 256, 0, stream>>>(qp);
+    qp.part = part; qp.groups = GD; qp.dbias = c.dbias;
+    bwd_post_kernel<<<grid_for(rows * PRE_LANES + (GD > 1 ? (int64_t)B * H * N * N / 4 : 0), 256), 256, 0, stream>>>(qp);
     ++*launched;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }

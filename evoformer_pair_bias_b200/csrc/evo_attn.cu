@@ -35,6 +35,18 @@ namespace {
 using evo::Strides;
 
 std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_limit_ns{EVO_WAIT_LIMIT_NS};
+
+// 2^x through the FMA-pipe exponential of the attention kernels, two values per call.
+__global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n;
+         i += 2 * (int64_t)gridDim.x * blockDim.x) {
+        const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.0f;
+        const uint64_t r = evo::sm100::exp2_poly2(evo::sm100::f2(a, b));
+        y[i] = evo::sm100::f2lo(r);
+        if (i + 1 < n) y[i + 1] = evo::sm100::f2hi(r);
+    }
+}
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -129,11 +141,12 @@ evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p,
 constexpr int kFwdNsub = 2;
 
 evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const void* v, const void* g,
-                      const evo_strides_t& in, const void* mask, const void* bias, void* out,
+                      const evo_strides_t& in, const void* mask, const void* bias, void* out, void* out_lo,
                       const evo_strides_t& os, float* lse, cudaStream_t stream) {
     if (sh.C != evo::fwd::HD || sh.N % 8 != 0) return EVO_ERR_UNSUPPORTED;
     if (!strides_mult(&in, 8) || !strides_mult(&os, 8)) return EVO_ERR_UNSUPPORTED;
     for (const void* ptr : {q, k, v, g, (const void*)out}) if (!aligned(ptr, 16)) return EVO_ERR_UNSUPPORTED;
+    if (out_lo && !aligned(out_lo, 16)) return EVO_ERR_UNSUPPORTED;
     if ((mask && !aligned(mask, 16)) || (bias && !aligned(bias, 16))) return EVO_ERR_UNSUPPORTED;
     const int64_t n_it = (sh.N + evo::fwd::BM - 1) / evo::fwd::BM;
     const int64_t n_sg = (sh.S + kFwdNsub - 1) / kFwdNsub;
@@ -155,11 +168,14 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
     p.n_items = (int)n_items;
     p.scale = 1.0f / sqrtf((float)sh.C);
     p.r_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)sh.C)));
+    p.r2_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)sh.C) - p.r_bf16));
     p.g = static_cast<const __nv_bfloat16*>(g);
     p.in = to_strides(in);
     p.out = static_cast<__nv_bfloat16*>(out);
+    p.out_lo = static_cast<__nv_bfloat16*>(out_lo);
     p.os = to_strides(os);
     p.lse = lse;
+    p.wait_ns = g_wait_limit_ns.load();
     if (mask && bias) return launch_fwd_bf16<kFwdNsub, true, true>(maps, p, stream);
     if (mask) return launch_fwd_bf16<kFwdNsub, true, false>(maps, p, stream);
     if (bias) return launch_fwd_bf16<kFwdNsub, false, true>(maps, p, stream);
@@ -169,7 +185,7 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
 // ---------------------------------------------------------------- backward
 struct BwdWorkspace {
     size_t d_off, nl_off, doa_off, dol_off, dqacc_off, biast_off, part_off, total;
-    int groups;
+    int groups, db_groups;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -187,6 +203,9 @@ BwdWorkspace bwd_workspace(const evo_shape_t& sh, evo_dtype_t dt) {
         const size_t padded_rows = (size_t)sh.B * sh.S * sh.H * (size_t)((sh.N + 127) / 128 * 128);
         off = align256(w.d_off + padded_rows * 4);
         w.groups = evo::bwd::num_groups(sh.B, sh.S, sh.N, sh.H);
+        // the d_pair_bias kernel's row groups, chosen for a 148-SM B200 (a pure function
+        // of the shape, so that the workspace size never depends on the device)
+        w.db_groups = evo::dbias::num_groups(sh.B, sh.S, sh.N, sh.H, 148);
         w.nl_off = off;
         off = align256(off + padded_rows * 4);
         w.doa_off = off;
@@ -198,7 +217,7 @@ BwdWorkspace bwd_workspace(const evo_shape_t& sh, evo_dtype_t dt) {
         w.biast_off = off;
         off = align256(off + pair * 2);
         w.part_off = off;
-        off = align256(off + pair * 4 * (size_t)(w.groups > 1 ? w.groups : 0));
+        off = align256(off + pair * 4 * (size_t)(w.db_groups > 1 ? w.db_groups : 0));
     }
     w.total = off;
     return w;
@@ -355,6 +374,18 @@ const char* evo_status_string(evo_status_t s) {
 
 int evo_attn_version(void) { return EVO_VERSION; }
 
+uint64_t evo_attn_set_wait_limit_ns(uint64_t ns) { return g_wait_limit_ns.exchange(ns); }
+
+evo_status_t evo_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return EVO_ERR_INVALID_ARG;
+    if (n == 0) return EVO_OK;
+    if (!aligned(x, 4) || !aligned(y, 4)) return EVO_ERR_INVALID_ARG;
+    const int blocks = (int)std::min<int64_t>((n + 511) / 512, 148 * 8);
+    exp2_fma_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
 uint64_t evo_attn_launch_count(void) { return g_launches.load(); }
 
 evo_status_t evo_attn_timing_enable(int on) { return evo::timing::enable(on); }
@@ -380,7 +411,7 @@ size_t evo_attn_bwd_workspace_bytes(const evo_shape_t* shape, evo_dtype_t dtype)
 
 evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
                           const void* v, const void* g, const evo_strides_t* in_str, const void* mask_bias,
-                          const void* pair_bias, void* out, const evo_strides_t* out_str, float* lse,
+                          const void* pair_bias, void* out, void* out_lo, const evo_strides_t* out_str, float* lse,
                           void* stream) {
     evo_status_t st = check_shape(shape);
     if (st != EVO_OK) return st;
@@ -390,6 +421,7 @@ evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
     if (!q || !k || !v || !g || !out || !lse) return EVO_ERR_INVALID_ARG;
     if (!non_overlapping(*shape, *out_str)) return EVO_ERR_INVALID_ARG;
     if (!aligned(lse, 4)) return EVO_ERR_INVALID_ARG;
+    if (out_lo && out_lo == out) return EVO_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == EVO_DTYPE_F32) {
         if (shape->C > evo::simt::kMaxC) return EVO_ERR_UNSUPPORTED;
@@ -398,12 +430,12 @@ evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
         if (shape->S > 65535) return EVO_ERR_UNSUPPORTED;
         return fwd_f32(*shape, q, k, v, g, *in_str, mask_bias, pair_bias, out, *out_str, lse, s);
     }
-    return fwd_bf16(*shape, q, k, v, g, *in_str, mask_bias, pair_bias, out, *out_str, lse, s);
+    return fwd_bf16(*shape, q, k, v, g, *in_str, mask_bias, pair_bias, out, out_lo, *out_str, lse, s);
 }
 
 evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
                           const void* v, const void* g, const evo_strides_t* in_str, const void* mask_bias,
-                          const void* pair_bias, const void* out, const void* dout,
+                          const void* pair_bias, const void* out, const void* out_lo, const void* dout,
                           const evo_strides_t* out_str, const float* lse, void* dq, void* dk, void* dv,
                           void* dg, const evo_strides_t* grad_str, float* d_pair_bias, void* workspace,
                           size_t workspace_bytes, void* stream) {
@@ -445,12 +477,14 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
     evo::bwd::Call c{};
     c.shape = *shape;
     c.q = q; c.k = k; c.v = v; c.g = g; c.in = *in_str;
-    c.mask = mask_bias; c.bias = pair_bias; c.out = out; c.dout = dout; c.os = *out_str; c.lse = lse;
+    c.mask = mask_bias; c.bias = pair_bias; c.out = out; c.out_lo = out_lo; c.dout = dout; c.os = *out_str;
+    c.lse = lse;
     c.dq = dq; c.dk = dk; c.dv = dv; c.dg = dg; c.gs = *grad_str; c.dbias = d_pair_bias;
     c.ws = static_cast<char*>(workspace);
     c.d_off = ws.d_off; c.nl_off = ws.nl_off; c.doa_off = ws.doa_off; c.dol_off = ws.dol_off;
     c.dqacc_off = ws.dqacc_off;
-    c.biast_off = ws.biast_off; c.part_off = ws.part_off; c.groups = ws.groups;
+    c.biast_off = ws.biast_off; c.part_off = ws.part_off; c.groups = ws.groups; c.db_groups = ws.db_groups;
+    c.wait_ns = g_wait_limit_ns.load();
     int launched = 0;
     evo_status_t rs;
     {
@@ -468,19 +502,58 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype, const voi
 static __device__ __align__(256) unsigned char g_evo_noalloc_ws[EVO_ATTN_NOALLOC_WORKSPACE_BYTES];
 
 static std::mutex g_noalloc_mu;
-static void* g_noalloc_addr[256] = {};
+struct NoallocSlot {
+    unsigned long long ctx_id;   // the context the address belongs to (0: none yet)
+    void* addr;
+};
+static NoallocSlot g_noalloc_slot[256] = {};
 
+// Identifier of the calling thread's current context, unique among the
+// contexts this process creates (cuCtxGetId), or 0 when it cannot be had.  A
+// context created after cudaDeviceReset gets a new identifier, so an address
+// cached for the old context is never reused.
+static unsigned long long current_ctx_id() {
+    static std::once_flag once;
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current device's context.  It
+// is looked up (cudaGetSymbolAddress, with that device current) on the first
+// call in each context and cached; a later call in the same context reuses
+// it, a call in a new context (after cudaDeviceReset) looks it up again.
+// Without a context identifier it is looked up on every call.
 static evo_status_t noalloc_workspace(void** addr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return EVO_ERR_CUDA;
     if (dev < 0 || dev >= 256) return EVO_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {            // once per device, with that device current
+    unsigned long long id = current_ctx_id();
+    NoallocSlot& slot = g_noalloc_slot[dev];
+    if (id == 0 || slot.ctx_id != id || !slot.addr) {
         void* a = nullptr;
         if (cudaGetSymbolAddress(&a, g_evo_noalloc_ws) != cudaSuccess || !a) return EVO_ERR_CUDA;
-        g_noalloc_addr[dev] = a;
+        if (id == 0) id = current_ctx_id();      // the lookup may have made the context current
+        slot.ctx_id = id;
+        slot.addr = a;
     }
-    *addr = g_noalloc_addr[dev];
+    *addr = slot.addr;
     return EVO_OK;
 }
 
@@ -599,7 +672,7 @@ evo_status_t evo_sum_partials(int64_t count, const float* const* parts, int64_t 
 
 evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, const void* q, const void* k,
                                   const void* v, const void* g, const evo_strides_t* in_str, const void* mask_bias,
-                                  const void* pair_bias, const void* out, const void* dout,
+                                  const void* pair_bias, const void* out, const void* out_lo, const void* dout,
                                   const evo_strides_t* out_str, const float* lse, void* dq, void* dk, void* dv,
                                   void* dg, const evo_strides_t* grad_str, float* d_pair_bias, void* stream) {
     const evo_status_t st = check_shape(shape);
@@ -610,8 +683,8 @@ evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype, c
     void* ws = nullptr;
     const evo_status_t wst = noalloc_workspace(&ws);
     if (wst != EVO_OK) return wst;
-    return evo_attn_bwd(shape, dtype, q, k, v, g, in_str, mask_bias, pair_bias, out, dout, out_str, lse, dq, dk,
-                        dv, dg, grad_str, d_pair_bias, ws, EVO_ATTN_NOALLOC_WORKSPACE_BYTES, stream);
+    return evo_attn_bwd(shape, dtype, q, k, v, g, in_str, mask_bias, pair_bias, out, out_lo, dout, out_str, lse,
+                        dq, dk, dv, dg, grad_str, d_pair_bias, ws, EVO_ATTN_NOALLOC_WORKSPACE_BYTES, stream);
 }
 
 }  // extern "C"

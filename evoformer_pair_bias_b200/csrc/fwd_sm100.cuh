@@ -8,11 +8,11 @@
 // MegaFold summary, section "EvoFlash-3D").
 //
 // The mask row is added by the tensor core:
-//   S_u = Q_u K_u^T + (r e_0) m_u^T,        r = bf16(sqrt(C))
+//   S_u = Q_u K_u^T + (r1 e_0 + r2 e_8) m_u^T,   r1 = bf16(sqrt(C)), r2 = bf16(sqrt(C) - r1)
 // accumulates, in fp32 TMEM, sqrt(C) times the logit without the pair bias:
 // the last term is one 16-deep K step whose B block carries the mask row of
-// row s in its first row (exact products in fp32; the mask enters with the
-// relative error of r/sqrt(C), 1.1e-4 for C = 32).  The pair-bias tile
+// row s in its rows 0 and 8 (exact products in fp32; r1 + r2 equals sqrt(C)
+// to 3e-7 relative, so the mask enters exactly up to that and fp32 rounding).  The pair-bias tile
 // (TMA-loaded once per key tile and shared by all NSUB rows s -- it is the
 // same for every s) is added by the softmax threads from shared memory, one
 // fused multiply-add per logit pair, while the other row group has its turn
@@ -22,8 +22,13 @@
 // to the softmax warpgroups with setmaxnreg):
 //   warps 0 .. 4*NSUB-1   one 4-warp softmax group per row s (see below)
 //   warp 4*NSUB           TMA producer: per item Q (double-buffered by item
-//            parity), then per key tile K, V and the mask row (per row s) and
-//            the pair-bias tile into a 2-stage ring that runs across items.
+//            parity), then per key tile K and the mask row (per row s) and
+//            the pair-bias tile into a 2-stage ring ("A") that runs across
+//            items.  A stage of ring A is released as soon as both S MMAs and
+//            both row groups' bias reads are done, so the next tiles' loads
+//            start early instead of waiting for the P V products.
+//   warp 4*NSUB+NSUB+1    TMA producer of V (per row s) into its own 2-stage
+//            ring ("B"), released when the P V products of the tile are done.
 //   warps 4*NSUB+1+u      MMA issuer of row group u (one lane; the first also
 //            owns TMEM): S_u as above (M=128, N=128), then O_u += P_u V_u
 //            (M=128, N=32, K=128, P read from TMEM).  The S MMA of the next
@@ -51,13 +56,14 @@ using namespace evo::sm100;
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per tile
 constexpr int HD = 32;                  // head dim C
-constexpr int STAGES = 2;
+constexpr int STAGES_A = 2;             // K, pair-bias tile, mask blocks
+constexpr int STAGES_B = 2;             // V
 constexpr int Q_BYTES = BM * HD * 2;    // 8 KB, 64-byte rows, 64B swizzle
 constexpr int KV_BYTES = BN * HD * 2;   // 8 KB each for K and V
 constexpr int BIAS_BOX = BM * 64 * 2;   // 16 KB: 128 rows x 64 keys, 128B swizzle
 constexpr int BIAS_BYTES = 2 * BIAS_BOX;
-constexpr int MASKB_BYTES = 4096;       // 16 x 128 bf16 B block (row 0 = mask row), 128B swizzle
-constexpr int ONES_BYTES = 128 * 16 * 2;     // r * e_0 column, K-major, no swizzle
+constexpr int MASKB_BYTES = 4096;       // 16 x 128 bf16 B block (rows 0 and 8 = mask row), 128B swizzle
+constexpr int ONES_BYTES = 128 * 16 * 2;     // r1 e_0 + r2 e_8 columns, K-major, no swizzle
 // per row group: S, P, and two O accumulators (items alternate between them,
 // so an item's epilogue can run after the next item's first tile)
 constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192, SUBCOLS = 256;
@@ -76,16 +82,20 @@ template <int NSUB>
 struct Layout {
     static constexpr int qbuf(int k, int u) { return (k * NSUB + u) * Q_BYTES; }   // per item parity k
     static constexpr int ones = 2 * NSUB * Q_BYTES;
+    // ring A: per stage K (per row), the pair-bias tile, the mask blocks (per row)
     static constexpr int stage0 = round_up(ones + ONES_BYTES, 1024);
     static constexpr int k_off(int u) { return u * KV_BYTES; }
-    static constexpr int v_off(int u) { return (NSUB + u) * KV_BYTES; }
-    static constexpr int bias_off = 2 * NSUB * KV_BYTES;
+    static constexpr int bias_off = NSUB * KV_BYTES;
     static constexpr int maskb_off(int u) { return bias_off + BIAS_BYTES + u * MASKB_BYTES; }
     static constexpr int stage_bytes = round_up(bias_off + BIAS_BYTES + NSUB * MASKB_BYTES, 1024);
-    static constexpr int bars = stage0 + STAGES * stage_bytes;
-    // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[u], s_free[u], p_full[u], o_full[u],
-    // mma_done[u], exp_turn[u]
-    static constexpr int nbars = 4 + 2 * STAGES + 6 * NSUB;
+    // ring B: per stage V (per row)
+    static constexpr int vstage0 = stage0 + STAGES_A * stage_bytes;
+    static constexpr int v_off(int u) { return u * KV_BYTES; }
+    static constexpr int vstage_bytes = round_up(NSUB * KV_BYTES, 1024);
+    static constexpr int bars = vstage0 + STAGES_B * vstage_bytes;
+    // q_full[2], q_empty[2], ka_full[SA], ka_empty[SA], v_full[SB], v_empty[SB], s_full[u], s_free[u],
+    // p_full[u], o_full[u], mma_done[u], exp_turn[u]
+    static constexpr int nbars = 4 + 2 * STAGES_A + 2 * STAGES_B + 6 * NSUB;
     static constexpr int misc = bars + nbars * 8;   // tmem base (u32), abort flag (u32)
     static constexpr int bytes = misc + 16 + 1024;  // + slack to align the base to 1024
     static constexpr uint32_t tmem_cols = NSUB == 1 ? 256 : 512;
@@ -105,12 +115,15 @@ struct Params {
     int n_sg;                 // row groups of NSUB rows
     int n_items;              // B * H * n_sg * n_it
     float scale;              // 1/sqrt(C)
-    float r_bf16;             // bf16(sqrt(C)), the nonzero of the mask MMA column
+    float r_bf16;             // r1 = bf16(sqrt(C)) and r2 = bf16(sqrt(C) - r1): the mask MMA's
+    float r2_bf16;            //   two nonzero columns, whose sum is sqrt(C) to 3e-7
     const __nv_bfloat16* g;   // gate, strides `in`
     Strides in;
     __nv_bfloat16* out;       // strides `os`
+    __nv_bfloat16* out_lo;    // strides `os`: bf16(out_fp32 - out), or null
     Strides os;
     float* lse;               // [B,S,H,N]
+    uint64_t wait_ns;         // limit of every wait but the final drains (EVO_WAIT_LIMIT_NS by default)
 };
 
 struct Item {
@@ -146,19 +159,24 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kProducer = 4 * NSUB, kMma = 4 * NSUB + 1;   // MMA issuers: warps kMma .. kMma+NSUB-1
+    constexpr int kProducerV = kMma + NSUB;
+    static_assert(kProducerV < L::threads / 32, "warp roles");
 
     const uint32_t bar0 = base + L::bars;
+    constexpr int kS = 4 + 2 * STAGES_A + 2 * STAGES_B;        // first per-row-group barrier
     auto q_full = [&](int x) { return bar0 + 8u * (0 + x); };
     auto q_empty = [&](int x) { return bar0 + 8u * (2 + x); };
-    auto kv_full = [&](int st) { return bar0 + 8u * (4 + st); };
-    auto kv_empty = [&](int st) { return bar0 + 8u * (4 + STAGES + st); };
-    auto s_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + u); };
-    auto s_free = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + NSUB + u); };
-    auto p_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 2 * NSUB + u); };
-    auto o_full = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 3 * NSUB + u); };
-    auto mma_done = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 4 * NSUB + u); };
+    auto ka_full = [&](int st) { return bar0 + 8u * (4 + st); };
+    auto ka_empty = [&](int st) { return bar0 + 8u * (4 + STAGES_A + st); };
+    auto v_full = [&](int st) { return bar0 + 8u * (4 + 2 * STAGES_A + st); };
+    auto v_empty = [&](int st) { return bar0 + 8u * (4 + 2 * STAGES_A + STAGES_B + st); };
+    auto s_full = [&](int u) { return bar0 + 8u * (kS + u); };
+    auto s_free = [&](int u) { return bar0 + 8u * (kS + NSUB + u); };
+    auto p_full = [&](int u) { return bar0 + 8u * (kS + 2 * NSUB + u); };
+    auto o_full = [&](int u) { return bar0 + 8u * (kS + 3 * NSUB + u); };
+    auto mma_done = [&](int u) { return bar0 + 8u * (kS + 4 * NSUB + u); };
     // exp_turn[u]: row group u may start the exponentials of its next tile
-    auto exp_turn = [&](int u) { return bar0 + 8u * (4 + 2 * STAGES + 5 * NSUB + u); };
+    auto exp_turn = [&](int u) { return bar0 + 8u * (kS + 5 * NSUB + u); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::misc + 4);
 
@@ -167,9 +185,13 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             mbar_init(q_full(x), 1);
             mbar_init(q_empty(x), NSUB);           // one commit per MMA issuer
         }
-        for (int st = 0; st < STAGES; ++st) {
-            mbar_init(kv_full(st), 1);
-            mbar_init(kv_empty(st), NSUB);
+        for (int st = 0; st < STAGES_A; ++st) {
+            mbar_init(ka_full(st), 1);
+            mbar_init(ka_empty(st), NSUB + 4 * NSUB);   // the S MMAs' commits + every softmax warp's bias reads
+        }
+        for (int st = 0; st < STAGES_B; ++st) {
+            mbar_init(v_full(st), 1);
+            mbar_init(v_empty(st), NSUB);               // the P V MMAs' commits
         }
         for (int u = 0; u < NSUB; ++u) {
             mbar_init(s_full(u), 1);
@@ -196,14 +218,15 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     if (warp < 4 * NSUB) {
         // Constant MMA operand (element (row, k) of a no-swizzle K-major tile is
         // at (row % 8) * 16 + (row / 8) * SBO + (k / 8) * 128 + (k % 8) * 2):
-        //   column r*e_0 (SBO 256), and rows 1..15 of every mask block zero
-        //   (the TMA writes row 0 each stage).
+        //   columns r1 e_0 + r2 e_8 (SBO 256), and every mask block zero but
+        //   its rows 0 and 8 (the TMA writes those each stage).
         const int t = threadIdx.x;
         const int nt = 128 * NSUB;
         const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
+        const uint16_t rb2 = (uint16_t)(__float_as_uint(p.r2_bf16) >> 16);
         for (int o = t * 16; o < ONES_BYTES; o += nt * 16)
             *reinterpret_cast<uint4*>(gbase + L::ones + o) = make_uint4(0u, 0u, 0u, 0u);
-        for (int st = 0; st < STAGES; ++st)
+        for (int st = 0; st < STAGES_A; ++st)
             for (int u = 0; u < NSUB; ++u)
                 for (int o = t * 16; o < MASKB_BYTES; o += nt * 16)
                     *reinterpret_cast<uint4*>(gbase + L::stage0 + st * L::stage_bytes + L::maskb_off(u) + o) =
@@ -213,6 +236,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         if (t < 128) {
             const int rr = t;
             *reinterpret_cast<uint16_t*>(gbase + L::ones + (rr % 8) * 16 + (rr / 8) * 256) = rb;
+            *reinterpret_cast<uint16_t*>(gbase + L::ones + (rr % 8) * 16 + (rr / 8) * 256 + 128) = rb2;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -225,8 +249,8 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         regs_decrease<L::control_regs>();
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            constexpr uint32_t tx = 2 * NSUB * KV_BYTES + (HAS_BIAS ? BIAS_BYTES : 0) + (HAS_MASK ? NSUB * 256 : 0);
-            int q_issued[2] = {0, 0}, kv_issued[STAGES] = {};
+            constexpr uint32_t tx = NSUB * KV_BYTES + (HAS_BIAS ? BIAS_BYTES : 0) + (HAS_MASK ? NSUB * 512 : 0);
+            int q_issued[2] = {0, 0}, kv_issued[STAGES_A] = {};
             int tg = 0;
             bool ok = true;
             for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
@@ -236,7 +260,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
 #pragma unroll
                 for (int u = 0; u < NSUB; ++u) s_ld[u] = min(s0 + u, p.S - 1);
                 const int qb = k & 1;
-                if (k >= 2) ok = mbar_wait(q_empty(qb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x001);
+                if (k >= 2) ok = mbar_wait(q_empty(qb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x001, p.wait_ns);
                 if (!ok) break;
                 mbar_arrive_expect_tx(q_full(qb), NSUB * Q_BYTES);
 #pragma unroll
@@ -244,26 +268,28 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     tma_load_5d(base + L::qbuf(qb, u), &tm_q, q_full(qb), 0, itm.i0, itm.h, s_ld[u], itm.b);
                 ++q_issued[qb];
                 for (int j = 0; j < p.n_kv; ++j, ++tg) {
-                    const int st = tg % STAGES;
+                    const int st = tg % STAGES_A;
                     const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
-                    if (tg >= STAGES)
-                        ok = mbar_wait(kv_empty(st), ((tg / STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x002);
+                    if (tg >= STAGES_A)
+                        ok = mbar_wait(ka_empty(st), ((tg / STAGES_A) - 1) & 1, abort_flag, kTimeoutBase | 0x002, p.wait_ns);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(kv_full(st), tx);
+                    mbar_arrive_expect_tx(ka_full(st), tx);
 #pragma unroll
-                    for (int u = 0; u < NSUB; ++u) {
-                        tma_load_5d(sb + L::k_off(u), &tm_k, kv_full(st), 0, j * BN, itm.h, s_ld[u], itm.b);
-                        tma_load_5d(sb + L::v_off(u), &tm_v, kv_full(st), 0, j * BN, itm.h, s_ld[u], itm.b);
-                    }
+                    for (int u = 0; u < NSUB; ++u)
+                        tma_load_5d(sb + L::k_off(u), &tm_k, ka_full(st), 0, j * BN, itm.h, s_ld[u], itm.b);
                     if (HAS_BIAS) {
-                        tma_load_4d(sb + L::bias_off, &tm_bias, kv_full(st), j * BN, itm.i0, itm.h, itm.b);
-                        tma_load_4d(sb + L::bias_off + BIAS_BOX, &tm_bias, kv_full(st), j * BN + 64, itm.i0, itm.h, itm.b);
+                        tma_load_4d(sb + L::bias_off, &tm_bias, ka_full(st), j * BN, itm.i0, itm.h, itm.b);
+                        tma_load_4d(sb + L::bias_off + BIAS_BOX, &tm_bias, ka_full(st), j * BN + 64, itm.i0, itm.h, itm.b);
                     }
                     if (HAS_MASK) {
 #pragma unroll
                         for (int u = 0; u < NSUB; ++u) {
-                            tma_load_3d(sb + L::maskb_off(u), &tm_mask, kv_full(st), j * BN, s_ld[u], itm.b);
-                            tma_load_3d(sb + L::maskb_off(u) + 2048, &tm_mask, kv_full(st), j * BN + 64, s_ld[u], itm.b);
+                            // rows 0 and 8 of the two 64-key halves (rows 0 and 8 both start a
+                            // 128B-swizzle atom, so the unswizzled row lands as the MMA reads it)
+                            tma_load_3d(sb + L::maskb_off(u), &tm_mask, ka_full(st), j * BN, s_ld[u], itm.b);
+                            tma_load_3d(sb + L::maskb_off(u) + 1024, &tm_mask, ka_full(st), j * BN, s_ld[u], itm.b);
+                            tma_load_3d(sb + L::maskb_off(u) + 2048, &tm_mask, ka_full(st), j * BN + 64, s_ld[u], itm.b);
+                            tma_load_3d(sb + L::maskb_off(u) + 3072, &tm_mask, ka_full(st), j * BN + 64, s_ld[u], itm.b);
                         }
                     }
                     ++kv_issued[st];
@@ -273,8 +299,35 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             volatile int no_abort = 0;
             for (int x = 0; x < 2; ++x)
                 if (q_issued[x]) mbar_wait(q_full(x), (q_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x003);
-            for (int st = 0; st < STAGES; ++st)
-                if (kv_issued[st]) mbar_wait(kv_full(st), (kv_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x004);
+            for (int st = 0; st < STAGES_A; ++st)
+                if (kv_issued[st]) mbar_wait(ka_full(st), (kv_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x004);
+        }
+    } else if (warp == kProducerV) {
+        regs_decrease<L::control_regs>();
+        // ------------------------------------------------------------ producer of V
+        if (lane == 0) {
+            int v_issued[STAGES_B] = {};
+            int tg = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+                const Item itm = decode(p, item);
+                const int s0 = itm.sg * NSUB;
+                for (int j = 0; j < p.n_kv; ++j, ++tg) {
+                    const int st = tg % STAGES_B;
+                    const uint32_t vb = base + L::vstage0 + st * L::vstage_bytes;
+                    if (tg >= STAGES_B)
+                        ok = mbar_wait(v_empty(st), ((tg / STAGES_B) - 1) & 1, abort_flag, kTimeoutBase | 0x006, p.wait_ns);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(v_full(st), NSUB * KV_BYTES);
+#pragma unroll
+                    for (int u = 0; u < NSUB; ++u)
+                        tma_load_5d(vb + L::v_off(u), &tm_v, v_full(st), 0, j * BN, itm.h, min(s0 + u, p.S - 1), itm.b);
+                    ++v_issued[st];
+                }
+            }
+            volatile int no_abort = 0;
+            for (int st = 0; st < STAGES_B; ++st)
+                if (v_issued[st]) mbar_wait(v_full(st), (v_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x007);
         }
     } else if (warp >= kMma && warp < kMma + NSUB) {
         regs_decrease<L::control_regs>();
@@ -288,29 +341,32 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                            t_o = tmem + u * SUBCOLS + COL_O;
             bool ok = true;
             int tg = 0;
-            int prev_st = 0, prev_j = 0, prev_k = 0;   // the tile whose PV is still to be issued
+            int prev_j = 0, prev_k = 0;   // the tile (tg - 1) whose PV is still to be issued
             bool pending = false;
             auto issue_pv = [&]() -> bool {   // PV of tile tg-1
-                const uint32_t sb = base + L::stage0 + prev_st * L::stage_bytes;
-                if (!mbar_wait(p_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x104)) return false;
+                const int vs = (tg - 1) % STAGES_B;
+                const uint32_t vb = base + L::vstage0 + vs * L::vstage_bytes;
+                if (!mbar_wait(p_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x104, p.wait_ns)) return false;
+                if (!mbar_wait(v_full(vs), ((tg - 1) / STAGES_B) & 1, abort_flag, kTimeoutBase | 0x106, p.wait_ns))
+                    return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = smem_desc(sb + L::v_off(u) + kk * 1024, KV_BYTES, 512, kSw64);
+                    const uint64_t bd = smem_desc(vb + L::v_off(u) + kk * 1024, KV_BYTES, 512, kSw64);
                     mma_ts(t_o + (uint32_t)(prev_k & 1) * HD, t_p + kk * 8, bd, IDESC_PV, (prev_j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(o_full(u));
-                mma_commit(kv_empty(prev_st));
+                mma_commit(v_empty(vs));
                 return true;
             };
             for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
                 const int qb = k & 1;
-                ok = mbar_wait(q_full(qb), (k >> 1) & 1, abort_flag, kTimeoutBase | 0x101);
+                ok = mbar_wait(q_full(qb), (k >> 1) & 1, abort_flag, kTimeoutBase | 0x101, p.wait_ns);
                 for (int j = 0; ok && j < p.n_kv; ++j) {
-                    const int st = tg % STAGES;
+                    const int st = tg % STAGES_A;
                     const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
-                    ok = mbar_wait(kv_full(st), (tg / STAGES) & 1, abort_flag, kTimeoutBase | 0x102);
-                    if (ok && tg > 0) ok = mbar_wait(s_free(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x103);
+                    ok = mbar_wait(ka_full(st), (tg / STAGES_A) & 1, abort_flag, kTimeoutBase | 0x102, p.wait_ns);
+                    if (ok && tg > 0) ok = mbar_wait(s_free(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x103, p.wait_ns);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -319,14 +375,14 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                         const uint64_t bd = smem_desc(sb + L::k_off(u) + kk * 32, 16, 512, kSw64);
                         mma_ss(t_s, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
                     }
-                    if (HAS_MASK) {                               // + r * mask[s, j]
+                    if (HAS_MASK) {                               // + (r1 + r2) * mask[s, j]
                         const uint64_t ad = smem_desc(base + L::ones, 128, 256, kSwNone);
                         const uint64_t bd = smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128);
                         mma_ss(t_s, ad, bd, IDESC_MASK, 1u);
                     }
                     mma_commit(s_full(u));
+                    mma_commit(ka_empty(st));                     // K and the mask blocks read
                     if (pending) ok = issue_pv();
-                    prev_st = st;
                     prev_j = j;
                     prev_k = k;
                     pending = true;
@@ -374,11 +430,12 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             uint32_t o[HD];
             tmem_ld32_sync(lane_addr + COL_O + (uint32_t)epi.obuf * HD, o);
             if (epi.row_ok) {
-                __nv_bfloat16* op = p.out + p.os.off(epi.b, epi.s, epi.i, epi.h);
+                const int64_t oo = p.os.off(epi.b, epi.s, epi.i, epi.h);
+                __nv_bfloat16* op = p.out + oo;
 #pragma unroll
                 for (int q = 0; q < HD / 8; ++q) {
                     const uint32_t gv[4] = {gw[q].x, gw[q].y, gw[q].z, gw[q].w};
-                    uint32_t ov[4];
+                    uint32_t ov[4], lv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         // out = O / (l * (1 + exp(-g))): the backward's D = sum(dout * out)
@@ -392,8 +449,11 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                         const float o0 = __fdividef(__uint_as_float(o[q * 8 + 2 * e]), epi.l * (1.0f + e0));
                         const float o1 = __fdividef(__uint_as_float(o[q * 8 + 2 * e + 1]), epi.l * (1.0f + e1));
                         ov[e] = pack_bf16(o0, o1);
+                        lv[e] = pack_bf16(o0 - bf16lo(ov[e]), o1 - bf16hi(ov[e]));   // rounding residual
                     }
                     *reinterpret_cast<uint4*>(op + q * 8) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+                    if (p.out_lo)
+                        *reinterpret_cast<uint4*>(p.out_lo + oo + q * 8) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
                 }
                 p.lse[((int64_t)(epi.b * p.S + epi.s) * p.H + epi.h) * p.N + epi.i] =
                     (epi.ms + __log2f(epi.l)) * EVO_LN2;
@@ -414,7 +474,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     // the gate row is only needed by the item's epilogue: start bringing it into L2
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(p.g + p.in.off(itm.b, s, i, itm.h)));
                 }
-                ok = mbar_wait(s_full(u), tg & 1, abort_flag, kTimeoutBase | 0x201);
+                ok = mbar_wait(s_full(u), tg & 1, abort_flag, kTimeoutBase | 0x201, p.wait_ns);
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t xr[BN];
@@ -426,13 +486,13 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 // y = S * sc2 + bias * log2(e): the pair-bias row of this query from
                 // the stage's tile (two 64-key boxes, 128B swizzle: 16-byte chunk c
                 // of row r sits at chunk c ^ (r & 7)), two logits per instruction
+                const int st = tg % STAGES_A;
                 if (HAS_BIAS) {
                     // acquire the TMA writes of this stage (already complete: S used them)
-                    ok = mbar_wait(kv_full(tg % STAGES), (tg / STAGES) & 1, abort_flag, kTimeoutBase | 0x206);
+                    ok = mbar_wait(ka_full(st), (tg / STAGES_A) & 1, abort_flag, kTimeoutBase | 0x206, p.wait_ns);
                     if (!ok) break;
                 }
                 {
-                    const int st = tg % STAGES;
                     const uint8_t* brow = gbase + L::stage0 + st * L::stage_bytes + L::bias_off + r * 128;
 #pragma unroll
                     for (int q = 0; q < BN / 8; ++q) {
@@ -451,6 +511,10 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                         }
                     }
                 }
+                // this warp no longer reads the stage's bias tile: with both S MMAs done,
+                // the stage can take the tile after next
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ka_empty(st));
                 const int valid = p.N - j * BN;      // keys beyond N are padding: exclude them
                 if (valid < BN) {
 #pragma unroll
@@ -474,7 +538,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 const float alpha = move ? ex2(ms - ms_new) : 1.0f;   // 0 on an item's first tile
                 if (tg > 0) {
                     // PV of the previous tile must be done before P is overwritten and O rescaled.
-                    ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x203);
+                    ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x203, p.wait_ns);
                     if (!ok) break;
                     tc_fence_after();
                 }
@@ -490,8 +554,8 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 // group 1's tile t, so one group's exponentials overlap the other's
                 // loads, maxima and waits instead of competing with its exponentials.
                 if (NSUB == 2) {
-                    if (u == 1) ok = mbar_wait(exp_turn(1), tg & 1, abort_flag, kTimeoutBase | 0x205);
-                    else if (tg > 0) ok = mbar_wait(exp_turn(0), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x205);
+                    if (u == 1) ok = mbar_wait(exp_turn(1), tg & 1, abort_flag, kTimeoutBase | 0x205, p.wait_ns);
+                    else if (tg > 0) ok = mbar_wait(exp_turn(0), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x205, p.wait_ns);
                     if (!ok) break;
                 }
                 const uint64_t NEG_MS2 = f2(-ms_new, -ms_new);
@@ -537,7 +601,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             epi.l = l; epi.ms = ms;
         }
         if (ok && epi.pending) {   // the last item: wait for its last PV
-            ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x204);
+            ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x204, p.wait_ns);
             if (ok) {
                 tc_fence_after();
                 run_epilogue();

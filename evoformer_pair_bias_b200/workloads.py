@@ -87,8 +87,9 @@ WORKLOADS = {
                               "tail:64", 20266, "long AF3-style triangle attention"),
 }
 
-#: Bench default: MSA-row attention at AF2 initial-training size.
-DEFAULT_BENCH = "msa_row_256"
+#: Bench default: the long AF3-style triangle attention (N_res = 1536), the largest
+#: configuration that runs on one GPU and the regime (N_res >= 384) the targets are stated for.
+DEFAULT_BENCH = "tri_long_1536"
 
 
 def mask_columns(w: Workload, gen: torch.Generator) -> torch.Tensor | None:
@@ -162,6 +163,26 @@ def make_inputs(w: Workload, device="cpu", with_dout: bool = True) -> dict:
     return res
 
 
+def finite_mask(w: Workload, kind: str, seed: int, device="cpu") -> torch.Tensor:
+    """A seeded additive mask ``[B, S, 1, 1, N]`` with finite values that differ per row s.
+
+    ``"gauss3"``: every entry ~ 3 N(0, 1); ``"gauss1"``: ~ N(0, 1).  ``"mixed"``: every entry ~ 2 N(0, 1),
+    then a random 20% of the entries of each row s set to ``-1e9`` (at least one
+    key of every row stays finite).  Rounded to ``w.dtype``.
+    """
+    gen = torch.Generator("cpu").manual_seed(seed)
+    if kind in ("gauss3", "gauss1"):
+        m = (3.0 if kind == "gauss3" else 1.0) * torch.randn((w.B, w.S, 1, 1, w.N), generator=gen)
+    elif kind == "mixed":
+        m = 2.0 * torch.randn((w.B, w.S, 1, 1, w.N), generator=gen)
+        drop = torch.rand((w.B, w.S, 1, 1, w.N), generator=gen) < 0.2
+        drop[..., 0] = False
+        m[drop] = MASK_VALUE
+    else:
+        raise ValueError(f"unknown mask kind {kind!r}")
+    return m.to(w.torch_dtype).to(device)
+
+
 def sample_rows(n: int, count: int, seed: int) -> list[int]:
     """A seeded sorted sample of ``count`` distinct indices in [0, n), always with 0 and n-1."""
     gen = torch.Generator("cpu").manual_seed(seed)
@@ -185,7 +206,7 @@ def ceil_div(a: int, b: int) -> int:
     return -(-a // b)
 
 
-__all__ = ["Workload", "WORKLOADS", "DEFAULT_BENCH", "MASK_VALUE", "make_inputs",
+__all__ = ["Workload", "WORKLOADS", "DEFAULT_BENCH", "MASK_VALUE", "make_inputs", "finite_mask",
            "logical_view", "storage_empty", "sample_rows", "logits_bytes", "pair_rep_bytes",
            "mask_columns", "ceil_div", "ProjWorkload", "PROJ_WORKLOADS", "make_proj_inputs",
            "make_pair_bias_params", "TriMulWorkload", "TRI_MUL_WORKLOADS", "make_tri_mul_inputs",

@@ -102,6 +102,14 @@ size_t evo_attn_bwd_workspace_bytes(const evo_shape_t* shape, evo_dtype_t dtype)
  *   pair_bias    device pointer, contiguous [B,1,H,N,N] indexed [b,h,i,j]
  *                (query i, key j), or NULL for none.
  *   out          device pointer, logical [B,S,N,H,C] with strides `out_str`.
+ *   out_lo       bf16 only, optional (NULL = not written): device pointer with
+ *                `out`'s layout and strides that receives the rounding residual
+ *                of out, bf16(out_fp32 - out), so that out + out_lo carries
+ *                about 16 significant bits of the fp32 result.  Passed back to
+ *                evo_attn_bwd, it makes the row sums D_i = sum_c dout*out exact
+ *                to that precision; d_pair_bias adds the error of D_i over all
+ *                rows s, so this is what keeps its error small at large N_seq.
+ *                Ignored (may be NULL) on the fp32 path.
  *   lse          device pointer, contiguous fp32 [B,S,H,N]: the natural-log
  *                sum-exp of each logit row, saved for the backward pass.
  *   stream       cudaStream_t to enqueue on (NULL = legacy default stream).
@@ -110,7 +118,7 @@ evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype,
                           const void* q, const void* k, const void* v, const void* g,
                           const evo_strides_t* in_str,
                           const void* mask_bias, const void* pair_bias,
-                          void* out, const evo_strides_t* out_str,
+                          void* out, void* out_lo, const evo_strides_t* out_str,
                           float* lse, void* stream);
 
 /*
@@ -123,6 +131,8 @@ evo_status_t evo_attn_fwd(const evo_shape_t* shape, evo_dtype_t dtype,
  *                     sums over fixed row groups are added in a fixed order,
  *                     with no floating-point atomics.
  *   out, dout         the forward output and its gradient (strides `out_str`).
+ *   out_lo            the forward's out_lo (bf16 only), or NULL: without it D_i
+ *                     is taken from the bf16 out alone.
  *   lse               the forward's saved lse.
  *   workspace         device buffer of at least evo_attn_bwd_workspace_bytes()
  *                     bytes, 256-byte aligned; contents need not be initialised.
@@ -134,8 +144,8 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype,
                           const void* q, const void* k, const void* v, const void* g,
                           const evo_strides_t* in_str,
                           const void* mask_bias, const void* pair_bias,
-                          const void* out, const void* dout, const evo_strides_t* out_str,
-                          const float* lse,
+                          const void* out, const void* out_lo, const void* dout,
+                          const evo_strides_t* out_str, const float* lse,
                           void* dq, void* dk, void* dv, void* dg, const evo_strides_t* grad_str,
                           float* d_pair_bias,
                           void* workspace, size_t workspace_bytes, void* stream);
@@ -159,8 +169,10 @@ evo_status_t evo_attn_bwd(const evo_shape_t* shape, evo_dtype_t dtype,
  * 128-row, 8-head MSA-row shape at N=256 does not.
  *
  * The first call on a device looks up the scratch area's device address (a
- * one-time, host-side query; it allocates nothing); make that first call
- * before any stream capture on that device.  All calls share the one scratch
+ * host-side query that allocates nothing) and caches it for the device's
+ * current context; make that first call before any stream capture on that
+ * device.  After cudaDeviceReset the next call runs in a new context and
+ * looks the address up again (again before any stream capture).  All calls share the one scratch
  * area and it keeps the last call's contents; every part of it that must
  * start at zero is cleared by the call itself.  Calls whose kernels overlap
  * on the GPU (different streams, or different host threads, with no ordering
@@ -172,8 +184,8 @@ evo_status_t evo_attn_bwd_noalloc(const evo_shape_t* shape, evo_dtype_t dtype,
                                   const void* q, const void* k, const void* v, const void* g,
                                   const evo_strides_t* in_str,
                                   const void* mask_bias, const void* pair_bias,
-                                  const void* out, const void* dout, const evo_strides_t* out_str,
-                                  const float* lse,
+                                  const void* out, const void* out_lo, const void* dout,
+                                  const evo_strides_t* out_str, const float* lse,
                                   void* dq, void* dk, void* dv, void* dg, const evo_strides_t* grad_str,
                                   float* d_pair_bias, void* stream);
 
@@ -299,6 +311,30 @@ const char* evo_status_string(evo_status_t status);
  */
 evo_status_t evo_attn_device_status(int clear);
 
+/*
+ * Limit, in nanoseconds, of the bounded in-kernel waits of the forward kernel
+ * and of the backward's d_pair_bias kernel launched after this call (default
+ * 2e9, i.e. 2 s); returns the previous limit.  It exists so that the timeout path can be exercised without
+ * breaking anything: with a limit of 0 every wait that is not satisfied at
+ * once gives up, the kernel drains its own copies and tensor-core work (those
+ * drains always keep the 2 s default) and returns, and
+ * evo_attn_device_status() reports EVO_ERR_DEVICE_TIMEOUT.  The outputs of
+ * such a call are undefined; the context stays usable.  Affects every device;
+ * not for use while other threads launch attention kernels.
+ */
+uint64_t evo_attn_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * y[i] = 2^x[i] for n fp32 values (device pointers, 4-byte aligned), computed
+ * by the FMA-pipe exponential the attention kernels use in place of the MUFU
+ * unit for part of their exponentials: a cubic in the fraction after a
+ * round-to-nearest split of x, relative error below 8e-5 for -125 <= x <= 126;
+ * arguments below -125 give 2^-125.  Exported so that the device function
+ * itself can be checked against 2^x on the GPU.  Returns EVO_ERR_INVALID_ARG
+ * for n < 0 or a null pointer with n > 0.
+ */
+evo_status_t evo_exp2_fma(const float* x, float* y, int64_t n, void* stream);
+
 /* ABI version, major * 10000 + minor * 100 + patch. */
 int evo_attn_version(void);
 
@@ -325,15 +361,16 @@ uint64_t evo_attn_launch_count(void);
  * read (that phase is then left out of the sums).  Both functions are safe to
  * call from several host threads.
  */
-#define EVO_TIMING_PHASES 7
+#define EVO_TIMING_PHASES 8
 enum {
     EVO_PHASE_FWD_MAIN = 0,   /* the forward kernel                         */
-    EVO_PHASE_BWD_MAIN = 1,   /* the backward's main (tensor-core) kernel    */
+    EVO_PHASE_BWD_MAIN = 1,   /* the backward's dq, dk, dv kernel            */
     EVO_PHASE_BWD_ALL = 2,    /* every kernel and memset of one evo_attn_bwd */
     EVO_PHASE_PROJ = 3,       /* the evo_ln_linear kernel                    */
     EVO_PHASE_PAIR_BIAS = 4,  /* the evo_ln_pair_bias kernel                 */
     EVO_PHASE_TRI_MUL = 5,    /* the evo_tri_mul kernel                      */
-    EVO_PHASE_OPM = 6         /* the evo_outer_product_mean kernel           */
+    EVO_PHASE_OPM = 6,        /* the evo_outer_product_mean kernel           */
+    EVO_PHASE_BWD_DBIAS = 7   /* the backward's d_pair_bias kernel           */
 };
 typedef struct {
     uint64_t calls[EVO_TIMING_PHASES];

@@ -22,6 +22,10 @@ from evoformer_pair_bias_b200 import attention as A
 from evoformer_pair_bias_b200.workloads import make_inputs
 
 TOL = {"bf16": dict(max_abs=2e-2, rel_l2=5e-3), "f32": dict(max_abs=None, rel_l2=1e-4)}
+#: Outputs the bf16 path stores in bf16 (lse and d_pair_bias are fp32).
+BF16_STORED = ("out", "dq", "dk", "dv", "dg")
+#: Largest relative change of rounding a real number to bf16 (8 significant bits, round to nearest).
+BF16_ROUNDING = 2.0 ** -8
 ROW_TENSORS = ("q", "k", "v", "g", "dout")
 
 
@@ -33,15 +37,23 @@ def f64(t):
     return None if t is None else t.detach().to("cpu", torch.float64).numpy()
 
 
-def gpu_fwd_bwd(d, want_bwd=True):
-    out, lse = A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"])
+def gpu_fwd_bwd(d, want_bwd=True, with_out_lo=None):
+    """Forward + backward through the C-ABI binding.  bf16 calls pass the forward's
+    rounding residual of out to the backward (with_out_lo defaults to True for bf16)."""
+    if with_out_lo is None:
+        with_out_lo = d["q"].dtype == torch.bfloat16
+    if with_out_lo:
+        out, lse, out_lo = A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"],
+                                          out_lo=True)
+    else:
+        (out, lse), out_lo = A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"]), None
     res = {"out": out, "lse": lse}
     if want_bwd:
         dout = d["dout"]
         if dout.stride() != out.stride():
             dout = A.empty_like_rows(out).copy_(dout)
         res.update(A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"],
-                                  out, lse, dout))
+                                  out, lse, dout, out_lo=out_lo))
     torch.cuda.synchronize()
     return res
 
@@ -112,21 +124,35 @@ def report(case, name, m):
             f.write(json.dumps(dict(case=case, tensor=name, **m)) + "\n")
 
 
-def assert_close(case, name, got, ref, dtype):
+def assert_close(case, name, got, ref, dtype, beyond_output_rounding=False):
+    """Check one output tensor against the oracle at the benchmark spec tolerances.
+
+    With ``beyond_output_rounding`` (cases whose bf16-stored outputs reach
+    magnitudes of 4 and more), the max-abs bound applies to the error beyond
+    the output's own rounding to bf16: |gpu - oracle| <= 2e-2 + 2^-8 |oracle|
+    element by element.  Rounding the exact value x to bf16 alone moves it by up
+    to 2^-8 |x| (0.031 at |x| = 8), which a fixed 2e-2 cannot hold for large
+    outputs whatever the kernel does; rel-L2 stays at 5e-3.
+    """
     m = metrics(got, ref)
-    report(case, name, m)
     tol = TOL[dtype]
+    allow = beyond_output_rounding and dtype == "bf16" and name in BF16_STORED
+    if allow:
+        g, r = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+        m["max_abs_beyond_rounding"] = float(np.max(np.abs(g - r) - BF16_ROUNDING * np.abs(r))) if r.size else 0.0
+    report(case, name, m)
     assert m["finite"], (case, name, "non-finite values")
     assert m["rel_l2"] <= tol["rel_l2"], (case, name, m)
     if tol["max_abs"] is not None:
-        assert m["max_abs"] <= tol["max_abs"], (case, name, m)
+        assert (m["max_abs_beyond_rounding"] if allow else m["max_abs"]) <= tol["max_abs"], (case, name, m)
     return m
 
 
-def compare_all(case, gpu, ref, dtype, names=("out", "lse", "dq", "dk", "dv", "dg", "d_pair_bias")):
+def compare_all(case, gpu, ref, dtype, names=("out", "lse", "dq", "dk", "dv", "dg", "d_pair_bias"),
+                beyond_output_rounding=False):
     for n in names:
         if n in ref:
-            assert_close(case, n, f64(gpu[n]), ref[n], dtype)
+            assert_close(case, n, f64(gpu[n]), ref[n], dtype, beyond_output_rounding)
 
 
 def workload_inputs(w, drop_bias=False, drop_mask=False):

@@ -17,7 +17,7 @@ import oracle
 from _parity import (TOL, assert_close, compare_all, f64, gpu_fwd_bwd, oracle_fwd_bwd, to_gpu,
                      workload_inputs)
 from evoformer_pair_bias_b200 import attention as A
-from evoformer_pair_bias_b200.workloads import WORKLOADS, Workload, make_inputs, sample_rows
+from evoformer_pair_bias_b200.workloads import WORKLOADS, Workload, finite_mask, make_inputs, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -65,6 +65,35 @@ def test_optional_biases(drop):
     gpu = gpu_fwd_bwd(to_gpu(inp))
     ref = oracle_fwd_bwd(inp)
     compare_all(w.name, gpu, ref, "bf16")
+
+
+MASKED = [
+    # name, B, S, N, H, C, dtype, layout, mask kind
+    ("gauss3_bf16", 2, 3, 200, 2, 32, "bf16", "msa_row", "gauss3"),
+    ("mixed_bf16", 1, 4, 264, 2, 32, "bf16", "msa_row", "mixed"),
+    ("mixed_tri_end_bf16", 1, 136, 136, 1, 32, "bf16", "tri_end", "mixed"),
+    ("gauss1_bf16", 1, 3, 392, 2, 32, "bf16", "msa_row", "gauss1"),
+    ("gauss3_f32", 1, 3, 45, 3, 16, "f32", "msa_row", "gauss3"),
+    ("mixed_f32", 2, 2, 40, 2, 8, "f32", "msa_row", "mixed"),
+]
+
+
+@pytest.mark.parametrize("spec", MASKED, ids=[s[0] for s in MASKED])
+def test_finite_masks_that_differ_per_row(spec):
+    """mask_bias is a float input: finite values (3 N(0,1); N(0,1); or 2 N(0,1) with 20% of each
+    row at -1e9), different in every row s, enter the logits of both passes like the pair bias.
+
+    Masks of scale 2 and 3 sharpen the softmax until dv and dk reach 5 to 11 in magnitude,
+    where rounding the exact value to the bf16 output alone can move it by up to 0.031: those
+    cases hold max-abs 2e-2 on the error beyond that rounding (rel-L2 5e-3 unchanged).  The
+    N(0,1) mask keeps the outputs small and is held to the plain bound."""
+    name, B, S, N, H, C, dt, layout, kind = spec
+    w = Workload(name, B, S, N, H, C, dt, layout, 1.0, "none", zlib.crc32(name.encode()) % 100000 + 11)
+    inp = workload_inputs(w)
+    inp["mask_bias"] = finite_mask(w, kind, w.seed + 1)
+    gpu = gpu_fwd_bwd(to_gpu(inp))
+    ref = oracle_fwd_bwd(inp)
+    compare_all(w.name, gpu, ref, w.dtype, beyond_output_rounding=kind != "gauss1")
 
 
 def test_tiny_fp32_config():
