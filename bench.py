@@ -2,18 +2,26 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = one forward and one backward pass (every kernel of the path) over
-one batch of the workload's synthetic inputs, which are resident in HBM when
-the timed region starts.  The L2 cache (126 MB) is flushed before every step
-by writing a 256 MB buffer outside the per-step CUDA-event brackets.  The
+One step = R forward and backward passes (every kernel of the path) over one
+batch of the workload's synthetic inputs, which are resident in HBM when the
+timed region starts; R (``passes_per_step`` in the JSON line, usually 1) is
+the smallest count that makes the K timed steps last at least 0.5 s, so that
+the clock samples see the GPU under load.  The default workload is the long
+triangle attention (N_res = 1536).  The L2 cache (126 MB) is flushed before
+every pass by writing a 256 MB buffer outside the per-pass CUDA-event
+brackets.  The
 metric is achieved TFLOP/s (FlashAttention flop convention: 4*L*C forward,
 10*L*C backward, L = B*S*H*N^2 logits) and its fraction of the measured bf16
 dense tensor peak.
 
-Multi-GPU: rows are independent problems, so every rank runs its own batch of
-the same workload with no collective on the data path (weak scaling); the
-reported time is the max over ranks and ``value`` counts the work of all
-ranks.
+Multi-GPU (attention workloads): one problem, its rows s split over the N
+ranks (strong scaling).  The forward needs no communication; the backward's
+one exchange, the all-gather of the fp32 d_pair_bias partials over NCCL and
+their rank-ordered sum, is inside the timed region and reported on its own
+next to its NVLink floor.  The reported time is the max over ranks and
+``value`` counts the whole problem once.  The other workloads (projection,
+triangular update, outer product mean) run independent replicas (weak
+scaling).
 
 ``--impl reference`` times the fp64 CPU oracle (the correctness reference)
 on a bounded sample of the same workload, on this host's cores.
@@ -244,13 +252,16 @@ def algorithmic(w, phase: str):
     ff, bf = flops(w)
     if phase == "fwd_main":                      # q, k, v, g, mask, bias -> out, lse
         return ff, rows * w.C * e * 5 + (mask + pair) * e + stats
-    # q, k, v, gated dout, lse, D, mask, bias -> dq, dk, dv, d_pair_bias (fp32)
-    return bf, rows * w.C * e * 7 + (mask + pair) * e + 2 * stats + pair * 4
+    if phase == "bwd_dbias":                     # q, k, v, gated dout, lse, D, mask, bias -> d_pair_bias
+        # its own work: S and dP recomputed (two of the five backward products), 4*C per logit
+        return 4 * w.logits * w.C, rows * w.C * e * 4 + (mask + pair) * e + 2 * stats + pair * 4
+    # q, k, v, gated dout, lse, D, mask, bias -> dq, dk, dv (all five products, 10*C per logit)
+    return bf, rows * w.C * e * 7 + (mask + pair) * e + 2 * stats
 
 
 def roofline(w, kt, pk, timed_s: float):
     """Roofline entry for the main kernel that took the most device time in the timed region."""
-    phase = max(("fwd_main", "bwd_main"), key=lambda p: kt[p][1])
+    phase = max(("fwd_main", "bwd_main", "bwd_dbias"), key=lambda p: kt[p][1])
     n, ms = kt[phase]
     if n == 0:
         return None
@@ -263,9 +274,10 @@ def roofline(w, kt, pk, timed_s: float):
     tr = TRAFFIC.get((phase, w.name))
     if tr is not None and tr[2] is not None and _source_sha(tr[1]) == tr[2]:
         traffic = tr[0]
-    kernel = {"fwd_main": "fwd::fwd_bf16_kernel", "bwd_main": "bwd::bwd_main_kernel"}[phase]
+    kernel = {"fwd_main": "fwd::fwd_bf16_kernel", "bwd_main": "bwd::bwd_main_kernel",
+              "bwd_dbias": "dbias::dbias_kernel"}[phase]
     if w.dtype != "bf16":
-        kernel = {"fwd_main": "simt::fwd_kernel", "bwd_main": "simt backward"}[phase]
+        kernel = {"fwd_main": "simt::fwd_kernel", "bwd_main": "simt backward", "bwd_dbias": "simt backward"}[phase]
     common = {"kernel": kernel, "launches": n, "us_per_launch": sec * 1e6, "flops_per_launch": fl,
               "algorithmic_bytes_per_launch": by, "traffic": traffic,
               "tensor_floor_us": t_tensor * 1e6, "hbm_floor_us": t_hbm * 1e6}
@@ -387,6 +399,191 @@ def run_e2e(K: int, h2d, compute, d2h, world: int, dev, barrier) -> float:
     e1.record(cur)
     torch.cuda.synchronize()
     return max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+
+
+MIN_TIMED_S = 0.5
+
+
+# ---------------------------------------------------------------------------
+# Several GPUs: the rows s of one problem split over the ranks (row_shards).
+
+
+def row_block(inp: dict, s0: int, s1: int) -> dict:
+    """Rows [s0, s1) of one problem: the per-row tensors and the mask sliced (contiguous
+    copies, so a transposed-pair layout becomes a plain block), the pair bias whole."""
+    return {k: (v if v is None or k == "pair_bias" else v[:, s0:s1].contiguous()) for k, v in inp.items()}
+
+
+def split_pass(blk: dict, group=None, fwd=None, bwd=None, **bwd_kw):
+    """One forward + backward pass of this rank's row block, with d_pair_bias summed over
+    every rank of ``group`` (rank order).  fwd / bwd default to row_shards.attn_fwd /
+    attn_bwd; returns (out, lse, grads)."""
+    from evoformer_pair_bias_b200 import row_shards
+    fwd = fwd or row_shards.attn_fwd
+    bwd = bwd or row_shards.attn_bwd
+    out, lse = fwd(blk["q"], blk["k"], blk["v"], blk["g"], blk["mask_bias"], blk["pair_bias"])
+    grads = bwd(blk["q"], blk["k"], blk["v"], blk["g"], blk["mask_bias"], blk["pair_bias"], out, lse, blk["dout"],
+                group=group, **bwd_kw)
+    return out, lse, grads
+
+
+def run_row_split(args, w, rank, world, local):
+    """--gpus N > 1: one problem, its rows split over the N ranks (strong scaling).
+
+    Each rank runs the forward and backward of its own block of rows; the one
+    exchange is the all-gather of the fp32 d_pair_bias partials (NCCL) and
+    their rank-ordered sum (evo_sum_partials), inside the timed region.  The
+    pass's time is the slowest rank's; ``value`` counts the whole problem once.
+    """
+    import datetime
+
+    import torch.distributed as dist
+    from evoformer_pair_bias_b200 import row_shards
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        A.load_library()
+        s0, s1 = row_shards.row_range(w.S, world, rank)
+        inp = make_inputs(w, device="cpu")
+        host = row_block(inp, s0, s1)
+        blk = {k: (None if v is None else v.to(dev)) for k, v in host.items()}
+        bw = w.with_(S=s1 - s0, layout="msa_row" if w.layout == "tri_end" else w.layout)
+        q = blk["q"]
+        out = A.empty_like_rows(q)
+        lse = torch.empty((w.B, s1 - s0, w.H, w.N), dtype=torch.float32, device=dev)
+        grads = {n: A.empty_like_rows(q) for n in ("dq", "dk", "dv", "dg")}
+        grads["d_pair_bias"] = torch.empty((w.B, 1, w.H, w.N, w.N), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(A.workspace_bytes(q), 1), dtype=torch.uint8, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        out_lo = A.empty_like_rows(q) if w.dtype == "bf16" else None
+
+        def fwd_bwd(evs=None):
+            if evs:
+                evs[0].record()
+            row_shards.attn_fwd(q, blk["k"], blk["v"], blk["g"], blk["mask_bias"], blk["pair_bias"], out=out,
+                                lse=lse, out_lo=out_lo)
+            if evs:
+                evs[1].record()
+            _, pending = row_shards.attn_bwd(q, blk["k"], blk["v"], blk["g"], blk["mask_bias"], blk["pair_bias"],
+                                             out, lse, blk["dout"], grads=grads, workspace=ws, async_op=True,
+                                             out_lo=out_lo)
+            if evs:
+                evs[2].record()
+            pending.wait()
+            if evs:
+                evs[3].record()
+
+        A.timing_enable(True)
+        wev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        for i in range(args.warmup):
+            flush.zero_()
+            fwd_bwd(wev if i == args.warmup - 1 else None)
+        torch.cuda.synchronize()
+        A.timing_collect()
+        if A.device_status(clear=True) != 0:
+            raise RuntimeError("a kernel reported a timed-out wait during warm-up")
+        K = args.steps
+        R = passes_per_step(wev[0].elapsed_time(wev[3]), K, world, dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K * R)]
+        with ClockSampler(gpu_uuid(dev)) as clk:
+            dist.barrier()
+            torch.cuda.synchronize()
+            n0 = A.launch_count()
+            for i in range(K * R):
+                flush.zero_()
+                fwd_bwd(ev[i])
+            torch.cuda.synchronize()
+            dist.barrier()
+            launches = A.launch_count() - n0
+        kt = A.timing_collect()
+        A.timing_enable(False)
+        f_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+        b_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+        x_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
+        tot = sum(e[0].elapsed_time(e[3]) for e in ev)
+        tot, f_ms, b_ms, x_ms = max_over_ranks([tot, f_ms, b_ms, x_ms], world, dev)
+        if A.device_status(clear=True) != 0:
+            raise RuntimeError("a kernel reported a timed-out wait during the timed region")
+        ff, bf = flops(w)
+        value = (ff + bf) * K * R / (tot * 1e-3) / 1e12
+
+        # end to end: each rank copies its block in from pinned host memory and its results out
+        e2e = None
+        if not args.no_e2e:
+            hin = {k: (None if v is None else v.pin_memory()) for k, v in host.items()}
+            h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
+            slots = []
+            for _ in range(2):
+                sl = {"in": {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in hin.items()}}
+                sl["host"] = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                              "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
+                for n_, g_ in grads.items():
+                    sl["host"][n_] = torch.empty(g_.shape, dtype=g_.dtype).pin_memory()
+                slots.append(sl)
+            d2h = sum(v.numel() * v.element_size() for v in slots[0]["host"].values())
+            res = [{}, {}]
+
+            def e2e_h2d(b):
+                for k_, v_ in hin.items():
+                    if v_ is not None:
+                        slots[b]["in"][k_].copy_(v_, non_blocking=True)
+
+            def e2e_compute(b):
+                o, l_, g_ = split_pass(slots[b]["in"], workspace=ws)
+                res[b] = dict(g_, out=o, lse=l_)
+
+            def e2e_d2h(b):
+                for n_, t_ in slots[b]["host"].items():
+                    t_.copy_(res[b][n_], non_blocking=True)
+
+            et = run_e2e(K, e2e_h2d, e2e_compute, e2e_d2h, world, dev, dist.barrier)
+            e2e = {"value": (ff + bf) * K / (et * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": et / K,
+                   "note": "per rank: its row block in, its results and the summed d_pair_bias out"}
+        if rank == 0:
+            pk = peaks()
+            pair = w.B * w.H * w.N * w.N
+            link_gbs = 770.0
+            line = {
+                "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": tot / K, "ms_per_pass": tot / (K * R),
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+                "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "N_seq": w.S, "N_res": w.N, "H": w.H, "c": w.C,
+                           "layout": w.layout, "mask": w.mask, "passes_per_step": R,
+                           "l2": "flushed (256 MB write) before every pass, outside the timed brackets",
+                           "parallelism": f"rows s split over {world} ranks ({s1 - s0} on rank 0); d_pair_bias "
+                                          "partials all-gathered with NCCL and summed in rank order"},
+                "fwd": {"us_per_call": 1e3 * f_ms / (K * R)},
+                "bwd": {"us_per_call": 1e3 * b_ms / (K * R)},
+                "exchange": {"us_per_pass": 1e3 * x_ms / (K * R), "bytes_in_per_rank": (world - 1) * pair * 4,
+                             "nvlink_floor_us": (world - 1) * pair * 4 / (link_gbs * 1e9) * 1e6,
+                             "link_gbs": link_gbs, "what": "all-gather wait + evo_sum_partials, after the "
+                                                           "backward kernels"},
+                "roofline": roofline(bw, kt, pk, timed_s=tot * 1e-3),
+                "kernels": {p_: {"launches": kt[p_][0], "us_per_launch": 1e3 * kt[p_][1] / max(kt[p_][0], 1)}
+                            for p_ in A.PHASES if kt[p_][0]},
+                "cpu_baseline": None,
+                "e2e": e2e,
+                "gpu_launches": launches,
+                "clocks": clk.summary(),
+            }
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.destroy_process_group()
+    return 0
+
+
+def passes_per_step(pass_ms: float, steps: int, world: int, device) -> int:
+    """Forward + backward passes per timed step so that `steps` steps take >= MIN_TIMED_S.
+
+    From one warm-up pass's device time (the slowest rank's, so every rank
+    agrees); at least 1.
+    """
+    pass_ms = max_over_ranks([pass_ms], world, device)[0]
+    need = MIN_TIMED_S * 1e3 / max(pass_ms * max(steps, 1), 1e-6)
+    return max(1, int(np.ceil(need)))
 
 
 def run_reference(args, w, rank, world):
@@ -525,12 +722,10 @@ def run_projection(args, pw, rank, world, local):
         print(json.dumps(line), flush=True)
         return 0
 
-    import datetime
+    if world > 1:
+        return run_row_split(args, w, rank, world, local)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     def barrier():
         if world > 1:
@@ -1060,7 +1255,7 @@ def run_opm(args, ow, rank, world, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS) + sorted(PROJ_WORKLOADS) + sorted(TRI_MUL_WORKLOADS) + sorted(OPM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -1105,42 +1300,58 @@ def main():
     grads["d_pair_bias"] = torch.empty((w.B, 1, w.H, w.N, w.N), dtype=torch.float32, device=dev)
     ws = torch.empty(max(A.workspace_bytes(d["q"]), 1), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # bf16: the forward also writes out's rounding residual, which the backward uses for D_i
+    out_lo = A.empty_like_rows(d["q"]) if w.dtype == "bf16" else None
+
+    def fwd():
+        A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out=out, lse=lse,
+                       out_lo=out_lo)
+
+    def bwd():
+        A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out, lse, dout,
+                       grads=grads, workspace=ws, out_lo=out_lo)
 
     def step():
-        A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out=out, lse=lse)
-        A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out, lse, dout,
-                       grads=grads, workspace=ws)
+        fwd()
+        bwd()
 
     A.timing_enable(True)
-    for _ in range(args.warmup):
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for i in range(args.warmup):
         flush.zero_()
+        if i == args.warmup - 1:
+            wev[0].record()
         step()
+    wev[1].record()
     torch.cuda.synchronize()
     A.timing_collect()
     if A.device_status(clear=True) != 0:
         raise RuntimeError("a kernel reported a timed-out wait during warm-up")
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    # Passes per step: enough forward + backward passes that the K timed steps
+    # span at least MIN_TIMED_S of device time (so that the clock samples see
+    # the GPU under load), the same number on every rank.
+    R = passes_per_step(wev[0].elapsed_time(wev[1]), K, world, dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K * R)]
     with ClockSampler(gpu_uuid(dev)) as clk:
         barrier()
         torch.cuda.synchronize()
         n0 = A.launch_count()
-        for i in range(K):
+        for i in range(K * R):
             flush.zero_()
             ev[i][0].record()
-            A.evo_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out=out, lse=lse)
+            fwd()
             ev[i][1].record()
-            A.evo_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out, lse, dout,
-                           grads=grads, workspace=ws)
+            bwd()
             ev[i][2].record()
         torch.cuda.synchronize()
         barrier()
         launches = A.launch_count() - n0
     kt = A.timing_collect()
     A.timing_enable(False)
-    fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K * R)]
+    bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K * R)]
     tot_ms = sum(fwd_ms) + sum(bwd_ms)
     tot_ms, fsum, bsum = max_over_ranks([tot_ms, sum(fwd_ms), sum(bwd_ms)], world, dev)
     if A.device_status(clear=True) != 0:
@@ -1148,9 +1359,9 @@ def main():
 
     ff, bf = flops(w)
     pk = peaks()
-    value = job_throughput(ff + bf, K, world, tot_ms)
-    fwd_tf = ff * K / (fsum * 1e-3) / 1e12
-    bwd_tf = bf * K / (bsum * 1e-3) / 1e12
+    value = job_throughput(R * (ff + bf), K, world, tot_ms)
+    fwd_tf = ff * K * R / (fsum * 1e-3) / 1e12
+    bwd_tf = bf * K * R / (bsum * 1e-3) / 1e12
 
     # end to end: pinned host inputs -> device, fwd + bwd through the public API, results -> pinned host
     e2e = None
@@ -1165,6 +1376,7 @@ def main():
         for _ in range(2):           # device inputs, outputs and pinned host results per buffer set
             sl = {"in": {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in hin.items()},
                   "out": A.empty_like_rows(d["q"]),
+                  "out_lo": A.empty_like_rows(d["q"]) if w.dtype == "bf16" else None,
                   "lse": torch.empty((w.B, w.S, w.H, w.N), dtype=torch.float32, device=dev),
                   "dout": A.empty_like_rows(d["q"]),
                   "grads": {n: A.empty_like_rows(d["q"]) for n in ("dq", "dk", "dv", "dg")}}
@@ -1185,10 +1397,12 @@ def main():
             sl = slots[b]
             di = sl["in"]
             q, k_, v_, g_, do = (logical_view(w, di[n]) for n in ("q", "k", "v", "g", "dout"))
-            o, l_ = A.evo_attn_fwd(q, k_, v_, g_, di["mask_bias"], di["pair_bias"], out=sl["out"], lse=sl["lse"])
+            r = A.evo_attn_fwd(q, k_, v_, g_, di["mask_bias"], di["pair_bias"], out=sl["out"], lse=sl["lse"],
+                               out_lo=sl["out_lo"])
+            o, l_ = r[0], r[1]
             do = do if do.stride() == o.stride() else sl["dout"].copy_(do)
             A.evo_attn_bwd(q, k_, v_, g_, di["mask_bias"], di["pair_bias"], o, l_, do, grads=sl["grads"],
-                           workspace=ws)
+                           workspace=ws, out_lo=sl["out_lo"])
 
         def e2e_d2h(b):
             sl = slots[b]
@@ -1212,18 +1426,23 @@ def main():
             cpu = {"error": repr(exc)}
 
     if rank == 0:
-        fwd_us = 1e3 * fsum / K
+        fwd_us = 1e3 * fsum / (K * R)
         roof = roofline(w, kt, pk, timed_s=tot_ms * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": tot_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N_seq": w.S, "N_res": w.N, "H": w.H, "c": w.C,
-                       "layout": w.layout, "mask": w.mask, "l2": "flushed (256 MB write) before every step",
-                       "parallelism": f"replicas x{world}, rows independent, no collective"},
+                       "layout": w.layout, "mask": w.mask, "passes_per_step": R,
+                       "l2": "flushed (256 MB write) before every forward + backward pass, outside the timed "
+                             "brackets" + ("; inputs also larger than L2" if 5 * w.B * w.S * w.N * w.H
+                                                                            * w.C * 2 > (126 << 20) else ""),
+                       "parallelism": "one GPU (with --gpus N the rows are split over N ranks)"},
+            "ms_per_pass": tot_ms / (K * R),
             "fwd": {"tflops": fwd_tf, "us_per_call": fwd_us, "frac_measured_peak": fwd_tf / pk["bf16"],
                     "frac_nominal_peak": fwd_tf / NOMINAL_BF16_TFLOPS},
-            "bwd": {"tflops": bwd_tf, "us_per_call": 1e3 * bsum / K, "frac_measured_peak": bwd_tf / pk["bf16"],
+            "bwd": {"tflops": bwd_tf, "us_per_call": 1e3 * bsum / (K * R),
+                    "frac_measured_peak": bwd_tf / pk["bf16"],
                     "frac_nominal_peak": bwd_tf / NOMINAL_BF16_TFLOPS},
             "frac_measured_peak": value / world / pk["bf16"],
             "roofline": roof,
