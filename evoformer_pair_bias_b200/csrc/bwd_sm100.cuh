@@ -20,7 +20,9 @@
 //   bwd_main       CTA = (key tile j, row group g, b*H + h); loops over the
 //                  group's rows s (outer) and query tiles i (inner):
 //                    S^T  = K_j Q_i^T      dP^T = V_j (dOa_hi + dOa_lo)_i^T  (TMEM)
-//                    P^T  = exp2(S^T*scale*log2e + bias + mask + nl_i)
+//                    P^T  = exp2(S^T*scale*log2e + bias*log2e*r1/sqrt(C) + mask + nl_i)
+//                    (the pair bias with the scale the forward's tensor core gives it,
+//                    r1 = bf16(sqrt(C)), so that P matches the forward's lse)
 //                    dS^T = P^T (dP^T - D_i)
 //                    dV_j += P^T dOa_hi_i  dK_j += dS^T Q_i         (TMEM)
 //                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
@@ -79,12 +81,15 @@ constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 // Warps 0..7: two dS warpgroups (queries 0..63 / 64..127 of the tile); warp 8 TMA;
 // three MMA issuers, so that no single issuing thread serialises a step's 33
-// instructions: warp 9 S^T and dP^T of the next step, warp 10 dV and dK, warp 11 dQ.  The last warpgroup hands registers to the dS
-// warpgroups: 2*128*208 + 128*88 = 384*168, the launch's register pool.
-constexpr int THREADS = 384;
-constexpr int LAUNCH_REGS = 168;
-constexpr uint32_t DS_REGS = 208, CONTROL_REGS = 88;
-static_assert((2 * DS_REGS + CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
+// instructions: warp 9 S^T and dP^T of the next step, warp 10 dV and dK, warp 11 dQ.
+// Warps 12..15 drain dQ: each step's 128 x 32 fp32 product goes from TMEM into the
+// global fp32 accumulator with vector reductions, off the dS warps' path.
+// The two control warpgroups hand registers to the dS warpgroups:
+// 2*128*200 + 2*128*56 = 512*128, the launch's register pool.
+constexpr int THREADS = 512;
+constexpr int LAUNCH_REGS = 128;
+constexpr uint32_t DS_REGS = 200, CONTROL_REGS = 56;
+static_assert((2 * DS_REGS + 2 * CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
 // TMEM columns: S^T, dP^T, two P^T buffers (bf16 pairs), dV, dK, dQ accumulators
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 384, TM_DK = 416, TM_DQ = 448, TM_COLS = 512;
 
@@ -106,6 +111,7 @@ struct MainParams {
     int n_it;            // query tiles
     int gsz;             // rows s per group
     float sc2;           // log2(e) / sqrt(C)
+    float bsc;           // log2(e) * r1 / sqrt(C): the pair bias enters as the forward's tensor core adds it
     float rs;            // 1 / sqrt(C)
     float r_bf16;        // r1 = bf16(sqrt(C))
     float r2_bf16;       // r2 = bf16(sqrt(C) - r1): the mask enters as (r1 + r2) * mask
@@ -175,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(sdp_free, 8);
         mbar_init(ds_free, 2);                    // dK and dQ read the dS^T tile
         mbar_init(dq_full, 1);
-        mbar_init(dq_free, 8);
+        mbar_init(dq_free, 4);                    // the dQ drain warps
         mbar_init(dkv_full, 1);
         mbar_init(dkv_free, 8);
         for (int x = 0; x < 3; ++x) mbar_init(mma_done(x), 1);
@@ -226,157 +232,187 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProducer) {
+    // setmaxnreg is warpgroup-wide: all four warps of a warpgroup execute the same
+    // instruction, so each warpgroup changes its count before its warps' roles split.
+    if (warp >= 8) {
         regs_decrease<CONTROL_REGS>();
-        // ---------------------------------------------------------------- producer
-        if (lane == 0 && T > 0) {
-            int kv_issued[2] = {0, 0}, x_issued[X_STAGES] = {}, y_issued[Y_STAGES] = {};
-            bool ok = true;
-            for (int si = 0; si < ns && ok; ++si) {
-                const int s = s_begin + si, x = si & 1;
-                const uint32_t kb = base + OFF_KV + x * KVB;
-                if (si >= 2) ok = mbar_wait(kv_empty(x), ((si >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01);
-                if (!ok) break;
-                mbar_arrive_expect_tx(kv_full(x), 2 * TILE_BYTES + (HAS_MASK ? 512 : 0));
-                tma_load_5d(kb + KV_K, &tm_k, kv_full(x), 0, j0, h, s, b);
-                tma_load_5d(kb + KV_V, &tm_v, kv_full(x), 0, j0, h, s, b);
-                if (HAS_MASK) {   // mask row of s into rows 0 and 8 of the two 64-key halves of the A block
-                    tma_load_3d(kb + KV_MASK, &tm_mask, kv_full(x), j0, s, b);
-                    tma_load_3d(kb + KV_MASK + 1024, &tm_mask, kv_full(x), j0, s, b);
-                    tma_load_3d(kb + KV_MASK + 2048, &tm_mask, kv_full(x), j0 + 64, s, b);
-                    tma_load_3d(kb + KV_MASK + 3072, &tm_mask, kv_full(x), j0 + 64, s, b);
+        if (warp == kProducer) {
+            // ---------------------------------------------------------------- producer
+            if (lane == 0 && T > 0) {
+                int kv_issued[2] = {0, 0}, x_issued[X_STAGES] = {}, y_issued[Y_STAGES] = {};
+                bool ok = true;
+                for (int si = 0; si < ns && ok; ++si) {
+                    const int s = s_begin + si, x = si & 1;
+                    const uint32_t kb = base + OFF_KV + x * KVB;
+                    if (si >= 2) ok = mbar_wait(kv_empty(x), ((si >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(kv_full(x), 2 * TILE_BYTES + (HAS_MASK ? 512 : 0));
+                    tma_load_5d(kb + KV_K, &tm_k, kv_full(x), 0, j0, h, s, b);
+                    tma_load_5d(kb + KV_V, &tm_v, kv_full(x), 0, j0, h, s, b);
+                    if (HAS_MASK) {   // mask row of s into rows 0 and 8 of the two 64-key halves of the A block
+                        tma_load_3d(kb + KV_MASK, &tm_mask, kv_full(x), j0, s, b);
+                        tma_load_3d(kb + KV_MASK + 1024, &tm_mask, kv_full(x), j0, s, b);
+                        tma_load_3d(kb + KV_MASK + 2048, &tm_mask, kv_full(x), j0 + 64, s, b);
+                        tma_load_3d(kb + KV_MASK + 3072, &tm_mask, kv_full(x), j0 + 64, s, b);
+                    }
+                    ++kv_issued[x];
+                    for (int it = 0; it < ni; ++it) {
+                        const int t = si * ni + it, i0 = it * BQ;
+                        const int xs = t % X_STAGES, ys = t % Y_STAGES;
+                        const uint32_t xb = base + OFF_X + xs * XB, yb = base + OFF_Y + ys * YB;
+                        if (t >= X_STAGES)
+                            ok = mbar_wait(x_empty(xs), ((t / X_STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(x_full(xs), TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 4 * 256);
+                        if (HAS_BIAS) {
+                            tma_load_4d(xb + X_BT, &tm_bt, x_full(xs), i0, j0, h, b);
+                            tma_load_4d(xb + X_BT + BT_BOX, &tm_bt, x_full(xs), i0 + 64, j0, h, b);
+                        }
+                        tma_load_5d(xb + X_DOL, &tm_dol, x_full(xs), 0, i0, h, s, b);
+                        // rows 0..1 (high, low) of the two 64-query atoms of the nl and -D blocks
+                        tma_load_5d(xb + X_NL, &tm_nl, x_full(xs), i0, 0, h, s, b);
+                        tma_load_5d(xb + X_NL + 2048, &tm_nl, x_full(xs), i0 + 64, 0, h, s, b);
+                        tma_load_5d(xb + X_ND, &tm_d, x_full(xs), i0, 0, h, s, b);
+                        tma_load_5d(xb + X_ND + 2048, &tm_d, x_full(xs), i0 + 64, 0, h, s, b);
+                        ++x_issued[xs];
+                        if (t >= Y_STAGES)
+                            ok = mbar_wait(y_empty(ys), ((t / Y_STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x05);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(y_full(ys), 2 * TILE_BYTES);
+                        tma_load_5d(yb + Y_Q, &tm_q, y_full(ys), 0, i0, h, s, b);
+                        tma_load_5d(yb + Y_DOH, &tm_doa, y_full(ys), 0, i0, h, s, b);
+                        ++y_issued[ys];
+                    }
                 }
-                ++kv_issued[x];
-                for (int it = 0; it < ni; ++it) {
-                    const int t = si * ni + it, i0 = it * BQ;
+                volatile int no_abort = 0;
+                for (int x = 0; x < 2; ++x)
+                    if (kv_issued[x]) mbar_wait(kv_full(x), (kv_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x03);
+                for (int x = 0; x < X_STAGES; ++x)
+                    if (x_issued[x]) mbar_wait(x_full(x), (x_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
+                for (int x = 0; x < Y_STAGES; ++x)
+                    if (y_issued[x]) mbar_wait(y_full(x), (y_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x06);
+            }
+        } else if (warp == kMma || warp == kMmaKV || warp == kMmaQ) {
+            // ---------------------------------------------------------------- MMA issuers
+            const int role = warp - kMma;            // 0: S^T, dP^T   1: dV, dK   2: dQ
+            if (lane == 0 && T > 0) {
+                constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // S^T, dP^T
+                constexpr uint32_t ID_RT = idesc_bf16(BK, BQ, false, true);    // ones x rank-term block
+                constexpr uint32_t ID_MK = idesc_bf16(BK, BQ, true, false);    // mask block x r-row
+                constexpr uint32_t ID_KV = idesc_bf16(BK, HD, false, true);    // dV, dK (B MN-major)
+                constexpr uint32_t ID_Q = idesc_bf16(BQ, HD, true, true);      // dQ (A and B MN-major)
+                bool ok = true;
+                const uint32_t ds = base + OFF_DS;
+                for (int t = 0; ok && t < T; ++t) {
+                    const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
                     const int xs = t % X_STAGES, ys = t % Y_STAGES;
-                    const uint32_t xb = base + OFF_X + xs * XB, yb = base + OFF_Y + ys * YB;
-                    if (t >= X_STAGES)
-                        ok = mbar_wait(x_empty(xs), ((t / X_STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x02);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(x_full(xs), TILE_BYTES + (HAS_BIAS ? 2 * BT_BOX : 0) + 4 * 256);
-                    if (HAS_BIAS) {
-                        tma_load_4d(xb + X_BT, &tm_bt, x_full(xs), i0, j0, h, b);
-                        tma_load_4d(xb + X_BT + BT_BOX, &tm_bt, x_full(xs), i0 + 64, j0, h, b);
+                    const uint32_t kb = base + OFF_KV + x * KVB, xb = base + OFF_X + xs * XB, yb = base + OFF_Y + ys * YB;
+                    if (role == 0) {
+                        // S^T = K Q^T - lse*sqrt(C) (+ (r1 + r2) * mask_j);  dP^T = V (dOa_hi + dOa_lo)^T - D.
+                        // Step t's products are issued as soon as the dS warps hold step t-1's in registers.
+                        if (it == 0) ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x11);
+                        if (ok) ok = mbar_wait(x_full(xs), (t / X_STAGES) & 1, abort_flag, kTimeoutBase | 0x12);
+                        if (ok) ok = mbar_wait(y_full(ys), (t / Y_STAGES) & 1, abort_flag, kTimeoutBase | 0x1D);
+                        if (ok && t > 0) ok = mbar_wait(sdp_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x13);
+                        if (!ok) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk)
+                            mma_ss(tmem + TM_ST, smem_desc(kb + KV_K + kk * 32, 16, 512, kSw64),
+                                   smem_desc(yb + Y_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                        mma_ss(tmem + TM_ST, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                               smem_desc(xb + X_NL, 2048, 1024, kSw128), ID_RT, 1u);
+                        if (HAS_MASK)
+                            mma_ss(tmem + TM_ST, smem_desc(kb + KV_MASK, 2048, 1024, kSw128),
+                                   smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk)
+                            mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
+                                   smem_desc(yb + Y_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk)
+                            mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
+                                   smem_desc(xb + X_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
+                        mma_ss(tmem + TM_DPT, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                               smem_desc(xb + X_ND, 2048, 1024, kSw128), ID_RT, 1u);
+                        mma_commit(sdp_full);
+                        mma_commit(x_empty(xs));
+                        mma_commit(y_empty(ys));
+                        if (it == ni - 1) mma_commit(kv_empty(x));
+                    } else if (role == 1) {
+                        // dV_j += P^T dOa_hi;  dK_j += dS^T Q
+                        ok = mbar_wait(y_full(ys), (t / Y_STAGES) & 1, abort_flag, kTimeoutBase | 0x14);
+                        if (ok) ok = mbar_wait(ds_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x15);
+                        if (ok && it == 0 && si > 0) ok = mbar_wait(dkv_free, (si - 1) & 1, abort_flag, kTimeoutBase | 0x16);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const int pb = t & 1;                // P^T buffer of this step
+#pragma unroll
+                        for (int kk = 0; kk < BQ / 16; ++kk)
+                            mma_ts(tmem + TM_DV, tmem + TM_PT + pb * 64 + kk * 8,
+                                   smem_desc(yb + Y_DOH + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(pt_free(pb));
+#pragma unroll
+                        for (int kk = 0; kk < BQ / 16; ++kk) {
+                            const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
+                            mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128),
+                                   smem_desc(yb + Y_Q + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(ds_free);
+                        mma_commit(y_empty(ys));
+                        if (it == ni - 1) mma_commit(dkv_full);
+                    } else {
+                        // dQ_i = dS K_j
+                        if (it == 0) ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x17);
+                        if (ok) ok = mbar_wait(ds_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x18);
+                        if (ok && t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x19);
+                        if (!ok) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
+                                   smem_desc(kb + KV_K + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
+                        mma_commit(ds_free);
+                        mma_commit(dq_full);
+                        if (it == ni - 1) mma_commit(kv_empty(x));
                     }
-                    tma_load_5d(xb + X_DOL, &tm_dol, x_full(xs), 0, i0, h, s, b);
-                    // rows 0..1 (high, low) of the two 64-query atoms of the nl and -D blocks
-                    tma_load_5d(xb + X_NL, &tm_nl, x_full(xs), i0, 0, h, s, b);
-                    tma_load_5d(xb + X_NL + 2048, &tm_nl, x_full(xs), i0 + 64, 0, h, s, b);
-                    tma_load_5d(xb + X_ND, &tm_d, x_full(xs), i0, 0, h, s, b);
-                    tma_load_5d(xb + X_ND + 2048, &tm_d, x_full(xs), i0 + 64, 0, h, s, b);
-                    ++x_issued[xs];
-                    if (t >= Y_STAGES)
-                        ok = mbar_wait(y_empty(ys), ((t / Y_STAGES) - 1) & 1, abort_flag, kTimeoutBase | 0x05);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(y_full(ys), 2 * TILE_BYTES);
-                    tma_load_5d(yb + Y_Q, &tm_q, y_full(ys), 0, i0, h, s, b);
-                    tma_load_5d(yb + Y_DOH, &tm_doa, y_full(ys), 0, i0, h, s, b);
-                    ++y_issued[ys];
+                }
+                // Drain: every MMA issued by this thread has finished before TMEM is released.
+                mma_commit(mma_done(role));
+                volatile int no_abort = 0;
+                mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x1A + role));
+            }
+        } else {
+            // ---------------------------------------------------------------- dQ drain warps
+            // dQ_i of step t (lanes = queries) into the fp32 accumulator, scaled by 1/sqrt(C).
+            const int quad = warp & 3;
+            const int r = quad * 32 + lane;
+            const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+            for (int t = 0; t < T; ++t) {
+                if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) break;
+                tc_fence_after();
+                uint32_t v[32];
+                tmem_ld32_sync(lane_addr + TM_DQ, v);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dq_free);
+                const int si = t / ni, it = t - si * ni;
+                const int i = it * BQ + r, s = s_begin + si;
+                if (i < p.N) {
+                    float* dst = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + i) * p.H + h) * HD;
+#pragma unroll
+                    for (int c = 0; c < HD; c += 4) {
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c),
+                                     "f"(__uint_as_float(v[c]) * p.rs), "f"(__uint_as_float(v[c + 1]) * p.rs),
+                                     "f"(__uint_as_float(v[c + 2]) * p.rs), "f"(__uint_as_float(v[c + 3]) * p.rs)
+                                     : "memory");
+                    }
                 }
             }
-            volatile int no_abort = 0;
-            for (int x = 0; x < 2; ++x)
-                if (kv_issued[x]) mbar_wait(kv_full(x), (kv_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x03);
-            for (int x = 0; x < X_STAGES; ++x)
-                if (x_issued[x]) mbar_wait(x_full(x), (x_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
-            for (int x = 0; x < Y_STAGES; ++x)
-                if (y_issued[x]) mbar_wait(y_full(x), (y_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x06);
         }
-    } else if (warp == kMma || warp == kMmaKV || warp == kMmaQ) {
-        regs_decrease<CONTROL_REGS>();
-        // ---------------------------------------------------------------- MMA issuers
-        const int role = warp - kMma;            // 0: S^T, dP^T   1: dV, dK   2: dQ
-        if (lane == 0 && T > 0) {
-            constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // S^T, dP^T
-            constexpr uint32_t ID_RT = idesc_bf16(BK, BQ, false, true);    // ones x rank-term block
-            constexpr uint32_t ID_MK = idesc_bf16(BK, BQ, true, false);    // mask block x r-row
-            constexpr uint32_t ID_KV = idesc_bf16(BK, HD, false, true);    // dV, dK (B MN-major)
-            constexpr uint32_t ID_Q = idesc_bf16(BQ, HD, true, true);      // dQ (A and B MN-major)
-            bool ok = true;
-            const uint32_t ds = base + OFF_DS;
-            for (int t = 0; ok && t < T; ++t) {
-                const int si = t / ni, it = t - si * ni, x = si & 1, st = t & 1;
-                const int xs = t % X_STAGES, ys = t % Y_STAGES;
-                const uint32_t kb = base + OFF_KV + x * KVB, xb = base + OFF_X + xs * XB, yb = base + OFF_Y + ys * YB;
-                if (role == 0) {
-                    // S^T = K Q^T - lse*sqrt(C) (+ (r1 + r2) * mask_j);  dP^T = V (dOa_hi + dOa_lo)^T - D.
-                    // Step t's products are issued as soon as the dS warps hold step t-1's in registers.
-                    if (it == 0) ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x11);
-                    if (ok) ok = mbar_wait(x_full(xs), (t / X_STAGES) & 1, abort_flag, kTimeoutBase | 0x12);
-                    if (ok) ok = mbar_wait(y_full(ys), (t / Y_STAGES) & 1, abort_flag, kTimeoutBase | 0x1D);
-                    if (ok && t > 0) ok = mbar_wait(sdp_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x13);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        mma_ss(tmem + TM_ST, smem_desc(kb + KV_K + kk * 32, 16, 512, kSw64),
-                               smem_desc(yb + Y_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-                    mma_ss(tmem + TM_ST, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
-                           smem_desc(xb + X_NL, 2048, 1024, kSw128), ID_RT, 1u);
-                    if (HAS_MASK)
-                        mma_ss(tmem + TM_ST, smem_desc(kb + KV_MASK, 2048, 1024, kSw128),
-                               smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
-                               smem_desc(yb + Y_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk)
-                        mma_ss(tmem + TM_DPT, smem_desc(kb + KV_V + kk * 32, 16, 512, kSw64),
-                               smem_desc(xb + X_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
-                    mma_ss(tmem + TM_DPT, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
-                           smem_desc(xb + X_ND, 2048, 1024, kSw128), ID_RT, 1u);
-                    mma_commit(sdp_full);
-                    mma_commit(x_empty(xs));
-                    mma_commit(y_empty(ys));
-                    if (it == ni - 1) mma_commit(kv_empty(x));
-                } else if (role == 1) {
-                    // dV_j += P^T dOa_hi;  dK_j += dS^T Q
-                    ok = mbar_wait(y_full(ys), (t / Y_STAGES) & 1, abort_flag, kTimeoutBase | 0x14);
-                    if (ok) ok = mbar_wait(ds_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x15);
-                    if (ok && it == 0 && si > 0) ok = mbar_wait(dkv_free, (si - 1) & 1, abort_flag, kTimeoutBase | 0x16);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const int pb = t & 1;                // P^T buffer of this step
-#pragma unroll
-                    for (int kk = 0; kk < BQ / 16; ++kk)
-                        mma_ts(tmem + TM_DV, tmem + TM_PT + pb * 64 + kk * 8,
-                               smem_desc(yb + Y_DOH + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(pt_free(pb));
-#pragma unroll
-                    for (int kk = 0; kk < BQ / 16; ++kk) {
-                        const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
-                        mma_ss(tmem + TM_DK, smem_desc(a, 16, 1024, kSw128),
-                               smem_desc(yb + Y_Q + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(ds_free);
-                    mma_commit(y_empty(ys));
-                    if (it == ni - 1) mma_commit(dkv_full);
-                } else {
-                    // dQ_i = dS K_j
-                    if (it == 0) ok = mbar_wait(kv_full(x), (si >> 1) & 1, abort_flag, kTimeoutBase | 0x17);
-                    if (ok) ok = mbar_wait(ds_full(st), (t >> 1) & 1, abort_flag, kTimeoutBase | 0x18);
-                    if (ok && t > 0) ok = mbar_wait(dq_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x19);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_ss(tmem + TM_DQ, smem_desc(ds + kk * 2048, BT_BOX, 1024, kSw128),
-                               smem_desc(kb + KV_K + kk * 1024, TILE_BYTES, 512, kSw64), ID_Q, kk > 0 ? 1u : 0u);
-                    mma_commit(ds_free);
-                    mma_commit(dq_full);
-                    if (it == ni - 1) mma_commit(kv_empty(x));
-                }
-            }
-            // Drain: every MMA issued by this thread has finished before TMEM is released.
-            mma_commit(mma_done(role));
-            volatile int no_abort = 0;
-            mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x1A + role));
-        }
-    } else if (warp < 8) {
+    } else {
         regs_increase<DS_REGS>();
         if (T > 0) {
         // ---------------------------------------------------------------- dS warpgroups
@@ -387,31 +423,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool jvalid = j < p.N;
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
         const uint64_t SC2 = f2(p.sc2, p.sc2);
-        const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
+        const uint64_t L2E2 = f2(p.bsc, p.bsc);
         bool ok = true;
 
-        auto drain_dq = [&](int t) -> bool {     // dQ rows of step t: lanes = queries
-            if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) return false;
-            tc_fence_after();
-            uint32_t v[16];
-            tmem_ld16_sync(lane_addr + TM_DQ + wg * 16, v);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dq_free);
-            const int si = t / ni, it = t - si * ni;
-            const int i = it * BQ + r, s = s_begin + si;
-            if (i < p.N) {
-                float* dst = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + i) * p.H + h) * HD + wg * 16;
-#pragma unroll
-                for (int c = 0; c < 16; c += 4) {
-                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c),
-                                 "f"(__uint_as_float(v[c]) * p.rs), "f"(__uint_as_float(v[c + 1]) * p.rs),
-                                 "f"(__uint_as_float(v[c + 2]) * p.rs), "f"(__uint_as_float(v[c + 3]) * p.rs)
-                                 : "memory");
-                }
-            }
-            return true;
-        };
         auto drain_dkv = [&](int si) -> bool {   // dK (wg 0) / dV (wg 1) of row s: lanes = keys
             if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
             tc_fence_after();
@@ -441,54 +455,66 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[128];                    // [0,64): S^T columns, [64,128): dP^T columns
-            tmem_ld32x4_sync(lane_addr + TM_ST + wg * 64, lane_addr + TM_ST + wg * 64 + 32,
-                             lane_addr + TM_DPT + wg * 64, lane_addr + TM_DPT + wg * 64 + 32, sv);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sdp_free);
-            if (!jvalid) {                       // padded key rows: P = 0
-#pragma unroll
-                for (int c = 0; c < 64; ++c) sv[c] = __float_as_uint(-INFINITY);
-            }
-
+            // the whole bias row of this thread (64 queries) into registers at once, so the
+            // stage of ring X is released early
             const int xs = t % X_STAGES;
             ok = mbar_wait(x_full(xs), (t / X_STAGES) & 1, abort_flag, kTimeoutBase | 0x25);
+            uint32_t bw[32];
+            if (HAS_BIAS) {
+                const uint8_t* bt_ptr = gbase + OFF_X + xs * XB + X_BT + wg * BT_BOX + r * 128;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(bt_ptr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
+                    bw[4 * q] = w.x; bw[4 * q + 1] = w.y; bw[4 * q + 2] = w.z; bw[4 * q + 3] = w.w;
+                }
+            }
+            // the TMA refills this stage once it is released: order the generic-proxy reads above
+            // before that async-proxy write (without the fence the refill can overtake them)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_empty(xs));           // bias tile of this stage consumed
             const int pb = t & 1;                // P^T buffer of this step
             if (ok && t >= 2) ok = mbar_wait(pt_free(pb), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
             if (!ok) break;
             tc_fence_after();
-            const uint8_t* bt_ptr = gbase + OFF_X + xs * XB + X_BT + wg * BT_BOX + r * 128;
+            const uint32_t ts = lane_addr + TM_ST + wg * 64, td = lane_addr + TM_DPT + wg * 64;
             const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * 32;
-            // P = exp2(S^T * sc2 + bias * log2e) (S^T already holds -lse and the mask),
+            // S^T and dP^T 16 queries at a time (v[0,16): S^T columns, v[16,32): dP^T columns).
+            // P = exp2(S^T * sc2 + bias * bsc) (S^T already holds -lse and the mask),
             // dS = P * dP^T (dP^T already holds -D); two columns per op
             uint32_t dk2[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {                      // 8 columns at a time
-                uint32_t bw[4] = {0u, 0u, 0u, 0u};
-                if (HAS_BIAS) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(bt_ptr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
-                    bw[0] = w.x; bw[1] = w.y; bw[2] = w.z; bw[3] = w.w;
+            for (int qd = 0; qd < 4; ++qd) {
+                uint32_t v[32];
+                tmem_ld16x2_sync(ts + qd * 16, td + qd * 16, v);
+                if (qd == 3) {                   // every S^T / dP^T column of this step is in registers
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sdp_free);
                 }
-                float dsq[8];
-                uint32_t pk4[4];
+                if (!jvalid) {                   // padded key rows: P = 0
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = q * 8 + 2 * e;
-                    uint64_t y2 = fmul2(f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), SC2);
-                    if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[e]), L2E2, y2);
-                    const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
-                    const uint64_t ds2 = fmul2(f2(p0, p1), f2(__uint_as_float(sv[64 + c]), __uint_as_float(sv[65 + c])));
-                    dsq[2 * e] = f2lo(ds2);
-                    dsq[2 * e + 1] = f2hi(ds2);
-                    pk4[e] = pack_bf16(p0, p1);
-                    dk2[q * 4 + e] = pack_bf16(dsq[2 * e], dsq[2 * e + 1]);
+                    for (int c = 0; c < 16; ++c) v[c] = __float_as_uint(-INFINITY);
                 }
-                asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt_addr + q * 4),
-                             "r"(pk4[0]), "r"(pk4[1]), "r"(pk4[2]), "r"(pk4[3]));
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {                // 8 columns (one bias chunk) at a time
+                    const int ch = qd * 2 + q2;
+                    uint32_t pk4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = q2 * 8 + 2 * e;             // column within the quarter
+                        uint64_t y2 = fmul2(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), SC2);
+                        if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[ch * 4 + e]), L2E2, y2);
+                        const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
+                        const uint64_t ds2 =
+                            fmul2(f2(p0, p1), f2(__uint_as_float(v[16 + c]), __uint_as_float(v[17 + c])));
+                        pk4[e] = pack_bf16(p0, p1);
+                        dk2[ch * 4 + e] = pack_bf16(f2lo(ds2), f2hi(ds2));
+                    }
+                    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt_addr + ch * 4),
+                                 "r"(pk4[0]), "r"(pk4[1]), "r"(pk4[2]), "r"(pk4[3]));
+                }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(x_empty(xs));           // bias tile of this stage consumed
             if (t > 0) ok = mbar_wait(ds_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x27);
             if (!ok) break;
             const uint32_t ds_row = base + OFF_DS + wg * BT_BOX + r * 128;
@@ -505,20 +531,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(ds_full(st));
 
-            // The previous step's dQ and (at a row change) the previous row's dK/dV
-            // are drained here, after this step's exponentials, so the MMAs that
-            // produce them overlap this step's work.
-            if (t > 0) {
-                ok = drain_dq(t - 1);
-                if (ok && it == 0) ok = drain_dkv(si - 1);
+            // At a row change the previous row's dK/dV are drained here, after this
+            // step's exponentials, so the MMAs that produce them overlap this step's work.
+            if (t > 0 && it == 0) {
+                ok = drain_dkv(si - 1);
                 if (!ok) break;
             }
         }
-        if (ok) ok = drain_dq(T - 1);
         if (ok) ok = drain_dkv(ns - 1);
         }
-    } else {
-        regs_decrease<CONTROL_REGS>();
     }
 
     tc_fence_before();
@@ -848,6 +869,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     mp.rs = 1.0f / sqrtf((float)HD);
     mp.r_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)HD)));
     mp.r2_bf16 = __bfloat162float(__float2bfloat16_rn(sqrtf((float)HD) - mp.r_bf16));
+    mp.bsc = mp.sc2 * mp.r_bf16;
     mp.dq_acc = dq_acc;
     mp.dk = static_cast<__nv_bfloat16*>(c.dk);
     mp.dv = static_cast<__nv_bfloat16*>(c.dv);
@@ -874,6 +896,7 @@ inline evo_status_t run(const Call& c, cudaStream_t stream, int* launched) {
     if (items > 0x7fffffff) return EVO_ERR_UNSUPPORTED;
     dp.n_items = (int)items;
     dp.sc2 = mp.sc2;
+    dp.bsc = mp.bsc;
     dp.r_bf16 = mp.r_bf16;
     dp.r2_bf16 = mp.r2_bf16;
     dp.out = part;

@@ -12,7 +12,8 @@
 // the main backward kernel (the logits never leave the chip):
 //   S^T  = K_j Q_i^T - lse_i sqrt(C) + (r1 + r2) mask_j      (tcgen05, TMEM)
 //   dP^T = V_j (dOa_hi + dOa_lo)_i^T - D_i                    (tcgen05, TMEM)
-//   P^T  = exp2(S^T log2(e)/sqrt(C) + bias^T log2(e)),   dS^T = P^T dP^T
+//   P^T  = exp2(S^T log2(e)/sqrt(C) + bias^T log2(e) r1/sqrt(C)),   dS^T = P^T dP^T
+//          (r1 = bf16(sqrt(C)): the bias with the forward's scale, see fwd_sm100.cuh)
 //   acc[j, i] += dS^T    (fp32 registers, rows s in order)
 // The row terms (-lse sqrt(C), -D as bf16 high/low pairs), the gated output
 // gradient split into two bf16 parts and the transposed pair bias are the
@@ -25,13 +26,13 @@
 // group; the finishing pass adds the slabs in group order.  The result is
 // therefore bitwise reproducible.
 //
-// Warp roles (384 threads):
-//   warps 0..7  two dS warpgroups (queries 0..63 / 64..127 of the tile);
-//               thread = key row j of the tile (TMEM lane), 64 sums each
-//   warp 8      TMA producer: per item the transposed bias tile (double
+// Warp roles (640 threads):
+//   warps 0..15 four dS warpgroups (queries 0..31, 32..63, 64..95, 96..127 of
+//               the tile); thread = key row j of the tile (TMEM lane), 32 sums each
+//   warp 16     TMA producer: per item the transposed bias tile (double
 //               buffered by item parity), per row s K, V, Q, dOa high/low,
 //               the mask and the two row terms into a 2-stage ring
-//   warp 9      MMA issuer of S^T; warp 10 MMA issuer of dP^T, both into a
+//   warp 17     MMA issuer of S^T; warp 18 MMA issuer of dP^T, both into a
 //               double-buffered TMEM pair (S^T, dP^T), so the MMAs of row
 //               s + 1 run while the dS warps work on row s
 #pragma once
@@ -67,10 +68,14 @@ constexpr int NBARS = 16;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-constexpr int THREADS = 384;
-constexpr int LAUNCH_REGS = 168;
-constexpr uint32_t DS_REGS = 208, CONTROL_REGS = 88;
-static_assert((2 * DS_REGS + CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
+// Four dS warpgroups, 32 queries each (more warps per SM hide the latency of the
+// per-row chain of TMEM loads, exponentials and sums), then the control warpgroup.
+constexpr int NWG = 4;
+constexpr int QW = BQ / NWG;                      // queries per dS warpgroup
+constexpr int THREADS = 128 * NWG + 128;
+constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
+constexpr uint32_t DS_REGS = 104, CONTROL_REGS = 56;
+static_assert((NWG * DS_REGS + CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
 // TMEM: buffer x holds S^T at 256 x and dP^T at 256 x + 128
 constexpr uint32_t TM_COLS = 512;
 // Every POLY_EVERY-th pair of exponentials runs on the FMA pipe (exp2_poly2)
@@ -116,6 +121,7 @@ struct Params {
     int gsz, groups;     // rows s per group, groups
     int n_items;         // B * H * n_t * n_t * groups
     float sc2;           // log2(e) / sqrt(C)
+    float bsc;           // log2(e) * r1 / sqrt(C): the pair bias enters as the forward's tensor core adds it
     float r_bf16, r2_bf16;
     float* out;          // [groups, B, H, N, N] partial slabs, or d_pair_bias when groups == 1
     uint64_t wait_ns;
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = 8, kMmaS = 9, kMmaD = 10;
+    constexpr int kDsWarps = 4 * NWG, kProducer = kDsWarps, kMmaS = kDsWarps + 1, kMmaD = kDsWarps + 2;
 
     const uint32_t bar0 = base + OFF_BAR;
     auto st_full = [&](int x) { return bar0 + 8u * (0 + x); };
@@ -174,10 +180,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(st_full(x), 1);
             mbar_init(st_empty(x), 2);      // one commit per MMA issuer
             mbar_init(bt_full(x), 1);
-            mbar_init(bt_empty(x), 8);      // one arrival per dS warp
+            mbar_init(bt_empty(x), kDsWarps);   // one arrival per dS warp
             mbar_init(s_full(x), 1);
             mbar_init(dp_full(x), 1);
-            mbar_init(sdp_free(x), 8);
+            mbar_init(sdp_free(x), kDsWarps);
             mbar_init(mma_done(x), 1);
         }
         *abort_flag = 0;
@@ -193,14 +199,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_alloc(base + OFF_MISC, TM_COLS);
         tmem_relinquish();
     }
-    if (warp < 8) {
+    if (warp < kDsWarps) {
         // Constant operands, and the zero rows of the per-stage blocks (the TMA
         // writes only rows 0..1 of the nl / -D blocks and rows 0, 8 of the mask
         // block).  No-swizzle K-major element (row, k) sits at
         // (row%8)*16 + (row/8)*256 + (k/8)*128 + (k%8)*2.
         const int t = threadIdx.x;
+        constexpr int nt = 32 * kDsWarps;
         auto zero = [&](int off, int bytes) {
-            for (int o = t * 16; o < bytes; o += 256 * 16)
+            for (int o = t * 16; o < bytes; o += nt * 16)
                 *reinterpret_cast<uint4*>(gbase + off + o) = make_uint4(0u, 0u, 0u, 0u);
         };
         zero(OFF_ONES, CONST_BYTES);
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             zero(OFF_ST + x * STB + ST_NL, RT_BYTES);
             zero(OFF_ST + x * STB + ST_ND, RT_BYTES);
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(nt) : "memory");
         if (t < 128) {
             const uint16_t one = 0x3F80u;
             const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
@@ -229,125 +236,128 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProducer) {
+    // setmaxnreg is warpgroup-wide: all four warps of a warpgroup execute the same
+    // instruction, so each warpgroup changes its count before its warps' roles split.
+    if (warp >= kDsWarps) {
         regs_decrease<CONTROL_REGS>();
-        // ---------------------------------------------------------------- producer
-        if (lane == 0) {
-            constexpr uint32_t tx = 5 * TILE_BYTES + 4 * 256 + (HAS_MASK ? 4 * 128 : 0);
-            int st_issued[2] = {0, 0}, bt_issued[2] = {0, 0};
-            int tg = 0;
-            bool ok = true;
-            for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
-                const Item x = decode(p, item);
-                const int i0 = x.it * BQ, j0 = x.jt * BK;
-                const int s0 = x.g * p.gsz, ns = min(p.gsz, p.S - s0);
-                if (HAS_BIAS) {
-                    const int bb = k & 1;
-                    if (k >= 2) ok = mbar_wait(bt_empty(bb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01, p.wait_ns);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(bt_full(bb), 2 * BT_BOX);
-                    const uint32_t bt = base + OFF_BT + bb * 2 * BT_BOX;
-                    tma_load_4d(bt, &tm_bt, bt_full(bb), i0, j0, x.h, x.b);
-                    tma_load_4d(bt + BT_BOX, &tm_bt, bt_full(bb), i0 + 64, j0, x.h, x.b);
-                    ++bt_issued[bb];
-                }
-                for (int si = 0; si < ns; ++si, ++tg) {
-                    const int s = s0 + si, st = tg & 1;
-                    const uint32_t sb = base + OFF_ST + st * STB;
-                    if (tg >= 2) ok = mbar_wait(st_empty(st), ((tg >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x02, p.wait_ns);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(st_full(st), tx);
-                    tma_load_5d(sb + ST_K, &tm_k, st_full(st), 0, j0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_V, &tm_v, st_full(st), 0, j0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_Q, &tm_q, st_full(st), 0, i0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_DOH, &tm_doa, st_full(st), 0, i0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_DOL, &tm_dol, st_full(st), 0, i0, x.h, s, x.b);
-                    if (HAS_MASK) {   // rows 0 and 8 of the two 64-key halves of the A block
-                        tma_load_3d(sb + ST_MASK, &tm_mask, st_full(st), j0, s, x.b);
-                        tma_load_3d(sb + ST_MASK + 1024, &tm_mask, st_full(st), j0, s, x.b);
-                        tma_load_3d(sb + ST_MASK + 2048, &tm_mask, st_full(st), j0 + 64, s, x.b);
-                        tma_load_3d(sb + ST_MASK + 3072, &tm_mask, st_full(st), j0 + 64, s, x.b);
+        if (warp == kProducer) {
+            // ---------------------------------------------------------------- producer
+            if (lane == 0) {
+                constexpr uint32_t tx = 5 * TILE_BYTES + 4 * 256 + (HAS_MASK ? 4 * 128 : 0);
+                int st_issued[2] = {0, 0}, bt_issued[2] = {0, 0};
+                int tg = 0;
+                bool ok = true;
+                for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
+                    const Item x = decode(p, item);
+                    const int i0 = x.it * BQ, j0 = x.jt * BK;
+                    const int s0 = x.g * p.gsz, ns = min(p.gsz, p.S - s0);
+                    if (HAS_BIAS) {
+                        const int bb = k & 1;
+                        if (k >= 2) ok = mbar_wait(bt_empty(bb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x01, p.wait_ns);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(bt_full(bb), 2 * BT_BOX);
+                        const uint32_t bt = base + OFF_BT + bb * 2 * BT_BOX;
+                        tma_load_4d(bt, &tm_bt, bt_full(bb), i0, j0, x.h, x.b);
+                        tma_load_4d(bt + BT_BOX, &tm_bt, bt_full(bb), i0 + 64, j0, x.h, x.b);
+                        ++bt_issued[bb];
                     }
-                    // rows 0..1 (high, low) of the two 64-query atoms of the nl and -D blocks
-                    tma_load_5d(sb + ST_NL, &tm_nl, st_full(st), i0, 0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_NL + 2048, &tm_nl, st_full(st), i0 + 64, 0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_ND, &tm_d, st_full(st), i0, 0, x.h, s, x.b);
-                    tma_load_5d(sb + ST_ND + 2048, &tm_d, st_full(st), i0 + 64, 0, x.h, s, x.b);
-                    ++st_issued[st];
+                    for (int si = 0; si < ns; ++si, ++tg) {
+                        const int s = s0 + si, st = tg & 1;
+                        const uint32_t sb = base + OFF_ST + st * STB;
+                        if (tg >= 2) ok = mbar_wait(st_empty(st), ((tg >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x02, p.wait_ns);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(st_full(st), tx);
+                        tma_load_5d(sb + ST_K, &tm_k, st_full(st), 0, j0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_V, &tm_v, st_full(st), 0, j0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_Q, &tm_q, st_full(st), 0, i0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_DOH, &tm_doa, st_full(st), 0, i0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_DOL, &tm_dol, st_full(st), 0, i0, x.h, s, x.b);
+                        if (HAS_MASK) {   // rows 0 and 8 of the two 64-key halves of the A block
+                            tma_load_3d(sb + ST_MASK, &tm_mask, st_full(st), j0, s, x.b);
+                            tma_load_3d(sb + ST_MASK + 1024, &tm_mask, st_full(st), j0, s, x.b);
+                            tma_load_3d(sb + ST_MASK + 2048, &tm_mask, st_full(st), j0 + 64, s, x.b);
+                            tma_load_3d(sb + ST_MASK + 3072, &tm_mask, st_full(st), j0 + 64, s, x.b);
+                        }
+                        // rows 0..1 (high, low) of the two 64-query atoms of the nl and -D blocks
+                        tma_load_5d(sb + ST_NL, &tm_nl, st_full(st), i0, 0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_NL + 2048, &tm_nl, st_full(st), i0 + 64, 0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_ND, &tm_d, st_full(st), i0, 0, x.h, s, x.b);
+                        tma_load_5d(sb + ST_ND + 2048, &tm_d, st_full(st), i0 + 64, 0, x.h, s, x.b);
+                        ++st_issued[st];
+                    }
+                }
+                // Never leave with copies in flight: wait (bounded) for the last fill of every buffer.
+                volatile int no_abort = 0;
+                for (int x = 0; x < 2; ++x) {
+                    if (st_issued[x]) mbar_wait(st_full(x), (st_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x03);
+                    if (bt_issued[x]) mbar_wait(bt_full(x), (bt_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
                 }
             }
-            // Never leave with copies in flight: wait (bounded) for the last fill of every buffer.
-            volatile int no_abort = 0;
-            for (int x = 0; x < 2; ++x) {
-                if (st_issued[x]) mbar_wait(st_full(x), (st_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x03);
-                if (bt_issued[x]) mbar_wait(bt_full(x), (bt_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x04);
+        } else if (warp == kMmaS || warp == kMmaD) {
+            // ---------------------------------------------------------------- MMA issuers
+            const int role = warp - kMmaS;   // 0: S^T, 1: dP^T
+            if (lane == 0) {
+                constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // K Q^T, V dOa^T
+                constexpr uint32_t ID_RT = idesc_bf16(BK, BQ, false, true);    // ones x row-term block
+                constexpr uint32_t ID_MK = idesc_bf16(BK, BQ, true, false);    // mask block x r-row
+                bool ok = true;
+                int tg = 0;
+                for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+                    const Item x = decode(p, item);
+                    const int ns = min(p.gsz, p.S - x.g * p.gsz);
+                    for (int si = 0; si < ns; ++si, ++tg) {
+                        const int st = tg & 1, buf = tg & 1;
+                        ok = mbar_wait(st_full(st), (tg >> 1) & 1, abort_flag, kTimeoutBase | (0x11 + role), p.wait_ns);
+                        if (ok && tg >= 2)
+                            ok = mbar_wait(sdp_free(buf), ((tg >> 1) - 1) & 1, abort_flag, kTimeoutBase | (0x13 + role), p.wait_ns);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t sb = base + OFF_ST + st * STB;
+                        const uint32_t d = tmem + 256u * (uint32_t)buf + (role == 0 ? 0u : 128u);
+                        if (role == 0) {
+                            // S^T = K Q^T - lse*sqrt(C) (+ (r1 + r2) * mask_j)
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                mma_ss(d, smem_desc(sb + ST_K + kk * 32, 16, 512, kSw64),
+                                       smem_desc(sb + ST_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+                            mma_ss(d, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                                   smem_desc(sb + ST_NL, 2048, 1024, kSw128), ID_RT, 1u);
+                            if (HAS_MASK)
+                                mma_ss(d, smem_desc(sb + ST_MASK, 2048, 1024, kSw128),
+                                       smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
+                            mma_commit(s_full(buf));
+                        } else {
+                            // dP^T = V (dOa_hi + dOa_lo)^T - D
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                mma_ss(d, smem_desc(sb + ST_V + kk * 32, 16, 512, kSw64),
+                                       smem_desc(sb + ST_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk)
+                                mma_ss(d, smem_desc(sb + ST_V + kk * 32, 16, 512, kSw64),
+                                       smem_desc(sb + ST_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
+                            mma_ss(d, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
+                                   smem_desc(sb + ST_ND, 2048, 1024, kSw128), ID_RT, 1u);
+                            mma_commit(dp_full(buf));
+                        }
+                        mma_commit(st_empty(st));    // this issuer no longer reads the stage
+                    }
+                }
+                // Drain: every MMA issued by this thread has finished before TMEM is released.
+                mma_commit(mma_done(role));
+                volatile int no_abort = 0;
+                mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x15 + role));
             }
         }
-    } else if (warp == kMmaS || warp == kMmaD) {
-        regs_decrease<CONTROL_REGS>();
-        // ---------------------------------------------------------------- MMA issuers
-        const int role = warp - kMmaS;   // 0: S^T, 1: dP^T
-        if (lane == 0) {
-            constexpr uint32_t ID_SS = idesc_bf16(BK, BQ, false, false);   // K Q^T, V dOa^T
-            constexpr uint32_t ID_RT = idesc_bf16(BK, BQ, false, true);    // ones x row-term block
-            constexpr uint32_t ID_MK = idesc_bf16(BK, BQ, true, false);    // mask block x r-row
-            bool ok = true;
-            int tg = 0;
-            for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-                const Item x = decode(p, item);
-                const int ns = min(p.gsz, p.S - x.g * p.gsz);
-                for (int si = 0; si < ns; ++si, ++tg) {
-                    const int st = tg & 1, buf = tg & 1;
-                    ok = mbar_wait(st_full(st), (tg >> 1) & 1, abort_flag, kTimeoutBase | (0x11 + role), p.wait_ns);
-                    if (ok && tg >= 2)
-                        ok = mbar_wait(sdp_free(buf), ((tg >> 1) - 1) & 1, abort_flag, kTimeoutBase | (0x13 + role), p.wait_ns);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t sb = base + OFF_ST + st * STB;
-                    const uint32_t d = tmem + 256u * (uint32_t)buf + (role == 0 ? 0u : 128u);
-                    if (role == 0) {
-                        // S^T = K Q^T - lse*sqrt(C) (+ (r1 + r2) * mask_j)
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk)
-                            mma_ss(d, smem_desc(sb + ST_K + kk * 32, 16, 512, kSw64),
-                                   smem_desc(sb + ST_Q + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-                        mma_ss(d, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
-                               smem_desc(sb + ST_NL, 2048, 1024, kSw128), ID_RT, 1u);
-                        if (HAS_MASK)
-                            mma_ss(d, smem_desc(sb + ST_MASK, 2048, 1024, kSw128),
-                                   smem_desc(base + OFF_RROW, 128, 256, kSwNone), ID_MK, 1u);
-                        mma_commit(s_full(buf));
-                    } else {
-                        // dP^T = V (dOa_hi + dOa_lo)^T - D
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk)
-                            mma_ss(d, smem_desc(sb + ST_V + kk * 32, 16, 512, kSw64),
-                                   smem_desc(sb + ST_DOH + kk * 32, 16, 512, kSw64), ID_SS, kk > 0);
-#pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk)
-                            mma_ss(d, smem_desc(sb + ST_V + kk * 32, 16, 512, kSw64),
-                                   smem_desc(sb + ST_DOL + kk * 32, 16, 512, kSw64), ID_SS, 1u);
-                        mma_ss(d, smem_desc(base + OFF_ONES, 128, 256, kSwNone),
-                               smem_desc(sb + ST_ND, 2048, 1024, kSw128), ID_RT, 1u);
-                        mma_commit(dp_full(buf));
-                    }
-                    mma_commit(st_empty(st));    // this issuer no longer reads the stage
-                }
-            }
-            // Drain: every MMA issued by this thread has finished before TMEM is released.
-            mma_commit(mma_done(role));
-            volatile int no_abort = 0;
-            mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x15 + role));
-        }
-    } else if (warp < 8) {
+    } else {
         regs_increase<DS_REGS>();
         // ---------------------------------------------------------------- dS warpgroups
-        const int wg = warp >> 2;                // 0: queries 0..63 of the tile, 1: 64..127
+        const int wg = warp >> 2;                // queries 32 wg .. 32 wg + 31 of the tile
         const int quad = warp & 3;
         const int r = quad * 32 + lane;          // key row within the tile = TMEM lane
-        const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(wg * 64);
+        const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(wg * QW);
         const uint64_t SC2 = f2(p.sc2, p.sc2);
-        const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
+        const uint64_t L2E2 = f2(p.bsc, p.bsc);
         bool ok = true;
         int tg = 0;
         for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
@@ -361,10 +371,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ok = mbar_wait(bt_full(bb), (k >> 1) & 1, abort_flag, kTimeoutBase | 0x21, p.wait_ns);
                 if (!ok) break;
             }
-            const uint8_t* bt_ptr = gbase + OFF_BT + bb * 2 * BT_BOX + wg * BT_BOX + r * 128;
-            uint64_t acc[32];
+            // this warpgroup's 32 queries: 64-query box wg / 2, 16-byte chunks 4 (wg % 2) .. + 3
+            const uint8_t* bt_ptr = gbase + OFF_BT + bb * 2 * BT_BOX + (wg >> 1) * BT_BOX + r * 128;
+            uint64_t acc[QW / 2];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc[c] = 0;
+            for (int c = 0; c < QW / 2; ++c) acc[c] = 0;
             for (int si = 0; si < ns; ++si, ++tg) {
                 const int buf = tg & 1;
                 ok = mbar_wait(s_full(buf), (tg >> 1) & 1, abort_flag, kTimeoutBase | 0x22, p.wait_ns);
@@ -372,29 +383,29 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t ts = lane_addr + 256u * (uint32_t)buf;
-                // 16 queries at a time: [0,16) S^T columns, [16,32) dP^T columns.  The load of
-                // the next quarter is issued before the current one is worked on.
-                uint32_t va[32], vb[32];
-                tmem_ld16x2_issue(ts, ts + 128, va);
-                tmem_ld_wait32(va);
+                // 16 queries at a time: cur[0,16) S^T columns, cur[16,32) dP^T columns
 #pragma unroll
-                for (int qd = 0; qd < 4; ++qd) {
-                    uint32_t* cur = (qd & 1) ? vb : va;
-                    uint32_t* nxt = (qd & 1) ? va : vb;
-                    if (qd < 3) tmem_ld16x2_issue(ts + (qd + 1) * 16, ts + 128 + (qd + 1) * 16, nxt);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t cur[32];
+                    tmem_ld16x2_sync(ts + 16 * hf, ts + 128 + 16 * hf, cur);
+                    if (hf == 1) {                       // both halves of this buffer in registers
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(sdp_free(buf));
+                    }
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {        // 8 queries (one 16-byte bias chunk) at a time
                         uint32_t bw[4] = {0u, 0u, 0u, 0u};
                         if (HAS_BIAS) {
-                            const int ch = qd * 2 + q;
+                            const int ch = (wg & 1) * 4 + hf * 2 + q;
                             const uint4 w = *reinterpret_cast<const uint4*>(
                                 bt_ptr + (((uint32_t)ch ^ (uint32_t)(r & 7)) << 4));
                             bw[0] = w.x; bw[1] = w.y; bw[2] = w.z; bw[3] = w.w;
                         }
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int c = q * 8 + 2 * e;          // column within the quarter
-                            const int pr = qd * 8 + q * 4 + e;    // column pair within the 64
+                            const int c = q * 8 + 2 * e;          // column within the half
+                            const int pr = hf * 8 + q * 4 + e;    // column pair within the 32
                             uint64_t y2 = fmul2(f2(__uint_as_float(cur[c]), __uint_as_float(cur[c + 1])), SC2);
                             if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[e]), L2E2, y2);
                             uint64_t p2;
@@ -407,34 +418,27 @@ __global__ void __launch_bounds__(THREADS, 1)
                             acc[pr] = fadd2(acc[pr], ds2);
                         }
                     }
-                    if (qd < 3) tmem_ld_wait32(nxt);
-                    if (qd == 2) {                       // every column of this buffer is in registers
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(sdp_free(buf));
-                    }
                 }
             }
             if (!ok) break;
             if (HAS_BIAS) {                      // the item's bias tile is no longer read
+                fence_proxy_async_smem();        // generic reads before the TMA's refill of the buffer
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bt_empty(bb));
             }
-            // d_pair_bias[b, h, i, j] for i = i0 + 64 wg + c: one column j per thread, so each
+            // d_pair_bias[b, h, i, j] for i = i0 + 32 wg + c: one column j per thread, so each
             // store of the warp covers 32 consecutive j (128 bytes).
             if (jvalid) {
                 float* dst = p.out + ((int64_t)x.g * p.B * p.H + (int64_t)x.b * p.H + x.h) * p.N * p.N +
-                             (int64_t)(i0 + wg * 64) * p.N + j;
-                const int ivalid = min(64, p.N - i0 - wg * 64);
+                             (int64_t)(i0 + wg * QW) * p.N + j;
+                const int ivalid = min(QW, p.N - i0 - wg * QW);
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
+                for (int c = 0; c < QW / 2; ++c) {
                     if (2 * c < ivalid) dst[(int64_t)(2 * c) * p.N] = f2lo(acc[c]);
                     if (2 * c + 1 < ivalid) dst[(int64_t)(2 * c + 1) * p.N] = f2hi(acc[c]);
                 }
             }
         }
-    } else {
-        regs_decrease<CONTROL_REGS>();
     }
 
     tc_fence_before();

@@ -132,7 +132,7 @@ evo_status_t launch_fwd_bf16(const CUtensorMap* maps, const evo::fwd::Params& p,
     const int grid = std::min(p.n_items, sm_count());
     {
         evo::timing::Scope t(EVO_PHASE_FWD_MAIN, stream);
-        kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+        kern<<<grid, L::threads, L::bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
     }
     g_launches += 1;
     return cudaGetLastError() == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
@@ -152,11 +152,12 @@ evo_status_t fwd_bf16(const evo_shape_t& sh, const void* q, const void* k, const
     const int64_t n_sg = (sh.S + kFwdNsub - 1) / kFwdNsub;
     const int64_t n_items = sh.B * sh.H * n_sg * n_it;
     if (n_items > (int64_t)1 << 30) return EVO_ERR_UNSUPPORTED;
-    CUtensorMap maps[5];
+    CUtensorMap maps[6];
     std::memset(maps, 0, sizeof(maps));
     if (!evo::tma::rows_bf16(&maps[0], q, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !evo::tma::rows_bf16(&maps[1], k, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B))
+        !evo::tma::rows_bf16(&maps[2], v, sh, in, evo::fwd::BN, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !evo::tma::rows_bf16(&maps[5], g, sh, in, evo::fwd::BM, CU_TENSOR_MAP_SWIZZLE_64B))
         return EVO_ERR_CUDA;
     if (bias && !evo::tma::square_bf16(&maps[3], bias, sh, evo::fwd::BM)) return EVO_ERR_CUDA;
     if (mask && !evo::tma::mask_bf16(&maps[4], mask, sh, 64)) return EVO_ERR_CUDA;

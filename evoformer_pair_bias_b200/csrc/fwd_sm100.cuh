@@ -12,11 +12,16 @@
 // accumulates, in fp32 TMEM, sqrt(C) times the logit without the pair bias:
 // the last term is one 16-deep K step whose B block carries the mask row of
 // row s in its rows 0 and 8 (exact products in fp32; r1 + r2 equals sqrt(C)
-// to 3e-7 relative, so the mask enters exactly up to that and fp32 rounding).  The pair-bias tile
-// (TMA-loaded once per key tile and shared by all NSUB rows s -- it is the
-// same for every s) is added by the softmax threads from shared memory, one
-// fused multiply-add per logit pair, while the other row group has its turn
-// on the exponentials (see below).
+// to 3e-7 relative, so the mask enters exactly up to that and fp32 rounding).
+// The pair-bias tile (TMA-loaded once per key tile and shared by all NSUB rows
+// s -- it is the same for every s) is added by the tensor core too, as
+// (r1 I) B with I the identity: eight more 16-deep K steps whose A blocks are
+// shifted 16 x 16 identities, all read from one small constant block (see
+// Layout::ident).  The bias therefore enters as (r1 / sqrt(C)) bias, scaled by
+// 1 - 1.07e-4 for C = 32 -- eighteen times below the 2^-9 rounding of the bf16
+// bias itself; the backward adds it with the same factor, so its recomputed P
+// matches this pass's log-sum-exp.  The softmax threads only scale, take
+// maxima and exponentiate.
 //
 // Warp roles (128*NSUB + 128 threads; the last warpgroup gives up registers
 // to the softmax warpgroups with setmaxnreg):
@@ -64,6 +69,15 @@ constexpr int BIAS_BOX = BM * 64 * 2;   // 16 KB: 128 rows x 64 keys, 128B swizz
 constexpr int BIAS_BYTES = 2 * BIAS_BOX;
 constexpr int MASKB_BYTES = 4096;       // 16 x 128 bf16 B block (rows 0 and 8 = mask row), 128B swizzle
 constexpr int ONES_BYTES = 128 * 16 * 2;     // r1 e_0 + r2 e_8 columns, K-major, no swizzle
+// The A operands of the bias MMAs, 128 x 16 blocks (r1 I)[:, 16 kk : 16 kk + 16], kk = 0..7,
+// all read from one array of 45 no-swizzle core matrices (8 x 8 bf16, 128 bytes each) that
+// is zero except r1 I_8 in cores IDENT_C0 and IDENT_C0 + 16.  K-step kk starts at core
+// IDENT_C0 - 2 kk with 8-row groups one core apart (SBO 128 B) and the second 8-wide K group
+// 15 cores further (LBO 1920 B): row group g, K group h reads core IDENT_C0 - 2 kk + g + 15 h,
+// which is an identity core exactly for (g, h) = (2 kk, 0) and (2 kk + 1, 1).
+constexpr int IDENT_C0 = 14;
+constexpr int IDENT_BYTES = 6144;            // 45 cores = 5760 bytes, rounded up
+constexpr uint32_t IDENT_SBO = 128, IDENT_LBO = 15 * 128;
 // per row group: S, P, and two O accumulators (items alternate between them,
 // so an item's epilogue can run after the next item's first tile)
 constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 192, SUBCOLS = 256;
@@ -81,9 +95,12 @@ __host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / 
 template <int NSUB>
 struct Layout {
     static constexpr int qbuf(int k, int u) { return (k * NSUB + u) * Q_BYTES; }   // per item parity k
-    static constexpr int ones = 2 * NSUB * Q_BYTES;
+    // the gate tile of each row s, read by the item's epilogue (same box and swizzle as Q)
+    static constexpr int gbuf(int k, int u) { return (2 * NSUB + k * NSUB + u) * Q_BYTES; }
+    static constexpr int ones = 4 * NSUB * Q_BYTES;
+    static constexpr int ident = ones + ONES_BYTES;
     // ring A: per stage K (per row), the pair-bias tile, the mask blocks (per row)
-    static constexpr int stage0 = round_up(ones + ONES_BYTES, 1024);
+    static constexpr int stage0 = round_up(ident + IDENT_BYTES, 1024);
     static constexpr int k_off(int u) { return u * KV_BYTES; }
     static constexpr int bias_off = NSUB * KV_BYTES;
     static constexpr int maskb_off(int u) { return bias_off + BIAS_BYTES + u * MASKB_BYTES; }
@@ -94,18 +111,19 @@ struct Layout {
     static constexpr int vstage_bytes = round_up(NSUB * KV_BYTES, 1024);
     static constexpr int bars = vstage0 + STAGES_B * vstage_bytes;
     // q_full[2], q_empty[2], ka_full[SA], ka_empty[SA], v_full[SB], v_empty[SB], s_full[u], s_free[u],
-    // p_full[u], o_full[u], mma_done[u], exp_turn[u]
-    static constexpr int nbars = 4 + 2 * STAGES_A + 2 * STAGES_B + 6 * NSUB;
+    // p_full[u], o_full[u], mma_done[2 NSUB], exp_turn[u], g_full[2], g_empty[2]
+    static constexpr int nbars = 4 + 2 * STAGES_A + 2 * STAGES_B + 7 * NSUB + 4;
     static constexpr int misc = bars + nbars * 8;   // tmem base (u32), abort flag (u32)
     static constexpr int bytes = misc + 16 + 1024;  // + slack to align the base to 1024
     static constexpr uint32_t tmem_cols = NSUB == 1 ? 256 : 512;
-    static constexpr int threads = 128 * NSUB + 128;
+    // softmax warpgroups, then two control warpgroups (producers, S issuers, P V issuers)
+    static constexpr int threads = 128 * NSUB + 256;
     // register split: launch count (65536 / threads, rounded down to 8) and the
     // per-warpgroup counts after setmaxnreg; softmax + control <= launch pool
     static constexpr int launch_regs = (65536 / threads) / 8 * 8;
     static constexpr uint32_t softmax_regs = NSUB == 2 ? 208 : 240;
-    static constexpr uint32_t control_regs = 88;
-    static_assert((int)(NSUB * softmax_regs + control_regs) * 128 <= launch_regs * threads, "register split");
+    static constexpr uint32_t control_regs = NSUB == 2 ? 48 : 64;
+    static_assert((int)(NSUB * softmax_regs + 2 * control_regs) * 128 <= launch_regs * threads, "register split");
 };
 
 struct Params {
@@ -150,7 +168,8 @@ template <int NSUB, bool HAS_MASK, bool HAS_BIAS>
 __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_bias,
-                    const __grid_constant__ CUtensorMap tm_mask, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_mask, const __grid_constant__ CUtensorMap tm_g,
+                    const Params p) {
     using L = Layout<NSUB>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -158,9 +177,10 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = 4 * NSUB, kMma = 4 * NSUB + 1;   // MMA issuers: warps kMma .. kMma+NSUB-1
-    constexpr int kProducerV = kMma + NSUB;
-    static_assert(kProducerV < L::threads / 32, "warp roles");
+    // S issuers: warps kMma .. kMma+NSUB-1; P V issuers: warps kMmaPV .. kMmaPV+NSUB-1
+    constexpr int kProducer = 4 * NSUB, kMma = 4 * NSUB + 1;
+    constexpr int kProducerV = kMma + NSUB, kMmaPV = kProducerV + 1;
+    static_assert(kMmaPV + NSUB <= L::threads / 32, "warp roles");
 
     const uint32_t bar0 = base + L::bars;
     constexpr int kS = 4 + 2 * STAGES_A + 2 * STAGES_B;        // first per-row-group barrier
@@ -174,9 +194,12 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     auto s_free = [&](int u) { return bar0 + 8u * (kS + NSUB + u); };
     auto p_full = [&](int u) { return bar0 + 8u * (kS + 2 * NSUB + u); };
     auto o_full = [&](int u) { return bar0 + 8u * (kS + 3 * NSUB + u); };
-    auto mma_done = [&](int u) { return bar0 + 8u * (kS + 4 * NSUB + u); };
+    auto mma_done = [&](int x) { return bar0 + 8u * (kS + 4 * NSUB + x); };      // x < 2 * NSUB
     // exp_turn[u]: row group u may start the exponentials of its next tile
-    auto exp_turn = [&](int u) { return bar0 + 8u * (kS + 5 * NSUB + u); };
+    auto exp_turn = [&](int u) { return bar0 + 8u * (kS + 6 * NSUB + u); };
+    // g_full[x] / g_empty[x]: the gate tiles of the item with parity x loaded / read by its epilogue
+    auto g_full = [&](int x) { return bar0 + 8u * (kS + 7 * NSUB + x); };
+    auto g_empty = [&](int x) { return bar0 + 8u * (kS + 7 * NSUB + 2 + x); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::misc + 4);
 
@@ -184,10 +207,12 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(q_full(x), 1);
             mbar_init(q_empty(x), NSUB);           // one commit per MMA issuer
+            mbar_init(g_full(x), 1);
+            mbar_init(g_empty(x), 4 * NSUB);       // one arrival per softmax warp, after its epilogue
         }
         for (int st = 0; st < STAGES_A; ++st) {
             mbar_init(ka_full(st), 1);
-            mbar_init(ka_empty(st), NSUB + 4 * NSUB);   // the S MMAs' commits + every softmax warp's bias reads
+            mbar_init(ka_empty(st), NSUB);              // the S MMAs' commits (K, mask and bias are MMA operands)
         }
         for (int st = 0; st < STAGES_B; ++st) {
             mbar_init(v_full(st), 1);
@@ -199,6 +224,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             mbar_init(p_full(u), 4);
             mbar_init(o_full(u), 1);
             mbar_init(mma_done(u), 1);
+            mbar_init(mma_done(NSUB + u), 1);
             mbar_init(exp_turn(u), 4);             // one arrival per warp of the other group
         }
         *abort_flag = 0;
@@ -208,6 +234,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_g);
         if (HAS_BIAS) prefetch_tmap(&tm_bias);
         if (HAS_MASK) prefetch_tmap(&tm_mask);
     }
@@ -224,7 +251,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         const int nt = 128 * NSUB;
         const uint16_t rb = (uint16_t)(__float_as_uint(p.r_bf16) >> 16);
         const uint16_t rb2 = (uint16_t)(__float_as_uint(p.r2_bf16) >> 16);
-        for (int o = t * 16; o < ONES_BYTES; o += nt * 16)
+        for (int o = t * 16; o < ONES_BYTES + IDENT_BYTES; o += nt * 16)   // ones and ident are adjacent
             *reinterpret_cast<uint4*>(gbase + L::ones + o) = make_uint4(0u, 0u, 0u, 0u);
         for (int st = 0; st < STAGES_A; ++st)
             for (int u = 0; u < NSUB; ++u)
@@ -238,6 +265,10 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             *reinterpret_cast<uint16_t*>(gbase + L::ones + (rr % 8) * 16 + (rr / 8) * 256) = rb;
             *reinterpret_cast<uint16_t*>(gbase + L::ones + (rr % 8) * 16 + (rr / 8) * 256 + 128) = rb2;
         }
+        if (t < 16) {   // the diagonals of the two identity cores: element (m, m) at 18 m bytes
+            const int core = IDENT_C0 + (t >> 3) * 16, m = t & 7;
+            *reinterpret_cast<uint16_t*>(gbase + L::ident + core * 128 + 18 * m) = rb;
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
@@ -245,169 +276,189 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProducer) {
+    // setmaxnreg is warpgroup-wide: all four warps of a warpgroup execute the same
+    // instruction, so each warpgroup changes its count before its warps' roles split.
+    if (warp >= 4 * NSUB) {
         regs_decrease<L::control_regs>();
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            constexpr uint32_t tx = NSUB * KV_BYTES + (HAS_BIAS ? BIAS_BYTES : 0) + (HAS_MASK ? NSUB * 512 : 0);
-            int q_issued[2] = {0, 0}, kv_issued[STAGES_A] = {};
-            int tg = 0;
-            bool ok = true;
-            for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
-                const Item itm = decode(p, item);
-                const int s0 = itm.sg * NSUB;
-                int s_ld[NSUB];
+        if (warp == kProducer) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0) {
+                constexpr uint32_t tx = NSUB * KV_BYTES + (HAS_BIAS ? BIAS_BYTES : 0) + (HAS_MASK ? NSUB * 512 : 0);
+                int q_issued[2] = {0, 0}, g_issued[2] = {0, 0}, kv_issued[STAGES_A] = {};
+                int tg = 0;
+                bool ok = true;
+                for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
+                    const Item itm = decode(p, item);
+                    const int s0 = itm.sg * NSUB;
+                    int s_ld[NSUB];
 #pragma unroll
-                for (int u = 0; u < NSUB; ++u) s_ld[u] = min(s0 + u, p.S - 1);
-                const int qb = k & 1;
-                if (k >= 2) ok = mbar_wait(q_empty(qb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x001, p.wait_ns);
-                if (!ok) break;
-                mbar_arrive_expect_tx(q_full(qb), NSUB * Q_BYTES);
-#pragma unroll
-                for (int u = 0; u < NSUB; ++u)
-                    tma_load_5d(base + L::qbuf(qb, u), &tm_q, q_full(qb), 0, itm.i0, itm.h, s_ld[u], itm.b);
-                ++q_issued[qb];
-                for (int j = 0; j < p.n_kv; ++j, ++tg) {
-                    const int st = tg % STAGES_A;
-                    const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
-                    if (tg >= STAGES_A)
-                        ok = mbar_wait(ka_empty(st), ((tg / STAGES_A) - 1) & 1, abort_flag, kTimeoutBase | 0x002, p.wait_ns);
+                    for (int u = 0; u < NSUB; ++u) s_ld[u] = min(s0 + u, p.S - 1);
+                    const int qb = k & 1;
+                    if (k >= 2) ok = mbar_wait(q_empty(qb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x001, p.wait_ns);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(ka_full(st), tx);
+                    mbar_arrive_expect_tx(q_full(qb), NSUB * Q_BYTES);
 #pragma unroll
                     for (int u = 0; u < NSUB; ++u)
-                        tma_load_5d(sb + L::k_off(u), &tm_k, ka_full(st), 0, j * BN, itm.h, s_ld[u], itm.b);
-                    if (HAS_BIAS) {
-                        tma_load_4d(sb + L::bias_off, &tm_bias, ka_full(st), j * BN, itm.i0, itm.h, itm.b);
-                        tma_load_4d(sb + L::bias_off + BIAS_BOX, &tm_bias, ka_full(st), j * BN + 64, itm.i0, itm.h, itm.b);
-                    }
-                    if (HAS_MASK) {
+                        tma_load_5d(base + L::qbuf(qb, u), &tm_q, q_full(qb), 0, itm.i0, itm.h, s_ld[u], itm.b);
+                    ++q_issued[qb];
+                    // the gate tiles of this item (buffer qb is free once item k-2's epilogue has read it)
+                    if (k >= 2) ok = mbar_wait(g_empty(qb), ((k >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x008, p.wait_ns);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(g_full(qb), NSUB * Q_BYTES);
 #pragma unroll
-                        for (int u = 0; u < NSUB; ++u) {
-                            // rows 0 and 8 of the two 64-key halves (rows 0 and 8 both start a
-                            // 128B-swizzle atom, so the unswizzled row lands as the MMA reads it)
-                            tma_load_3d(sb + L::maskb_off(u), &tm_mask, ka_full(st), j * BN, s_ld[u], itm.b);
-                            tma_load_3d(sb + L::maskb_off(u) + 1024, &tm_mask, ka_full(st), j * BN, s_ld[u], itm.b);
-                            tma_load_3d(sb + L::maskb_off(u) + 2048, &tm_mask, ka_full(st), j * BN + 64, s_ld[u], itm.b);
-                            tma_load_3d(sb + L::maskb_off(u) + 3072, &tm_mask, ka_full(st), j * BN + 64, s_ld[u], itm.b);
+                    for (int u = 0; u < NSUB; ++u)
+                        tma_load_5d(base + L::gbuf(qb, u), &tm_g, g_full(qb), 0, itm.i0, itm.h, s_ld[u], itm.b);
+                    ++g_issued[qb];
+                    for (int j = 0; j < p.n_kv; ++j, ++tg) {
+                        const int st = tg % STAGES_A;
+                        const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
+                        if (tg >= STAGES_A)
+                            ok = mbar_wait(ka_empty(st), ((tg / STAGES_A) - 1) & 1, abort_flag, kTimeoutBase | 0x002, p.wait_ns);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(ka_full(st), tx);
+#pragma unroll
+                        for (int u = 0; u < NSUB; ++u)
+                            tma_load_5d(sb + L::k_off(u), &tm_k, ka_full(st), 0, j * BN, itm.h, s_ld[u], itm.b);
+                        if (HAS_BIAS) {
+                            tma_load_4d(sb + L::bias_off, &tm_bias, ka_full(st), j * BN, itm.i0, itm.h, itm.b);
+                            tma_load_4d(sb + L::bias_off + BIAS_BOX, &tm_bias, ka_full(st), j * BN + 64, itm.i0, itm.h, itm.b);
                         }
-                    }
-                    ++kv_issued[st];
-                }
-            }
-            // Never leave with copies in flight: wait (bounded) for the last fill of every buffer.
-            volatile int no_abort = 0;
-            for (int x = 0; x < 2; ++x)
-                if (q_issued[x]) mbar_wait(q_full(x), (q_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x003);
-            for (int st = 0; st < STAGES_A; ++st)
-                if (kv_issued[st]) mbar_wait(ka_full(st), (kv_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x004);
-        }
-    } else if (warp == kProducerV) {
-        regs_decrease<L::control_regs>();
-        // ------------------------------------------------------------ producer of V
-        if (lane == 0) {
-            int v_issued[STAGES_B] = {};
-            int tg = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-                const Item itm = decode(p, item);
-                const int s0 = itm.sg * NSUB;
-                for (int j = 0; j < p.n_kv; ++j, ++tg) {
-                    const int st = tg % STAGES_B;
-                    const uint32_t vb = base + L::vstage0 + st * L::vstage_bytes;
-                    if (tg >= STAGES_B)
-                        ok = mbar_wait(v_empty(st), ((tg / STAGES_B) - 1) & 1, abort_flag, kTimeoutBase | 0x006, p.wait_ns);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(v_full(st), NSUB * KV_BYTES);
+                        if (HAS_MASK) {
 #pragma unroll
-                    for (int u = 0; u < NSUB; ++u)
-                        tma_load_5d(vb + L::v_off(u), &tm_v, v_full(st), 0, j * BN, itm.h, min(s0 + u, p.S - 1), itm.b);
-                    ++v_issued[st];
-                }
-            }
-            volatile int no_abort = 0;
-            for (int st = 0; st < STAGES_B; ++st)
-                if (v_issued[st]) mbar_wait(v_full(st), (v_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x007);
-        }
-    } else if (warp >= kMma && warp < kMma + NSUB) {
-        regs_decrease<L::control_regs>();
-        // ------------------------------------------------------------ MMA issuer of row group u
-        const int u = warp - kMma;
-        if (lane == 0) {
-            constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
-            constexpr uint32_t IDESC_MASK = idesc_bf16(BM, BN, false, true);   // B operand MN-major
-            constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, false, true);
-            const uint32_t t_s = tmem + u * SUBCOLS + COL_S, t_p = tmem + u * SUBCOLS + COL_P,
-                           t_o = tmem + u * SUBCOLS + COL_O;
-            bool ok = true;
-            int tg = 0;
-            int prev_j = 0, prev_k = 0;   // the tile (tg - 1) whose PV is still to be issued
-            bool pending = false;
-            auto issue_pv = [&]() -> bool {   // PV of tile tg-1
-                const int vs = (tg - 1) % STAGES_B;
-                const uint32_t vb = base + L::vstage0 + vs * L::vstage_bytes;
-                if (!mbar_wait(p_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x104, p.wait_ns)) return false;
-                if (!mbar_wait(v_full(vs), ((tg - 1) / STAGES_B) & 1, abort_flag, kTimeoutBase | 0x106, p.wait_ns))
-                    return false;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = smem_desc(vb + L::v_off(u) + kk * 1024, KV_BYTES, 512, kSw64);
-                    mma_ts(t_o + (uint32_t)(prev_k & 1) * HD, t_p + kk * 8, bd, IDESC_PV, (prev_j > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(o_full(u));
-                mma_commit(v_empty(vs));
-                return true;
-            };
-            for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
-                const int qb = k & 1;
-                ok = mbar_wait(q_full(qb), (k >> 1) & 1, abort_flag, kTimeoutBase | 0x101, p.wait_ns);
-                for (int j = 0; ok && j < p.n_kv; ++j) {
-                    const int st = tg % STAGES_A;
-                    const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
-                    ok = mbar_wait(ka_full(st), (tg / STAGES_A) & 1, abort_flag, kTimeoutBase | 0x102, p.wait_ns);
-                    if (ok && tg > 0) ok = mbar_wait(s_free(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x103, p.wait_ns);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        const uint64_t ad = smem_desc(base + L::qbuf(qb, u) + kk * 32, 16, 512, kSw64);
-                        const uint64_t bd = smem_desc(sb + L::k_off(u) + kk * 32, 16, 512, kSw64);
-                        mma_ss(t_s, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+                            for (int u = 0; u < NSUB; ++u) {
+                                // rows 0 and 8 of the two 64-key halves (rows 0 and 8 both start a
+                                // 128B-swizzle atom, so the unswizzled row lands as the MMA reads it)
+                                tma_load_3d(sb + L::maskb_off(u), &tm_mask, ka_full(st), j * BN, s_ld[u], itm.b);
+                                tma_load_3d(sb + L::maskb_off(u) + 1024, &tm_mask, ka_full(st), j * BN, s_ld[u], itm.b);
+                                tma_load_3d(sb + L::maskb_off(u) + 2048, &tm_mask, ka_full(st), j * BN + 64, s_ld[u], itm.b);
+                                tma_load_3d(sb + L::maskb_off(u) + 3072, &tm_mask, ka_full(st), j * BN + 64, s_ld[u], itm.b);
+                            }
+                        }
+                        ++kv_issued[st];
                     }
-                    if (HAS_MASK) {                               // + (r1 + r2) * mask[s, j]
-                        const uint64_t ad = smem_desc(base + L::ones, 128, 256, kSwNone);
-                        const uint64_t bd = smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128);
-                        mma_ss(t_s, ad, bd, IDESC_MASK, 1u);
-                    }
-                    mma_commit(s_full(u));
-                    mma_commit(ka_empty(st));                     // K and the mask blocks read
-                    if (pending) ok = issue_pv();
-                    prev_j = j;
-                    prev_k = k;
-                    pending = true;
-                    ++tg;
                 }
-                if (ok) mma_commit(q_empty(qb));   // Q of this item no longer read once these MMAs finish
+                // Never leave with copies in flight: wait (bounded) for the last fill of every buffer.
+                volatile int no_abort = 0;
+                for (int x = 0; x < 2; ++x) {
+                    if (q_issued[x]) mbar_wait(q_full(x), (q_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x003);
+                    if (g_issued[x]) mbar_wait(g_full(x), (g_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x009);
+                }
+                for (int st = 0; st < STAGES_A; ++st)
+                    if (kv_issued[st]) mbar_wait(ka_full(st), (kv_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x004);
             }
-            if (ok && pending) ok = issue_pv();
-            // Drain: every MMA issued by this thread has finished before TMEM is released.
-            mma_commit(mma_done(u));
-            volatile int no_abort = 0;
-            mbar_wait(mma_done(u), 0, &no_abort, kTimeoutBase | 0x105);
+        } else if (warp == kProducerV) {
+            // ------------------------------------------------------------ producer of V
+            if (lane == 0) {
+                int v_issued[STAGES_B] = {};
+                int tg = 0;
+                bool ok = true;
+                for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+                    const Item itm = decode(p, item);
+                    const int s0 = itm.sg * NSUB;
+                    for (int j = 0; j < p.n_kv; ++j, ++tg) {
+                        const int st = tg % STAGES_B;
+                        const uint32_t vb = base + L::vstage0 + st * L::vstage_bytes;
+                        if (tg >= STAGES_B)
+                            ok = mbar_wait(v_empty(st), ((tg / STAGES_B) - 1) & 1, abort_flag, kTimeoutBase | 0x006, p.wait_ns);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(v_full(st), NSUB * KV_BYTES);
+#pragma unroll
+                        for (int u = 0; u < NSUB; ++u)
+                            tma_load_5d(vb + L::v_off(u), &tm_v, v_full(st), 0, j * BN, itm.h, min(s0 + u, p.S - 1), itm.b);
+                        ++v_issued[st];
+                    }
+                }
+                volatile int no_abort = 0;
+                for (int st = 0; st < STAGES_B; ++st)
+                    if (v_issued[st]) mbar_wait(v_full(st), (v_issued[st] - 1) & 1, &no_abort, kTimeoutBase | 0x007);
+            }
+        } else if (warp >= kMma && warp < kMma + NSUB) {
+            // ------------------------------------------------------------ S issuer of row group u
+            const int u = warp - kMma;
+            if (lane == 0) {
+                constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
+                constexpr uint32_t IDESC_MASK = idesc_bf16(BM, BN, false, true);   // B operand MN-major
+                const uint32_t t_s = tmem + u * SUBCOLS + COL_S;
+                // descriptors that depend only on the stage are built once; per MMA only the
+                // start-address field (address / 16, in the low bits) moves
+                const uint64_t d_ones = smem_desc(base + L::ones, 128, 256, kSwNone);
+                const uint64_t d_id0 = smem_desc(base + L::ident + IDENT_C0 * 128, IDENT_LBO, IDENT_SBO, kSwNone);
+                bool ok = true;
+                int tg = 0;
+                for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
+                    const int qb = k & 1;
+                    ok = mbar_wait(q_full(qb), (k >> 1) & 1, abort_flag, kTimeoutBase | 0x101, p.wait_ns);
+                    const uint64_t d_q = smem_desc(base + L::qbuf(qb, u), 16, 512, kSw64);
+                    for (int j = 0; ok && j < p.n_kv; ++j, ++tg) {
+                        const int st = tg % STAGES_A;
+                        const uint32_t sb = base + L::stage0 + st * L::stage_bytes;
+                        ok = mbar_wait(ka_full(st), (tg / STAGES_A) & 1, abort_flag, kTimeoutBase | 0x102, p.wait_ns);
+                        if (ok && tg > 0) ok = mbar_wait(s_free(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x103, p.wait_ns);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t d_k = smem_desc(sb + L::k_off(u), 16, 512, kSw64);
+#pragma unroll
+                        for (int kk = 0; kk < HD / 16; ++kk)               // 32 bytes = 2 in the address field
+                            mma_ss(t_s, d_q + 2 * kk, d_k + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
+                        if (HAS_MASK)                                     // + (r1 + r2) * mask[s, j]
+                            mma_ss(t_s, d_ones, smem_desc(sb + L::maskb_off(u), 2048, 1024, kSw128), IDESC_MASK, 1u);
+                        if (HAS_BIAS) {                                   // + r1 * bias[i, j]: (r1 I) times the bias tile
+                            const uint64_t d_b = smem_desc(sb + L::bias_off, BIAS_BOX, 1024, kSw128);
+#pragma unroll
+                            for (int kk = 0; kk < BM / 16; ++kk)          // A: 2 cores (256 B) back, B: 2048 B on
+                                mma_ss(t_s, d_id0 - (uint64_t)(16 * kk), d_b + (uint64_t)(128 * kk), IDESC_MASK, 1u);
+                        }
+                        mma_commit(s_full(u));
+                        mma_commit(ka_empty(st));                         // K, mask and bias read
+                    }
+                    if (ok) mma_commit(q_empty(qb));   // Q of this item no longer read once these MMAs finish
+                }
+                // Drain: every MMA issued by this thread has finished before TMEM is released.
+                mma_commit(mma_done(u));
+                volatile int no_abort = 0;
+                mbar_wait(mma_done(u), 0, &no_abort, kTimeoutBase | 0x105);
+            }
+        } else if (warp >= kMmaPV && warp < kMmaPV + NSUB) {
+            // ------------------------------------------------------------ P V issuer of row group u
+            const int u = warp - kMmaPV;
+            if (lane == 0) {
+                constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, false, true);
+                const uint32_t t_p = tmem + u * SUBCOLS + COL_P, t_o = tmem + u * SUBCOLS + COL_O;
+                bool ok = true;
+                int tg = 0;
+                for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
+                    for (int j = 0; ok && j < p.n_kv; ++j, ++tg) {
+                        const int vs = tg % STAGES_B;
+                        ok = mbar_wait(p_full(u), tg & 1, abort_flag, kTimeoutBase | 0x104, p.wait_ns);
+                        if (ok) ok = mbar_wait(v_full(vs), (tg / STAGES_B) & 1, abort_flag, kTimeoutBase | 0x106, p.wait_ns);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t d_v = smem_desc(base + L::vstage0 + vs * L::vstage_bytes + L::v_off(u), KV_BYTES, 512,
+                                                       kSw64);
+                        const uint32_t o = t_o + (uint32_t)(k & 1) * HD;
+#pragma unroll
+                        for (int kk = 0; kk < BN / 16; ++kk)               // 16 keys = 1024 B = 64 in the address field
+                            mma_ts(o, t_p + kk * 8, d_v + (uint64_t)(64 * kk), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(o_full(u));
+                        mma_commit(v_empty(vs));
+                    }
+                }
+                mma_commit(mma_done(NSUB + u));
+                volatile int no_abort = 0;
+                mbar_wait(mma_done(NSUB + u), 0, &no_abort, kTimeoutBase | 0x107);
+            }
         }
-    } else if (warp < 4 * NSUB) {
+    } else {
         regs_increase<L::softmax_regs>();
         // ------------------------------------------------------------ softmax
         const int u = warp >> 2;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;          // query row within the tile = TMEM lane
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + u * SUBCOLS;
-        // S holds sqrt(C) * (q.k / sqrt(C) + mask); the logit in log2 units is
-        // y = S * sc2 + bias * log2(e), sc2 = log2(e)/sqrt(C); exponents are exp2(y - ms)
+        // S holds sqrt(C) times the logit; the logit in log2 units is y = S * sc2,
+        // sc2 = log2(e)/sqrt(C); exponents are exp2(y - ms)
         const float sc2 = p.scale * EVO_LOG2E;
         const uint64_t SC2 = f2(sc2, sc2);
-        const uint64_t L2E2 = f2(EVO_LOG2E, EVO_LOG2E);
         bool ok = true;
         int tg = 0;
         // The epilogue of an item (out = sigmoid(g) * O / l, lse) is deferred to
@@ -415,18 +466,23 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
         // complete (that tile waited for it), so no thread idles on it.
         struct Epi {
             bool pending, row_ok;
-            int b, s, i, h, obuf;
+            int b, s, i, h, obuf, k;
             float l, ms;
         } epi;
         epi.pending = false;
-        auto run_epilogue = [&]() {
-            // the gate row (prefetched into L2 during the item's last tile)
+        auto run_epilogue = [&]() -> bool {
+            // the gate row from the item's gate tile in shared memory (64B swizzle: 16-byte
+            // chunk c of row r sits at chunk c ^ ((r >> 1) & 3))
+            const int gb = epi.k & 1;
+            if (!mbar_wait(g_full(gb), (epi.k >> 1) & 1, abort_flag, kTimeoutBase | 0x207, p.wait_ns)) return false;
             uint4 gw[HD / 8];
-            if (epi.row_ok) {
-                const uint4* gp = reinterpret_cast<const uint4*>(p.g + p.in.off(epi.b, epi.s, epi.i, epi.h));
+            const uint8_t* grow = gbase + L::gbuf(gb, u) + r * 64;
 #pragma unroll
-                for (int q = 0; q < HD / 8; ++q) gw[q] = __ldg(gp + q);
-            }
+            for (int q = 0; q < HD / 8; ++q)
+                gw[q] = *reinterpret_cast<const uint4*>(grow + ((((uint32_t)q ^ (uint32_t)((r >> 1) & 3))) << 4));
+            fence_proxy_async_smem();            // generic reads before the TMA's refill of the buffer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(g_empty(gb));
             uint32_t o[HD];
             tmem_ld32_sync(lane_addr + COL_O + (uint32_t)epi.obuf * HD, o);
             if (epi.row_ok) {
@@ -459,6 +515,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     (epi.ms + __log2f(epi.l)) * EVO_LN2;
             }
             epi.pending = false;
+            return true;
         };
         for (int item = blockIdx.x, k = 0; ok && item < p.n_items; item += gridDim.x, ++k) {
             const Item itm = decode(p, item);
@@ -470,10 +527,6 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
             // l: running sum of exp2(S * sc2 - ms)
             float ms = -INFINITY, l = 0.f;
             for (int j = 0; j < p.n_kv; ++j, ++tg) {
-                if (j == p.n_kv - 1 && row_ok) {
-                    // the gate row is only needed by the item's epilogue: start bringing it into L2
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(p.g + p.in.off(itm.b, s, i, itm.h)));
-                }
                 ok = mbar_wait(s_full(u), tg & 1, abort_flag, kTimeoutBase | 0x201, p.wait_ns);
                 if (!ok) break;
                 tc_fence_after();
@@ -483,38 +536,8 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_free(u));
 
-                // y = S * sc2 + bias * log2(e): the pair-bias row of this query from
-                // the stage's tile (two 64-key boxes, 128B swizzle: 16-byte chunk c
-                // of row r sits at chunk c ^ (r & 7)), two logits per instruction
-                const int st = tg % STAGES_A;
-                if (HAS_BIAS) {
-                    // acquire the TMA writes of this stage (already complete: S used them)
-                    ok = mbar_wait(ka_full(st), (tg / STAGES_A) & 1, abort_flag, kTimeoutBase | 0x206, p.wait_ns);
-                    if (!ok) break;
-                }
-                {
-                    const uint8_t* brow = gbase + L::stage0 + st * L::stage_bytes + L::bias_off + r * 128;
-#pragma unroll
-                    for (int q = 0; q < BN / 8; ++q) {
-                        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                        if (HAS_BIAS)
-                            w = *reinterpret_cast<const uint4*>(brow + (q >> 3) * BIAS_BOX +
-                                                                ((((uint32_t)q & 7u) ^ (uint32_t)(r & 7)) << 4));
-                        const uint32_t bw[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = q * 8 + 2 * e;
-                            uint64_t y2 = fmul2(f2(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), SC2);
-                            if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[e]), L2E2, y2);
-                            xr[c] = __float_as_uint(f2lo(y2));
-                            xr[c + 1] = __float_as_uint(f2hi(y2));
-                        }
-                    }
-                }
-                // this warp no longer reads the stage's bias tile: with both S MMAs done,
-                // the stage can take the tile after next
-                __syncwarp();
-                if (lane == 0) mbar_arrive(ka_empty(st));
+                // S already holds sqrt(C) times the whole logit (q.k, mask and bias); the
+                // logit in log2 units is y = S * sc2, taken inside the exponent's FMA below
                 const int valid = p.N - j * BN;      // keys beyond N are padding: exclude them
                 if (valid < BN) {
 #pragma unroll
@@ -529,7 +552,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                         : "f"(mx[(c >> 1) & 3]), "f"(__uint_as_float(xr[c])), "f"(__uint_as_float(xr[c + 1])));
                     mx[(c >> 1) & 3] = m3;
                 }
-                const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sc2;   // sc2 > 0
 
                 // lazy rescale: move the running max only when this tile's max exceeds it by > 2^8
                 const float mcand = mloc;
@@ -567,7 +590,7 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     for (int cc = 0; cc < BN / 4; ++cc) {
                         const int c = half * (BN / 4) + cc;
                         const uint64_t y2 =
-                            fadd2(f2(__uint_as_float(xr[2 * c]), __uint_as_float(xr[2 * c + 1])), NEG_MS2);
+                            ffma2(f2(__uint_as_float(xr[2 * c]), __uint_as_float(xr[2 * c + 1])), SC2, NEG_MS2);
                         uint64_t pp;
                         if (POLY_EVERY > 0 && c % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1)
                             pp = exp2_poly2(y2);
@@ -592,25 +615,24 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                 if (lane == 0) mbar_arrive(p_full(u));
                 // the previous item's epilogue: its last PV finished before this
                 // tile's P was written (the o_full wait above)
-                if (j == 0 && epi.pending) run_epilogue();
+                if (j == 0 && epi.pending && !run_epilogue()) {
+                    ok = false;
+                    break;
+                }
             }
             if (!ok) break;
             epi.pending = true;
             epi.row_ok = row_ok;
-            epi.b = itm.b; epi.s = s; epi.i = i; epi.h = itm.h; epi.obuf = k & 1;
+            epi.b = itm.b; epi.s = s; epi.i = i; epi.h = itm.h; epi.obuf = k & 1; epi.k = k;
             epi.l = l; epi.ms = ms;
         }
         if (ok && epi.pending) {   // the last item: wait for its last PV
             ok = mbar_wait(o_full(u), (tg - 1) & 1, abort_flag, kTimeoutBase | 0x204, p.wait_ns);
             if (ok) {
                 tc_fence_after();
-                run_epilogue();
+                ok = run_epilogue();
             }
         }
-    }
-
-    else {
-        regs_decrease<L::control_regs>();
     }
     tc_fence_before();
     __syncthreads();

@@ -275,17 +275,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_after();
                 const int n0 = (sl0 + si) * BNO;
                 const uint32_t taddr = tmem + (uint32_t)(buf * BNO) + ((uint32_t)(32 * q) << 16);
-                // TMEM columns 64g .. 64g+31 arrive in va, 64g+32 .. 64g+63 in vb; the load of
-                // the next 32 columns is in flight while the current ones are converted
+                // TMEM columns 64g .. 64g+31 arrive in va, 64g+32 .. 64g+63 in vb (each load
+                // waited for in the same statement that issues it)
                 uint32_t va[32], vb[32];
-                tmem_ld32_issue(taddr, va);
                 const bool has_bias = bias_src != nullptr;
 #pragma unroll 1
                 for (int g = 0; g < BNO / 64; ++g) {
                     const uint32_t sb = stg + (uint32_t)((g & 1) * STG_TILE);
                     const float* bg = has_bias ? bias_src + n0 + 64 * g : nullptr;
-                    tmem_ld_wait32(va);
-                    tmem_ld32_issue(taddr + 64 * g + 32, vb);
+                    tmem_ld32_sync(taddr + 64 * g, va);
                     if (lane == 0) bulk_wait_read<1>();    // the store that last read this buffer is done with it
                     __syncwarp();
 #pragma unroll
@@ -302,8 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                pack_bf16(__uint_as_float(vc[4]) + b1.x, __uint_as_float(vc[5]) + b1.y),
                                pack_bf16(__uint_as_float(vc[6]) + b1.z, __uint_as_float(vc[7]) + b1.w));
                     }
-                    tmem_ld_wait32(vb);
-                    if (g + 1 < BNO / 64) tmem_ld32_issue(taddr + 64 * (g + 1), va);
+                    tmem_ld32_sync(taddr + 64 * g + 32, vb);
 #pragma unroll
                     for (int c = 4; c < 8; ++c) {
                         float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;

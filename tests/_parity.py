@@ -125,7 +125,7 @@ def report(case, name, m):
 
 
 def assert_close(case, name, got, ref, dtype, beyond_output_rounding=False):
-    """Check one output tensor against the oracle at the benchmark spec tolerances.
+    """Check one output tensor against the oracle at the tolerances of TOL (module docstring).
 
     With ``beyond_output_rounding`` (cases whose bf16-stored outputs reach
     magnitudes of 4 and more), the max-abs bound applies to the error beyond
