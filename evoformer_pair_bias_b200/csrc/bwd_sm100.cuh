@@ -85,10 +85,10 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 // Warps 12..15 drain dQ: each step's 128 x 32 fp32 product goes from TMEM into the
 // global fp32 accumulator with vector reductions, off the dS warps' path.
 // The two control warpgroups hand registers to the dS warpgroups:
-// 2*128*200 + 2*128*56 = 512*128, the launch's register pool.
+// 2*128*168 + 2*128*88 = 512*128, the launch's register pool (no spills at this split).
 constexpr int THREADS = 512;
 constexpr int LAUNCH_REGS = 128;
-constexpr uint32_t DS_REGS = 200, CONTROL_REGS = 56;
+constexpr uint32_t DS_REGS = 168, CONTROL_REGS = 88;
 static_assert((2 * DS_REGS + 2 * CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
 // TMEM columns: S^T, dP^T, two P^T buffers (bf16 pairs), dV, dK, dQ accumulators
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 384, TM_DK = 416, TM_DQ = 448, TM_COLS = 512;
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(dq_full, 1);
         mbar_init(dq_free, 4);                    // the dQ drain warps
         mbar_init(dkv_full, 1);
-        mbar_init(dkv_free, 8);
+        mbar_init(dkv_free, 4);                   // the drain warps
         for (int x = 0; x < 3; ++x) mbar_init(mma_done(x), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -385,11 +385,46 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x1A + role));
             }
         } else {
-            // ---------------------------------------------------------------- dQ drain warps
-            // dQ_i of step t (lanes = queries) into the fp32 accumulator, scaled by 1/sqrt(C).
+            // ---------------------------------------------------------------- drain warps
+            // dQ_i of step t (lanes = queries) into the fp32 accumulator, scaled by 1/sqrt(C);
+            // at the end of each row s, dK_j and dV_j (lanes = keys) into their bf16 outputs.
             const int quad = warp & 3;
             const int r = quad * 32 + lane;
+            const int j = j0 + r;
             const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+            auto drain_dkv = [&](int si) -> bool {
+                if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
+                tc_fence_after();
+                uint32_t vk[32], vv[32];
+                tmem_ld32_sync(lane_addr + TM_DK, vk);
+                tmem_ld32_sync(lane_addr + TM_DV, vv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dkv_free);
+                if (j < p.N) {
+                    __nv_bfloat16* dk = p.dk + p.gs.off(b, s_begin + si, j, h);
+                    __nv_bfloat16* dv = p.dv + p.gs.off(b, s_begin + si, j, h);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(vk[8 * q + 0]) * p.rs, __uint_as_float(vk[8 * q + 1]) * p.rs);
+                        w.y = pack_bf16(__uint_as_float(vk[8 * q + 2]) * p.rs, __uint_as_float(vk[8 * q + 3]) * p.rs);
+                        w.z = pack_bf16(__uint_as_float(vk[8 * q + 4]) * p.rs, __uint_as_float(vk[8 * q + 5]) * p.rs);
+                        w.w = pack_bf16(__uint_as_float(vk[8 * q + 6]) * p.rs, __uint_as_float(vk[8 * q + 7]) * p.rs);
+                        *reinterpret_cast<uint4*>(dk + 8 * q) = w;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(vv[8 * q + 0]), __uint_as_float(vv[8 * q + 1]));
+                        w.y = pack_bf16(__uint_as_float(vv[8 * q + 2]), __uint_as_float(vv[8 * q + 3]));
+                        w.z = pack_bf16(__uint_as_float(vv[8 * q + 4]), __uint_as_float(vv[8 * q + 5]));
+                        w.w = pack_bf16(__uint_as_float(vv[8 * q + 6]), __uint_as_float(vv[8 * q + 7]));
+                        *reinterpret_cast<uint4*>(dv + 8 * q) = w;
+                    }
+                }
+                return true;
+            };
             for (int t = 0; t < T; ++t) {
                 if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) break;
                 tc_fence_after();
@@ -410,6 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                      : "memory");
                     }
                 }
+                if (it == ni - 1 && !drain_dkv(si)) break;
             }
         }
     } else {
@@ -426,32 +462,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint64_t L2E2 = f2(p.bsc, p.bsc);
         bool ok = true;
 
-        auto drain_dkv = [&](int si) -> bool {   // dK (wg 0) / dV (wg 1) of row s: lanes = keys
-            if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
-            tc_fence_after();
-            uint32_t v[32];
-            tmem_ld32_sync(lane_addr + (wg == 0 ? TM_DK : TM_DV), v);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dkv_free);
-            if (jvalid) {
-                const float f = wg == 0 ? p.rs : 1.0f;
-                __nv_bfloat16* dst = (wg == 0 ? p.dk : p.dv) + p.gs.off(b, s_begin + si, j, h);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 w;
-                    w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * f, __uint_as_float(v[8 * q + 1]) * f);
-                    w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * f, __uint_as_float(v[8 * q + 3]) * f);
-                    w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * f, __uint_as_float(v[8 * q + 5]) * f);
-                    w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * f, __uint_as_float(v[8 * q + 7]) * f);
-                    *reinterpret_cast<uint4*>(dst + 8 * q) = w;
-                }
-            }
-            return true;
-        };
-
         for (int t = 0; t < T; ++t) {
-            const int si = t / ni, it = t - si * ni, st = t & 1;
+            const int st = t & 1;
             ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
             if (!ok) break;
             tc_fence_after();
@@ -530,15 +542,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(ds_full(st));
-
-            // At a row change the previous row's dK/dV are drained here, after this
-            // step's exponentials, so the MMAs that produce them overlap this step's work.
-            if (t > 0 && it == 0) {
-                ok = drain_dkv(si - 1);
-                if (!ok) break;
-            }
         }
-        if (ok) ok = drain_dkv(ns - 1);
         }
     }
 
@@ -791,7 +795,7 @@ inline cudaError_t launch_dbias(const CUtensorMap* m, const dbias::Params& dp, i
         cudaFuncAttributes fa{};
         return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : -1;
     }();
-    if (regs != dbias::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    if (regs != dbias::LAUNCH_REGS) return cudaErrorInvalidConfiguration;   // the setmaxnreg split assumes it
     {
         timing::Scope t(EVO_PHASE_BWD_DBIAS, stream);
         kern<<<grid, dbias::THREADS, dbias::SMEM_BYTES, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
