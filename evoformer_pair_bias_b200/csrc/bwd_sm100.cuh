@@ -79,17 +79,21 @@ constexpr int NBARS = 28;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-// Warps 0..7: two dS warpgroups (queries 0..63 / 64..127 of the tile); warp 8 TMA;
-// three MMA issuers, so that no single issuing thread serialises a step's 33
-// instructions: warp 9 S^T and dP^T of the next step, warp 10 dV and dK, warp 11 dQ.
-// Warps 12..15 drain dQ: each step's 128 x 32 fp32 product goes from TMEM into the
-// global fp32 accumulator with vector reductions, off the dS warps' path.
-// The two control warpgroups hand registers to the dS warpgroups:
-// 2*128*168 + 2*128*88 = 512*128, the launch's register pool (no spills at this split).
-constexpr int THREADS = 512;
-constexpr int LAUNCH_REGS = 128;
-constexpr uint32_t DS_REGS = 168, CONTROL_REGS = 88;
-static_assert((2 * DS_REGS + 2 * CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
+// Warps 0..15: four dS warpgroups, warpgroup w taking queries 32 w .. 32 w + 31 of the
+// tile (each dS warp's per-step chain of waits, loads, exponentials and stores is
+// mostly latency, which more warps per SM overlap); warp 16 TMA; three MMA issuers,
+// so that no single issuing thread serialises a step's 33 instructions: warp 17 S^T
+// and dP^T of the next step, warp 18 dV and dK, warp 19 dQ.  Warps 20..23 drain: each
+// step's 128 x 32 fp32 dQ goes from TMEM into the global fp32 accumulator with vector
+// reductions, and each row's dK and dV into their outputs, off the dS warps' path.
+// Registers: 4*128*96 + 128*56 + 128*40 = 768*80, the launch's register pool (no spills).
+constexpr int NWG = 4;                       // dS warpgroups
+constexpr int QW = BQ / NWG;                 // queries per dS warpgroup
+constexpr int DS_WARPS = 4 * NWG;
+constexpr int THREADS = 128 * NWG + 256;
+constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
+constexpr uint32_t DS_REGS = 96, CONTROL_REGS = 56, DRAIN_REGS = 40;
+static_assert((NWG * DS_REGS + CONTROL_REGS + DRAIN_REGS) * 128 <= LAUNCH_REGS * THREADS, "register split");
 // TMEM columns: S^T, dP^T, two P^T buffers (bf16 pairs), dV, dK, dQ accumulators
 constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_PT = 256, TM_DV = 384, TM_DK = 416, TM_DQ = 448, TM_COLS = 512;
 
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = 8, kMma = 9, kMmaKV = 10, kMmaQ = 11;
+    constexpr int kProducer = DS_WARPS, kMma = DS_WARPS + 1, kMmaKV = DS_WARPS + 2, kMmaQ = DS_WARPS + 3;
     const int j0 = blockIdx.x * BK;
     const int grp = blockIdx.y;
     const int b = blockIdx.z / p.H, h = blockIdx.z % p.H;
@@ -169,16 +173,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(kv_full(x), 1);
             mbar_init(kv_empty(x), 2);            // K and V read by the S^T / dP^T issuer and the dQ issuer
             mbar_init(x_full(x), 1);
-            mbar_init(x_empty(x), 1 + 8);         // the S^T / dP^T issuer and the dS warps (bias)
+            mbar_init(x_empty(x), 1 + DS_WARPS);  // the S^T / dP^T issuer and the dS warps (bias)
             mbar_init(pt_free(x), 1);
-            mbar_init(ds_full(x), 8);
+            mbar_init(ds_full(x), DS_WARPS);
         }
         for (int x = 0; x < Y_STAGES; ++x) {
             mbar_init(y_full(x), 1);
             mbar_init(y_empty(x), 2);             // the S^T / dP^T and the dV / dK issuers
         }
         mbar_init(sdp_full, 1);
-        mbar_init(sdp_free, 8);
+        mbar_init(sdp_free, DS_WARPS);
         mbar_init(ds_free, 2);                    // dK and dQ read the dS^T tile
         mbar_init(dq_full, 1);
         mbar_init(dq_free, 4);                    // the dQ drain warps
@@ -234,7 +238,75 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // setmaxnreg is warpgroup-wide: all four warps of a warpgroup execute the same
     // instruction, so each warpgroup changes its count before its warps' roles split.
-    if (warp >= 8) {
+    if (warp >= DS_WARPS + 4) {
+        regs_decrease<DRAIN_REGS>();
+        // ---------------------------------------------------------------- drain warps
+        // dQ_i of step t (lanes = queries) into the fp32 accumulator, scaled by 1/sqrt(C);
+        // at the end of each row s, dK_j and dV_j (lanes = keys) into their bf16 outputs.
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int j = j0 + r;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+        // 16 columns at a time (the drain warps run on 40 registers); a TMEM buffer is
+        // released once its last columns are in registers
+        auto store16 = [&](__nv_bfloat16* dst, const uint32_t* v, float f) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                uint4 w;
+                w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * f, __uint_as_float(v[8 * q + 1]) * f);
+                w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * f, __uint_as_float(v[8 * q + 3]) * f);
+                w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * f, __uint_as_float(v[8 * q + 5]) * f);
+                w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * f, __uint_as_float(v[8 * q + 7]) * f);
+                *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+            }
+        };
+        auto drain_dkv = [&](int si) -> bool {
+            if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
+            tc_fence_after();
+            const bool jv = j < p.N;
+            __nv_bfloat16* dk = p.dk + p.gs.off(b, s_begin + si, jv ? j : 0, h);
+            __nv_bfloat16* dv = p.dv + p.gs.off(b, s_begin + si, jv ? j : 0, h);
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {   // dK columns 0..15, 16..31, then dV's
+                uint32_t v[16];
+                tmem_ld16_sync(lane_addr + (part < 2 ? TM_DK : TM_DV) + (part & 1) * 16, v);
+                if (part == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(dkv_free);
+                }
+                if (jv) store16((part < 2 ? dk : dv) + (part & 1) * 16, v, part < 2 ? p.rs : 1.0f);
+            }
+            return true;
+        };
+        for (int t = 0; t < T; ++t) {
+            if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) break;
+            tc_fence_after();
+            const int si = t / ni, it = t - si * ni;
+            const int i = it * BQ + r, s = s_begin + si;
+            float* dst = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + (i < p.N ? i : 0)) * p.H + h) * HD;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[16];
+                tmem_ld16_sync(lane_addr + TM_DQ + hf * 16, v);
+                if (hf == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(dq_free);
+                }
+                if (i < p.N) {
+#pragma unroll
+                    for (int c = 0; c < 16; c += 4) {
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + hf * 16 + c),
+                                     "f"(__uint_as_float(v[c]) * p.rs), "f"(__uint_as_float(v[c + 1]) * p.rs),
+                                     "f"(__uint_as_float(v[c + 2]) * p.rs), "f"(__uint_as_float(v[c + 3]) * p.rs)
+                                     : "memory");
+                    }
+                }
+            }
+            if (it == ni - 1 && !drain_dkv(si)) break;
+        }
+    } else if (warp >= DS_WARPS) {
         regs_decrease<CONTROL_REGS>();
         if (warp == kProducer) {
             // ---------------------------------------------------------------- producer
@@ -292,7 +364,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int x = 0; x < Y_STAGES; ++x)
                     if (y_issued[x]) mbar_wait(y_full(x), (y_issued[x] - 1) & 1, &no_abort, kTimeoutBase | 0x06);
             }
-        } else if (warp == kMma || warp == kMmaKV || warp == kMmaQ) {
+        } else {
             // ---------------------------------------------------------------- MMA issuers
             const int role = warp - kMma;            // 0: S^T, dP^T   1: dV, dK   2: dQ
             if (lane == 0 && T > 0) {
@@ -384,75 +456,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 volatile int no_abort = 0;
                 mbar_wait(mma_done(role), 0, &no_abort, kTimeoutBase | (0x1A + role));
             }
-        } else {
-            // ---------------------------------------------------------------- drain warps
-            // dQ_i of step t (lanes = queries) into the fp32 accumulator, scaled by 1/sqrt(C);
-            // at the end of each row s, dK_j and dV_j (lanes = keys) into their bf16 outputs.
-            const int quad = warp & 3;
-            const int r = quad * 32 + lane;
-            const int j = j0 + r;
-            const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-            auto drain_dkv = [&](int si) -> bool {
-                if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
-                tc_fence_after();
-                uint32_t vk[32], vv[32];
-                tmem_ld32_sync(lane_addr + TM_DK, vk);
-                tmem_ld32_sync(lane_addr + TM_DV, vv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(dkv_free);
-                if (j < p.N) {
-                    __nv_bfloat16* dk = p.dk + p.gs.off(b, s_begin + si, j, h);
-                    __nv_bfloat16* dv = p.dv + p.gs.off(b, s_begin + si, j, h);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(vk[8 * q + 0]) * p.rs, __uint_as_float(vk[8 * q + 1]) * p.rs);
-                        w.y = pack_bf16(__uint_as_float(vk[8 * q + 2]) * p.rs, __uint_as_float(vk[8 * q + 3]) * p.rs);
-                        w.z = pack_bf16(__uint_as_float(vk[8 * q + 4]) * p.rs, __uint_as_float(vk[8 * q + 5]) * p.rs);
-                        w.w = pack_bf16(__uint_as_float(vk[8 * q + 6]) * p.rs, __uint_as_float(vk[8 * q + 7]) * p.rs);
-                        *reinterpret_cast<uint4*>(dk + 8 * q) = w;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(vv[8 * q + 0]), __uint_as_float(vv[8 * q + 1]));
-                        w.y = pack_bf16(__uint_as_float(vv[8 * q + 2]), __uint_as_float(vv[8 * q + 3]));
-                        w.z = pack_bf16(__uint_as_float(vv[8 * q + 4]), __uint_as_float(vv[8 * q + 5]));
-                        w.w = pack_bf16(__uint_as_float(vv[8 * q + 6]), __uint_as_float(vv[8 * q + 7]));
-                        *reinterpret_cast<uint4*>(dv + 8 * q) = w;
-                    }
-                }
-                return true;
-            };
-            for (int t = 0; t < T; ++t) {
-                if (!mbar_wait(dq_full, t & 1, abort_flag, kTimeoutBase | 0x21)) break;
-                tc_fence_after();
-                uint32_t v[32];
-                tmem_ld32_sync(lane_addr + TM_DQ, v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(dq_free);
-                const int si = t / ni, it = t - si * ni;
-                const int i = it * BQ + r, s = s_begin + si;
-                if (i < p.N) {
-                    float* dst = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + i) * p.H + h) * HD;
-#pragma unroll
-                    for (int c = 0; c < HD; c += 4) {
-                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c),
-                                     "f"(__uint_as_float(v[c]) * p.rs), "f"(__uint_as_float(v[c + 1]) * p.rs),
-                                     "f"(__uint_as_float(v[c + 2]) * p.rs), "f"(__uint_as_float(v[c + 3]) * p.rs)
-                                     : "memory");
-                    }
-                }
-                if (it == ni - 1 && !drain_dkv(si)) break;
-            }
         }
     } else {
         regs_increase<DS_REGS>();
         if (T > 0) {
         // ---------------------------------------------------------------- dS warpgroups
-        const int wg = warp >> 2;                // 0: queries 0..63 of the tile, 1: 64..127
+        const int wg = warp >> 2;                // queries QW wg .. QW wg + QW - 1 of the tile
         const int quad = warp & 3;
         const int r = quad * 32 + lane;          // key row within the tile = TMEM lane
         const int j = j0 + r;
@@ -467,16 +476,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = mbar_wait(sdp_full, t & 1, abort_flag, kTimeoutBase | 0x24);
             if (!ok) break;
             tc_fence_after();
-            // the whole bias row of this thread (64 queries) into registers at once, so the
-            // stage of ring X is released early
+            // this thread's bias row for the warpgroup's 32 queries (64-query box wg / 2,
+            // 16-byte chunks 4 (wg % 2) .. + 3) into registers at once, so the stage of ring X
+            // is released early
             const int xs = t % X_STAGES;
             ok = mbar_wait(x_full(xs), (t / X_STAGES) & 1, abort_flag, kTimeoutBase | 0x25);
-            uint32_t bw[32];
+            uint32_t bw[QW / 2];
             if (HAS_BIAS) {
-                const uint8_t* bt_ptr = gbase + OFF_X + xs * XB + X_BT + wg * BT_BOX + r * 128;
+                const uint8_t* bt_ptr = gbase + OFF_X + xs * XB + X_BT + (wg >> 1) * BT_BOX + r * 128;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(bt_ptr + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4));
+                for (int q = 0; q < QW / 8; ++q) {
+                    const uint32_t ch = (uint32_t)((wg & 1) * 4 + q);
+                    const uint4 w = *reinterpret_cast<const uint4*>(bt_ptr + ((ch ^ (uint32_t)(r & 7)) << 4));
                     bw[4 * q] = w.x; bw[4 * q + 1] = w.y; bw[4 * q + 2] = w.z; bw[4 * q + 3] = w.w;
                 }
             }
@@ -489,17 +500,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (ok && t >= 2) ok = mbar_wait(pt_free(pb), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t ts = lane_addr + TM_ST + wg * 64, td = lane_addr + TM_DPT + wg * 64;
-            const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * 32;
+            const uint32_t ts = lane_addr + TM_ST + wg * QW, td = lane_addr + TM_DPT + wg * QW;
+            const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * (QW / 2);
             // S^T and dP^T 16 queries at a time (v[0,16): S^T columns, v[16,32): dP^T columns).
             // P = exp2(S^T * sc2 + bias * bsc) (S^T already holds -lse and the mask),
             // dS = P * dP^T (dP^T already holds -D); two columns per op
-            uint32_t dk2[32];
+            uint32_t dk2[QW / 2];
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
+            for (int hf = 0; hf < QW / 16; ++hf) {
                 uint32_t v[32];
-                tmem_ld16x2_sync(ts + qd * 16, td + qd * 16, v);
-                if (qd == 3) {                   // every S^T / dP^T column of this step is in registers
+                tmem_ld16x2_sync(ts + hf * 16, td + hf * 16, v);
+                if (hf == QW / 16 - 1) {         // every S^T / dP^T column of this step is in registers
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(sdp_free);
@@ -510,11 +521,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2) {                // 8 columns (one bias chunk) at a time
-                    const int ch = qd * 2 + q2;
+                    const int ch = hf * 2 + q2;
                     uint32_t pk4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int c = q2 * 8 + 2 * e;             // column within the quarter
+                        const int c = q2 * 8 + 2 * e;             // column within the 16
                         uint64_t y2 = fmul2(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), SC2);
                         if (HAS_BIAS) y2 = ffma2(bf16x2_to_f2(bw[ch * 4 + e]), L2E2, y2);
                         const float p0 = ex2(f2lo(y2)), p1 = ex2(f2hi(y2));
@@ -529,10 +540,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             if (t > 0) ok = mbar_wait(ds_free, (t - 1) & 1, abort_flag, kTimeoutBase | 0x27);
             if (!ok) break;
-            const uint32_t ds_row = base + OFF_DS + wg * BT_BOX + r * 128;
+            const uint32_t ds_row = base + OFF_DS + (wg >> 1) * BT_BOX + r * 128;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint32_t addr = ds_row + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4);
+            for (int q = 0; q < QW / 8; ++q) {
+                const uint32_t addr = ds_row + ((((uint32_t)((wg & 1) * 4 + q)) ^ (uint32_t)(r & 7)) << 4);
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk2[4 * q]),
                              "r"(dk2[4 * q + 1]), "r"(dk2[4 * q + 2]), "r"(dk2[4 * q + 3])
                              : "memory");
