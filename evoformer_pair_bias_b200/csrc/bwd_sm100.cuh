@@ -26,9 +26,10 @@
 //                    dS^T = P^T (dP^T - D_i)
 //                    dV_j += P^T dOa_hi_i  dK_j += dS^T Q_i         (TMEM)
 //                    dQ_i  = dS K_j  -> fp32 atomic add into the accumulator
-//                  The dS^T smem tile and the P^T TMEM tile are double-buffered
-//                  by step parity, so the dS warps write step t while the MMAs of
-//                  step t-1 still read the other buffer.
+//                  The P^T TMEM tile is double-buffered by step parity, so the dS
+//                  warps write step t while dV of step t-1 still reads the other
+//                  buffer; the dS^T tile in shared memory is single-buffered (dK and
+//                  dQ of step t-1 finish before the dS warps store step t's).
 //   dbias          d_pair_bias, summed over the rows s on chip (dbias_sm100.cuh):
 //                  one partial slab per row group, plain stores.
 //   bwd_post       one launch: dq = bf16(accumulator); d_pair_bias = sum over
@@ -74,7 +75,7 @@ constexpr int OFF_ONES = OFF_DS + DS_BYTES;        // A operand: columns 0 and 1
 constexpr int OFF_RROW = OFF_ONES + CONST_BYTES;   // B operand: columns k = 0, 8 equal to r1, r2 (sum sqrt(C))
 constexpr int OFF_BAR = OFF_RROW + CONST_BYTES;
 // kv_full[2] kv_empty[2] x_full[2] x_empty[2] y_full[3] y_empty[3] sdp_full sdp_free ds_full[2]
-// pt_free[2] ds_free dq_full dq_free dkv_full dkv_free mma_done[3]
+// (18, 19 unused) ds_free dq_full dq_free dkv_full dkv_free mma_done[3]
 constexpr int NBARS = 28;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -160,7 +161,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ds_full[t & 1]: dS^T of step t in shared memory and P^T in TMEM (one barrier per step
     // parity, because two issuers consume it and the dS warps may run a step ahead of one)
     auto ds_full = [&](int x) { return bar0 + 8u * (16 + x); };
-    auto pt_free = [&](int x) { return bar0 + 8u * (18 + x); };
     const uint32_t ds_free = bar0 + 8u * 20;
     const uint32_t dq_full = bar0 + 8u * 21, dq_free = bar0 + 8u * 22;
     const uint32_t dkv_full = bar0 + 8u * 23, dkv_free = bar0 + 8u * 24;
@@ -174,7 +174,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(kv_empty(x), 2);            // K and V read by the S^T / dP^T issuer and the dQ issuer
             mbar_init(x_full(x), 1);
             mbar_init(x_empty(x), 1 + DS_WARPS);  // the S^T / dP^T issuer and the dS warps (bias)
-            mbar_init(pt_free(x), 1);
             mbar_init(ds_full(x), DS_WARPS);
         }
         for (int x = 0; x < Y_STAGES; ++x) {
@@ -424,7 +423,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                             mma_ts(tmem + TM_DV, tmem + TM_PT + pb * 64 + kk * 8,
                                    smem_desc(yb + Y_DOH + kk * 1024, TILE_BYTES, 512, kSw64), ID_KV,
                                    (it > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(pt_free(pb));
 #pragma unroll
                         for (int kk = 0; kk < BQ / 16; ++kk) {
                             const uint32_t a = ds + (kk >> 2) * BT_BOX + (kk & 3) * 32;
@@ -496,10 +494,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(x_empty(xs));           // bias tile of this stage consumed
-            const int pb = t & 1;                // P^T buffer of this step
-            if (ok && t >= 2) ok = mbar_wait(pt_free(pb), ((t >> 1) - 1) & 1, abort_flag, kTimeoutBase | 0x26);
+            // P^T buffer of this step.  Its last reader, dV of step t - 2, is complete: the dS
+            // warps waited for ds_free of step t - 2 before their dS stores of step t - 1, and
+            // that barrier's dV/dK commit covers every earlier MMA of the same issuer.
+            const int pb = t & 1;
             if (!ok) break;
-            tc_fence_after();
             const uint32_t ts = lane_addr + TM_ST + wg * QW, td = lane_addr + TM_DPT + wg * QW;
             const uint32_t pt_addr = lane_addr + TM_PT + pb * 64 + wg * (QW / 2);
             // S^T and dP^T 16 queries at a time (v[0,16): S^T columns, v[16,32): dP^T columns).
