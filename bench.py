@@ -217,10 +217,21 @@ def flops(w):
 # profiles/ summary, together with the SHA-256 of the kernel's source file at
 # that time.  Reported only while the source is unchanged.
 TRAFFIC = {
-    ("bwd_main", "msa_row_256"): (175.89e6, "bwd_sm100.cuh",
-                                "306a34cb2780647122fa8ce3fdd3177c53d14c7407588961ce6c6f6038fb266b"),
-    ("fwd_main", "msa_row_256"): (75.56e6, "fwd_sm100.cuh",
-                                "ccbab72209fc7ef6501f95e939be78536073bbefc7e9c99387ac6f81f106e9be"),
+    # DRAM bytes (read + write) per launch from one ncu pass over the full workload, with the
+    # sha256 of the kernel's source when they were taken (a changed source reports null)
+    ("bwd_main", "tri_long_1536"): (6937.8e6, "bwd_sm100.cuh",
+                                    "0e8e39c9fb13414ee55c6338b02c7ccb128281295e0a25df7a9a0cc7f381115e"),
+    ("fwd_main", "tri_long_1536"): (7770.0e6, "fwd_sm100.cuh",
+                                    "c38acf5f88b0678853aae653f09d843bfb4ef6cf985e72c21e645dfe936c403c"),
+    ("bwd_dbias", "tri_long_1536"): (9350.7e6, "dbias_sm100.cuh",
+                                     "b6748d47e784d489cf281e46c2893b09f326d4883b1d133dd5ac626b55c9e871"),
+    # one multi-pass capture at MSA-row N = 384 (cold caches)
+    ("bwd_main", "msa_row_384"): (1087.0e6, "bwd_sm100.cuh",
+                                  "0e8e39c9fb13414ee55c6338b02c7ccb128281295e0a25df7a9a0cc7f381115e"),
+    ("fwd_main", "msa_row_384"): (1184.8e6, "fwd_sm100.cuh",
+                                  "c38acf5f88b0678853aae653f09d843bfb4ef6cf985e72c21e645dfe936c403c"),
+    ("bwd_dbias", "msa_row_384"): (522.7e6, "dbias_sm100.cuh",
+                                   "b6748d47e784d489cf281e46c2893b09f326d4883b1d133dd5ac626b55c9e871"),
     # one launch after three warm-up steps; output bytes still held in the 126 MB L2 when the
     # captured launch ends are written back later and are not in the count
     ("qkvg", "msa_proj_256"): (27.29e6, "proj_sm100.cuh",
