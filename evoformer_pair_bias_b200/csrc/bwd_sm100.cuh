@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* gbase = smem_raw + (base - raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kProducer = DS_WARPS, kMma = DS_WARPS + 1, kMmaKV = DS_WARPS + 2, kMmaQ = DS_WARPS + 3;
+    constexpr int kProducer = DS_WARPS, kMma = DS_WARPS + 1;   // issuers: kMma (S^T, dP^T), + 1 (dV, dK), + 2 (dQ)
     const int j0 = blockIdx.x * BK;
     const int grp = blockIdx.y;
     const int b = blockIdx.z / p.H, h = blockIdx.z % p.H;
