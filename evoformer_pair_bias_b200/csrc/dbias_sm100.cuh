@@ -81,9 +81,11 @@ static_assert((NWG * DS_REGS + CONTROL_REGS) * 128 <= LAUNCH_REGS * THREADS, "re
 // TMEM: buffer x holds S^T at 256 x and dP^T at 256 x + 128
 constexpr uint32_t TM_COLS = 512;
 // Every POLY_EVERY-th pair of exponentials runs on the FMA pipe (exp2_poly2)
-// instead of the MUFU unit; 0 keeps all of them on MUFU.
+// instead of the MUFU unit; 0 keeps all of them on MUFU.  The kernel's dS warps are
+// bound by instruction issue, not by MUFU: every 2nd, 3rd, 4th or 6th pair on the FMA
+// pipe measured 19, 3, 3 and 2 % slower than none.
 #ifndef EVO_DBIAS_POLY_EVERY
-#define EVO_DBIAS_POLY_EVERY 3
+#define EVO_DBIAS_POLY_EVERY 0
 #endif
 constexpr int POLY_EVERY = EVO_DBIAS_POLY_EVERY;
 
