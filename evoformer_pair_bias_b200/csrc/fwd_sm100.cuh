@@ -23,31 +23,30 @@
 // matches this pass's log-sum-exp.  The softmax threads only scale, take
 // maxima and exponentiate.
 //
-// Warp roles (128*NSUB + 128 threads; the last warpgroup gives up registers
-// to the softmax warpgroups with setmaxnreg):
+// Warp roles (128*NSUB + 256 threads; the two control warpgroups give up
+// registers to the softmax warpgroups with setmaxnreg, one site per warpgroup):
 //   warps 0 .. 4*NSUB-1   one 4-warp softmax group per row s (see below)
-//   warp 4*NSUB           TMA producer: per item Q (double-buffered by item
-//            parity), then per key tile K and the mask row (per row s) and
-//            the pair-bias tile into a 2-stage ring ("A") that runs across
-//            items.  A stage of ring A is released as soon as both S MMAs and
-//            both row groups' bias reads are done, so the next tiles' loads
-//            start early instead of waiting for the P V products.
+//   warp 4*NSUB           TMA producer: per item Q and the gate tiles (each
+//            double-buffered by item parity), then per key tile K and the mask
+//            row (per row s) and the pair-bias tile into a 2-stage ring ("A")
+//            that runs across items, released by the S MMAs' commits (K, mask
+//            and bias are MMA operands only)
+//   warps 4*NSUB+1+u      S issuer of row group u (one lane; the first also
+//            owns TMEM): S_u = Q K^T + (r1 e_0 + r2 e_8) m^T + (r1 I) bias,
+//            2 + 1 + 8 MMAs of M = 128, N = 128
 //   warp 4*NSUB+NSUB+1    TMA producer of V (per row s) into its own 2-stage
-//            ring ("B"), released when the P V products of the tile are done.
-//   warps 4*NSUB+1+u      MMA issuer of row group u (one lane; the first also
-//            owns TMEM): S_u as above (M=128, N=128), then O_u += P_u V_u
-//            (M=128, N=32, K=128, P read from TMEM).  The S MMA of the next
-//            tile is issued before the PV of the current one, so it overlaps
-//            the softmax; one issuer per row group keeps the groups' pipelines
-//            independent of each other.
-//   softmax: thread = query row.  Load S from TMEM and add the pair-bias
-//            row, online max and sum in fp32 with a lazy rescale (the
-//            running max moves only when a tile's max exceeds it by more than
-//            2^8), P (bf16) back to TMEM, and at the end of the item
-//            out = sigmoid(g) * O / l, lse = log(l) + max.  The two row
-//            groups take turns on the exponentials (the MUFU unit is the
-//            scarce resource at C = 32): each group's loads, bias adds and
-//            maxima overlap the other group's exponentials.
+//            ring ("B"), released when the P V products of the tile are done
+//   warps 4*NSUB+NSUB+2+u P V issuer of row group u: O_u += P_u V_u (M = 128,
+//            N = 32, K = 128, P read from TMEM), O double-buffered by item
+//   softmax: thread = query row.  Load S from TMEM, online max and sum in fp32
+//            with a lazy rescale (the running max moves only when a tile's
+//            max exceeds it by more than 2^8), P (bf16) back to TMEM, and at
+//            the end of the item out = sigmoid(g) * O / l (the gate read from
+//            its TMA-loaded tile; out's bf16 rounding residual written too when
+//            asked), lse = log(l) + max.  The two row groups take turns on the
+//            exponentials (the MUFU unit is the scarce resource at C = 32):
+//            each group's loads and maxima overlap the other group's
+//            exponentials.
 // TMEM per row s: S 128 columns, P 64 columns (bf16 pairs), O 2 x 32 columns.
 #pragma once
 

@@ -165,3 +165,38 @@ def test_pending_wait_sums_gathered_parts_in_place():
     assert got is mine and work.waited == 1
     assert np.array_equal(got.cpu().numpy(), oracle.ordered_sum_f32(gathered.cpu().numpy()))
     assert pending.wait() is mine and work.waited == 1  # a second wait() does nothing more
+
+
+def test_pair_shards_on_one_gpu_match_the_oracle():
+    """The pair-sharded triangle attentions (pair_shards) with a single rank, on the GPU kernels:
+    around the starting node in place, around the ending node through the transposed view of the
+    (here whole) column block, forward and backward; each output against the oracle run on the
+    pair (ending node: on the explicitly transposed pair)."""
+    from evoformer_pair_bias_b200 import pair_shards
+    N = 136
+    w = Workload("pair_gpu", 1, N, N, 2, 32, "bf16", "tri_start", 1.0, "frac:0.1", 4711)
+    inp = workload_inputs(w)
+    d = to_gpu(inp)
+    x = {k: f64(v) for k, v in inp.items()}
+    T = lambda a: np.ascontiguousarray(np.swapaxes(a, 1, 2))            # noqa: E731
+    # starting node: rows s = i, keys j
+    out_s, lse_s = pair_shards.tri_start_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"])
+    g_s = pair_shards.tri_start_bwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], out_s, lse_s,
+                                    d["dout"])
+    torch.cuda.synchronize()
+    ref_out, _ = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"])
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["mask_bias"], x["pair_bias"], x["dout"])
+    assert_close("pair_gpu/start", "out", f64(out_s), ref_out, "bf16")
+    for n in ("dq", "dk", "dv", "dg", "d_pair_bias"):
+        assert_close("pair_gpu/start", n, f64(g_s[n]), ref[n], "bf16")
+    # ending node: rows s = j, keys i, on the row-sharded (here whole) pair
+    out_e, lse_e, saved = pair_shards.tri_end_fwd(d["q"], d["k"], d["v"], d["g"], d["mask_bias"], d["pair_bias"], N)
+    g_e = pair_shards.tri_end_bwd(saved, d["mask_bias"], d["pair_bias"], lse_e, d["dout"], N)
+    torch.cuda.synchronize()
+    xt = {n: T(x[n]) for n in ("q", "k", "v", "g", "dout")}
+    ref_out_e, _ = oracle.forward(xt["q"], xt["k"], xt["v"], xt["g"], x["mask_bias"], x["pair_bias"])
+    ref_e = oracle.backward(xt["q"], xt["k"], xt["v"], xt["g"], x["mask_bias"], x["pair_bias"], xt["dout"])
+    assert_close("pair_gpu/end", "out", f64(out_e), T(ref_out_e), "bf16")
+    for n in ("dq", "dk", "dv", "dg"):
+        assert_close("pair_gpu/end", n, f64(g_e[n]), T(ref_e[n]), "bf16")
+    assert_close("pair_gpu/end", "d_pair_bias", f64(g_e["d_pair_bias"]), ref_e["d_pair_bias"], "bf16")
