@@ -242,6 +242,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ---------------------------------------------------------------- drain warps
         // dQ_i of step t (lanes = queries) into the fp32 accumulator, scaled by 1/sqrt(C);
         // at the end of each row s, dK_j and dV_j (lanes = keys) into their bf16 outputs.
+        // The reductions are the kernel's heaviest traffic (one per element of dQ per key
+        // tile): a 16-byte reduction that covers half of a 32-byte sector costs the L2 about
+        // as much as a whole sector, so neighbouring lanes first trade halves (see below).
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const int j = j0 + r;
@@ -283,7 +286,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const int si = t / ni, it = t - si * ni;
             const int i = it * BQ + r, s = s_begin + si;
-            float* dst = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + (i < p.N ? i : 0)) * p.H + h) * HD;
+            const bool odd = (lane & 1) != 0;
+            const int i_even = i & ~1;
+            const int64_t row_stride = (int64_t)p.H * HD;
+            float* dst_even = p.dq_acc + ((((int64_t)b * p.S + s) * p.N + (i_even < p.N ? i_even : 0)) * p.H + h) * HD;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t v[16];
@@ -293,14 +299,27 @@ __global__ void __launch_bounds__(THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(dq_free);
                 }
-                if (i < p.N) {
+                // lanes 2m and 2m+1 hold query rows 2m and 2m+1; they trade half of each 32-byte
+                // sector of their rows, so that each vector reduction of the warp covers whole
+                // sectors of 16 rows: the even lane reduces low halves, the odd lane high halves
 #pragma unroll
-                    for (int c = 0; c < 16; c += 4) {
-                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + hf * 16 + c),
-                                     "f"(__uint_as_float(v[c]) * p.rs), "f"(__uint_as_float(v[c + 1]) * p.rs),
-                                     "f"(__uint_as_float(v[c + 2]) * p.rs), "f"(__uint_as_float(v[c + 3]) * p.rs)
-                                     : "memory");
+                for (int k = 0; k < 2; ++k) {
+                    float lo[4], hi[4], recv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        lo[e] = __uint_as_float(v[8 * k + e]) * p.rs;
+                        hi[e] = __uint_as_float(v[8 * k + 4 + e]) * p.rs;
+                        recv[e] = __shfl_xor_sync(0xffffffffu, odd ? lo[e] : hi[e], 1);
                     }
+                    const int col = hf * 16 + 8 * k + (odd ? 4 : 0);
+                    if (i_even < p.N)        // even row: its low half from the even lane, high half from the odd
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst_even + col),
+                                     "f"(odd ? recv[0] : lo[0]), "f"(odd ? recv[1] : lo[1]),
+                                     "f"(odd ? recv[2] : lo[2]), "f"(odd ? recv[3] : lo[3]) : "memory");
+                    if (i_even + 1 < p.N)    // odd row: its low half from the even lane, high half from the odd
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst_even + row_stride + col),
+                                     "f"(odd ? hi[0] : recv[0]), "f"(odd ? hi[1] : recv[1]),
+                                     "f"(odd ? hi[2] : recv[2]), "f"(odd ? hi[3] : recv[3]) : "memory");
                 }
             }
             if (it == ni - 1 && !drain_dkv(si)) break;
