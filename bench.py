@@ -219,15 +219,18 @@ def flops(w):
 TRAFFIC = {
     # DRAM bytes (read + write) per launch from one ncu pass over the full workload, with the
     # sha256 of the kernel's source when they were taken (a changed source reports null)
-    ("bwd_main", "tri_long_1536"): (6827.2e6, "bwd_sm100.cuh",
-                                    "c6acc27d9e916f877facaa8e6d28ffafa9b79563a80373114ce09b211303cbaa"),
-    ("fwd_main", "tri_long_1536"): (7951.3e6, "fwd_sm100.cuh",
-                                    "c38acf5f88b0678853aae653f09d843bfb4ef6cf985e72c21e645dfe936c403c"),
-    ("bwd_dbias", "tri_long_1536"): (12528.5e6, "dbias_sm100.cuh",
+    ("bwd_main", "tri_long_1536"): (7614.5e6, "bwd_sm100.cuh",
+                                    "cbee8e9cb9739b0d1c9ead30f47db35bd2ac92c43353aec9492a19e600a9f209"),
+    ("fwd_main", "tri_long_1536"): (7923.4e6, "fwd_sm100.cuh",
+                                    "0844cfc9469e937079959e8e5b52355071237e983dc19cdda1dc7ca4e74ba28f"),
+    ("bwd_dbias", "tri_long_1536"): (10434.4e6, "dbias_sm100.cuh",
                                      "da55b81462a57b720508e9c6dc5514fa6746503d42e82561eba31d04d4341b06"),
-    # one multi-pass capture at MSA-row N = 384 (cold caches)
-    ("fwd_main", "msa_row_384"): (1184.8e6, "fwd_sm100.cuh",
-                                  "c38acf5f88b0678853aae653f09d843bfb4ef6cf985e72c21e645dfe936c403c"),
+    ("fwd_main", "msa_row_384"): (1181.9e6, "fwd_sm100.cuh",
+                                  "0844cfc9469e937079959e8e5b52355071237e983dc19cdda1dc7ca4e74ba28f"),
+    ("bwd_main", "msa_row_384"): (1081.0e6, "bwd_sm100.cuh",
+                                  "cbee8e9cb9739b0d1c9ead30f47db35bd2ac92c43353aec9492a19e600a9f209"),
+    ("bwd_dbias", "msa_row_384"): (519.0e6, "dbias_sm100.cuh",
+                                   "da55b81462a57b720508e9c6dc5514fa6746503d42e82561eba31d04d4341b06"),
     # one pass after three warm-up steps; output bytes still held in the 126 MB L2 when the
     # captured launch ends are written back later and are not in the count
     ("qkvg", "msa_proj_256"): (24.35e6, "proj_sm100.cuh",
