@@ -493,14 +493,11 @@ __global__ void __launch_bounds__(Layout<NSUB>::threads, 1)
                     uint32_t ov[4], lv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        // out = O / (l * (1 + exp(-g))): the backward's D = sum(dout * out)
-                        // feeds a cancellation, so the gate is computed accurately
-                        // (exp on the FMA pipe, relative error < 8e-5; arguments
-                        // clamped to the exponent range, exp(-g) <= 2^126).
-                        const uint64_t ng = f2(fminf(-EVO_LOG2E * bf16lo(gv[e]), 126.0f),
-                                               fminf(-EVO_LOG2E * bf16hi(gv[e]), 126.0f));
-                        const uint64_t eg = exp2_poly2(ng);
-                        const float e0 = f2lo(eg), e1 = f2hi(eg);
+                        // out = O / (l * (1 + exp(-g))), exp(-g) from the MUFU unit (a few ulp:
+                        // the backward's D = sum(dout * out) feeds a cancellation, so the gate is
+                        // taken in full fp32; arguments clamped to the exponent range)
+                        const float e0 = ex2(fminf(-EVO_LOG2E * bf16lo(gv[e]), 126.0f));
+                        const float e1 = ex2(fminf(-EVO_LOG2E * bf16hi(gv[e]), 126.0f));
                         const float o0 = __fdividef(__uint_as_float(o[q * 8 + 2 * e]), epi.l * (1.0f + e0));
                         const float o1 = __fdividef(__uint_as_float(o[q * 8 + 2 * e + 1]), epi.l * (1.0f + e1));
                         ov[e] = pack_bf16(o0, o1);
