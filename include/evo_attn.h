@@ -326,9 +326,11 @@ uint64_t evo_attn_set_wait_limit_ns(uint64_t ns);
 
 /*
  * y[i] = 2^x[i] for n fp32 values (device pointers, 4-byte aligned), computed
- * by the FMA-pipe exponential the attention kernels use in place of the MUFU
- * unit for part of their exponentials: a cubic in the fraction after a
- * round-to-nearest split of x, relative error below 8e-5 for -125 <= x <= 126;
+ * by the FMA-pipe exponential that the attention kernels can take in place of
+ * the MUFU unit for a share of their exponentials (build switches
+ * EVO_FWD_POLY_EVERY and EVO_DBIAS_POLY_EVERY, off by default): a cubic in the
+ * fraction after a round-to-nearest split of x, relative error below 8e-5 for
+ * -125 <= x <= 126;
  * arguments below -125 give 2^-125.  Exported so that the device function
  * itself can be checked against 2^x on the GPU.  Returns EVO_ERR_INVALID_ARG
  * for n < 0 or a null pointer with n > 0.
