@@ -249,35 +249,45 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int r = quad * 32 + lane;
         const int j = j0 + r;
         const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-        // 16 columns at a time (the drain warps run on 40 registers); a TMEM buffer is
-        // released once its last columns are in registers
-        auto store16 = [&](__nv_bfloat16* dst, const uint32_t* v, float f) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                uint4 w;
-                w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * f, __uint_as_float(v[8 * q + 1]) * f);
-                w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * f, __uint_as_float(v[8 * q + 3]) * f);
-                w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * f, __uint_as_float(v[8 * q + 5]) * f);
-                w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * f, __uint_as_float(v[8 * q + 7]) * f);
-                *reinterpret_cast<uint4*>(dst + 8 * q) = w;
-            }
-        };
+        // dK / dV rows 16 columns (32 bytes) at a time, 8 columns per TMEM load (the drain warps
+        // run on 40 registers; the accumulators are released once their last columns are in
+        // registers); lanes 2m, 2m+1 (key rows 2m, 2m+1) trade halves, so each store of the
+        // warp writes whole 32-byte sectors of 16 rows
         auto drain_dkv = [&](int si) -> bool {
             if (!mbar_wait(dkv_full, si & 1, abort_flag, kTimeoutBase | 0x22)) return false;
             tc_fence_after();
-            const bool jv = j < p.N;
-            __nv_bfloat16* dk = p.dk + p.gs.off(b, s_begin + si, jv ? j : 0, h);
-            __nv_bfloat16* dv = p.dv + p.gs.off(b, s_begin + si, jv ? j : 0, h);
+            const bool odd = (lane & 1) != 0;
+            const int j_even = j & ~1;
+            const bool ok_e = j_even < p.N, ok_o = j_even + 1 < p.N;
+            const int64_t rs_n = p.gs.n;
 #pragma unroll
             for (int part = 0; part < 4; ++part) {   // dK columns 0..15, 16..31, then dV's
-                uint32_t v[16];
-                tmem_ld16_sync(lane_addr + (part < 2 ? TM_DK : TM_DV) + (part & 1) * 16, v);
+                const float f = part < 2 ? p.rs : 1.0f;
+                uint32_t w[2][4];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t v[8];
+                    tmem_ld8_sync(lane_addr + (part < 2 ? TM_DK : TM_DV) + (part & 1) * 16 + 8 * q, v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        w[q][e] = pack_bf16(__uint_as_float(v[2 * e]) * f, __uint_as_float(v[2 * e + 1]) * f);
+                }
                 if (part == 3) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(dkv_free);
                 }
-                if (jv) store16((part < 2 ? dk : dv) + (part & 1) * 16, v, part < 2 ? p.rs : 1.0f);
+                uint32_t rcv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) rcv[e] = __shfl_xor_sync(0xffffffffu, odd ? w[0][e] : w[1][e], 1);
+                __nv_bfloat16* row_even = (part < 2 ? p.dk : p.dv) + p.gs.off(b, s_begin + si, ok_e ? j_even : 0, h) +
+                                          (part & 1) * 16 + (odd ? 8 : 0);
+                if (ok_e)                            // even row: low half from the even lane, high from the odd
+                    *reinterpret_cast<uint4*>(row_even) = odd ? make_uint4(rcv[0], rcv[1], rcv[2], rcv[3])
+                                                              : make_uint4(w[0][0], w[0][1], w[0][2], w[0][3]);
+                if (ok_o)                            // odd row
+                    *reinterpret_cast<uint4*>(row_even + rs_n) = odd ? make_uint4(w[1][0], w[1][1], w[1][2], w[1][3])
+                                                                     : make_uint4(rcv[0], rcv[1], rcv[2], rcv[3]);
             }
             return true;
         };
